@@ -1,0 +1,54 @@
+"""CPU oracle for the draft-tree hot path.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
+baseline / reference legs of ``bench.py`` may import, call or execute anything
+in this package. The product library (``speculative_decoding_draft_07_b200``)
+never does, and this package never imports the product library: the two share
+no code. Inputs come from ``workloads`` (seeded generators only).
+
+Everything here is a plain, slow, float64 restatement of what the three source
+pages define, written step by step in their order and notation:
+
+* ``pctree.pct_tree_build``   -- Parent-Conditioned Drafting Tree (PCTree
+  article on qiita, section on the chain draft's weakness and the tree that
+  replaces it): per-parent scores z_d(p) = L_d + Markov(p), log-softmax over
+  the vocabulary, local top-k per parent, path score s(c) = sum log pi(v|u),
+  per-depth pruning to a beam, global top-N.
+* ``caddtree.cadd_tree_grow`` -- Cost-Aware Diffusion Draft Trees (gist.science
+  summary, technical summary, "Method: CaDDTree"): best-first growth by prefix
+  probability, greedy stop at the first non-positive marginal gain of
+  (1 + Phi(T)) / (C_d + C_v(n; l)).
+* ``verify.tree_verify_accept`` -- DSpark explainer (xiaohu-jiedu), section on
+  one round from drafting to confirmation: greedy argmax per node, accept the
+  longest matching root path, append the target's own token.
+* ``verify.tree_ancestor_mask`` -- the self-plus-ancestors mask used for tree
+  attention in the verification forward.
+
+Parity status of each function (what pins it, other than itself, is in
+``tests/test_oracle_*.py``):
+
+* ``pct_tree_build``: pinned by brute-force enumeration of every path (k = V,
+  unbounded beam), by the DSpark greedy chain (k = 1, N = B), by agreement with
+  the best-first tree when the Markov term is zero, and by a hand-derived finite
+  beam example. For larger finite k and beam, where the beam boundary itself is
+  only defined by the algorithm, the result is "parity unpinned" beyond that
+  hand example and the structural invariants the tests check.
+* ``cadd_tree_grow``: pinned by brute force (the top prefix-probability nodes
+  for every n), by an exhaustive scan of the throughput objective over n, by a
+  closed form on uniform marginals, and by Monte Carlo acceptance.
+* ``tree_verify_accept``: pinned by the pages' worked round (4 accepted drafts
+  plus 1 correction) and by planted paths.
+* ``tree_ancestor_mask``: pinned by an independent transitive closure of the
+  parent relation.
+"""
+from .numerics import decode_bf16, to_f64, row_log_softmax
+from .pctree import pct_tree_build, PCTreeResult
+from .caddtree import cadd_tree_grow, CaddResult, cadd_cost
+from .verify import tree_verify_accept, tree_ancestor_mask, VerifyResult
+
+__all__ = [
+    "decode_bf16", "to_f64", "row_log_softmax",
+    "pct_tree_build", "PCTreeResult",
+    "cadd_tree_grow", "CaddResult", "cadd_cost",
+    "tree_verify_accept", "tree_ancestor_mask", "VerifyResult",
+]

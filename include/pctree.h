@@ -1,0 +1,230 @@
+/*
+ * pctree.h -- C ABI of the draft-tree hot path (libpctree.so, sm_100a).
+ *
+ * One round of tree-based speculative decoding on one GPU:
+ *   pct_tree_build      parent-conditioned drafting tree (PCTree)
+ *   cadd_tree_grow      cost-aware best-first tree (CaDDTree)
+ *   tree_ancestor_mask  self-plus-ancestor bitmask for tree attention
+ *   tree_verify_accept  greedy verification: argmax, accept walk, correction
+ *   pct_score_parents   one depth of PCTree's batched parent scoring
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every data pointer is DEVICE memory owned by the caller (allocated and
+ *   freed by the caller; the library never allocates device memory). Arrays are
+ *   dense, row-major, in the layouts given per argument.
+ * - Calls are asynchronous on `cuda_stream` (a cudaStream_t passed as void*;
+ *   NULL means the legacy default stream). No host synchronisation happens
+ *   inside a call, so a call can be captured in a CUDA graph. The library keeps
+ *   no state between calls (apart from the optional kernel trace below) and is
+ *   re-entrant; two calls may share a workspace only if they are ordered.
+ * - Workspace: calls that need scratch memory take `workspace` / `ws_bytes`;
+ *   the size comes from the matching *_workspace() query, evaluated for the
+ *   current device. The workspace must be 256-byte aligned. Its contents on
+ *   entry are irrelevant and on exit unspecified.
+ * - Return value: PCT_OK, or an error detected on the host BEFORE anything is
+ *   launched (PCT_EINVAL, PCT_EWORKSPACE, PCT_EUNSUPPORTED, PCT_EDEVICE), or
+ *   PCT_ECUDA when a launch fails. Data errors found on the device are written
+ *   to the caller's per-request `dev_status` word (bits PCT_DEV_*; 0 = fine);
+ *   other requests still complete. There is no device trap, assert or
+ *   unbounded wait; a bounded wait that gives up sets PCT_DEV_TIMEOUT.
+ * - Node tables (tok, parent, depth, score), per request, slot 0 is the root:
+ *   tok = anchor, parent = -1, depth = 0, score = 0. Nodes are in canonical
+ *   BFS order: by depth, then by (parent index, token); parent[i] < i. Slots at
+ *   or past `count` hold tok = -1, parent = -1, depth = -1, score = -inf.
+ * - Total order used by every selection: higher score first, then lower depth,
+ *   then the lexicographically smaller token path (siblings: lower token id).
+ * - dtypes: PCT_F32 = IEEE binary32, PCT_BF16 = bfloat16 (upper half of a
+ *   binary32). Arithmetic is fp32 throughout (bf16 inputs are widened exactly).
+ */
+#ifndef PCTREE_H
+#define PCTREE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Host return codes. */
+enum {
+  PCT_OK = 0,
+  PCT_EINVAL = 1,        /* bad argument or shape; nothing launched            */
+  PCT_EWORKSPACE = 2,    /* workspace NULL, misaligned or smaller than needed   */
+  PCT_ECUDA = 3,         /* a CUDA runtime/driver call or a launch failed       */
+  PCT_EDEVICE = 4,       /* current device is not compute capability 10.x       */
+  PCT_ETIMEOUT = 5,      /* reserved for host-visible timeouts                  */
+  PCT_EUNSUPPORTED = 6   /* valid combination outside this build's limits       */
+};
+
+/* Element types. */
+enum { PCT_F32 = 0, PCT_BF16 = 1 };
+
+/* Device status bits, OR-ed into dev_status[request]. */
+enum {
+  PCT_DEV_BAD_PARENT = 1,     /* parent[i] not in [0, i) for 0 < i < count, or parent[0] != -1 */
+  PCT_DEV_BAD_TOKEN = 2,      /* a token or anchor outside [0, vocab)                         */
+  PCT_DEV_BAD_COUNT = 4,      /* count outside [1, n_stride]                                  */
+  PCT_DEV_DEPTH_OVERFLOW = 8, /* accept walk longer than max_depth                            */
+  PCT_DEV_BAD_COST = 16,      /* CaDDTree cost C(n) <= 0 for some n in [1, n_max]             */
+  PCT_DEV_TIMEOUT = 32        /* a bounded device wait gave up                                */
+};
+
+/* ------------------------------------------------------------------------ *
+ * PCTree: parent-conditioned drafting tree.
+ * Source: PCTree article (qiita), section on the chain draft's weakness and
+ * the tree built in its place: for every frontier parent p at depth d the
+ * drafter's logits are z_d(p) = L_d + Markov(p), all parents scored in one
+ * batched Markov call; each parent keeps its local top-k children; candidates
+ * are ranked by s(c) = sum log pi(v|u) along the path; each depth is pruned to
+ * a beam; a global top-N fits the verification budget.
+ * Here Markov(p) = E[p] . W, a rank-r stand-in for the drafter's head,
+ * pi(.|u) = softmax over the vocabulary of z_d(u), s(root) = 0, depth 1 is
+ * conditioned on the anchor, and the block has D = B - 1 drafted depths.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int32_t batch;        /* independent requests, >= 1                          */
+  int32_t depth;        /* D, drafted depths (block size B = D + 1), 1..64      */
+  int32_t vocab;        /* V, >= k                                              */
+  int32_t rank;         /* r of E [V][r] and W [r][V], 1..256                   */
+  int32_t k;            /* local top-k children per parent, 1..16              */
+  int32_t beam;         /* frontier width kept per depth, 1..256, beam*k <= 1024 */
+  int32_t n_nodes;      /* N, tree budget including the root, 1..4096;
+                           depth * beam <= 4096                                 */
+  int32_t logits_dtype; /* PCT_F32 or PCT_BF16, for L                           */
+  int32_t markov_dtype; /* PCT_F32 or PCT_BF16, for E and W. BF16 runs on the
+                           tcgen05 tensor cores and needs vocab % 8 == 0 (16-byte
+                           rows for TMA); F32 runs on the FP32 pipes.           */
+} pct_build_desc;
+
+/* Workspace bytes pct_tree_build needs for `desc` on the current device;
+ * 0 when desc is invalid. */
+size_t pct_tree_build_workspace(const pct_build_desc* desc);
+
+/* Build one PCTree per request.
+ *   L          [batch][D][V] logits_dtype  drafter logits; row d-1 serves depth d
+ *   anchor     [batch] int32               depth-0 token of each block
+ *   E          [V][r] markov_dtype,  W [r][V] markov_dtype
+ *   tok, parent, depth  [batch][N] int32;  score [batch][N] float (path log-prob)
+ *   count      [batch] int32   nodes written, min(N, 1 + sum_d |F_d|)
+ *   dev_status [batch] int32   0 or PCT_DEV_* bits
+ * Ties between exactly equal scores follow the total order above. */
+int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t* anchor,
+                       const void* E, const void* W, int32_t* tok, int32_t* parent,
+                       int32_t* depth, float* score, int32_t* count, int32_t* dev_status,
+                       void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* One depth of PCTree's batched parent scoring (the step inside
+ * pct_tree_build before the beam): for request b and each of its n_par
+ * parents p with token parent_tok[b][p],
+ *   z = L_row[b] + E[parent_tok] . W,  lse = log sum_v exp z,
+ *   top_tok[b][p][j], top_logpi[b][p][j] = the k best (z desc, token asc)
+ *   children and their log pi = z - lse.
+ * Uses desc->vocab, rank, k, logits_dtype, markov_dtype; desc->batch is the
+ * number of requests and n_par <= 1024 the parents per request.
+ *   L_row [batch][V], parent_tok [batch][n_par] int32, lse [batch][n_par] float,
+ *   top_tok [batch][n_par][k] int32, top_logpi [batch][n_par][k] float. */
+size_t pct_score_parents_workspace(const pct_build_desc* desc, int32_t n_par);
+int32_t pct_score_parents(const pct_build_desc* desc, int32_t n_par, const void* L_row,
+                          const int32_t* parent_tok, const void* E, const void* W,
+                          float* lse, int32_t* top_tok, float* top_logpi,
+                          int32_t* dev_status, void* workspace, size_t ws_bytes,
+                          void* cuda_stream);
+
+/* ------------------------------------------------------------------------ *
+ * CaDDTree: cost-aware best-first draft tree.
+ * Source: "Cost-Aware Diffusion Draft Trees for Speculative Decoding"
+ * (gist.science summary), technical summary, "Method: CaDDTree": a round
+ * costs C(T; l) = C_d + C_v(|T|; l); the tree maximises (1 + Phi(T)) / C;
+ * for a fixed size the best tree is greedy best-first by prefix probability;
+ * with convex C_v the objective is unimodal, so nodes are added one at a time
+ * until the marginal gain is non-positive.
+ * Here q_d = softmax(L_d) are per-position marginals, a node's prefix
+ * probability is prod_j q_j(v_j), Phi(T) sums it over non-root nodes, |T|
+ * counts the root, C_v(n; l) = a + b l + c n + e n^2, and growth stops at the
+ * first n with f(n + 1) <= f(n), f(n) = (1 + Phi_n) / C(n), at n = n_max, or
+ * when no candidate is left.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int32_t batch;        /* requests, >= 1                                   */
+  int32_t depth;        /* D, 1..63                                         */
+  int32_t vocab;        /* V, 1..2^24                                       */
+  int32_t n_max;        /* node cap including the root, 1..1024             */
+  int32_t logits_dtype; /* PCT_F32 or PCT_BF16                              */
+  float C_d;            /* draft cost                                       */
+  float a, b, c, e;     /* C_v coefficients; c >= 0 and e >= 0 (convex)     */
+} cadd_desc;
+
+size_t cadd_tree_grow_workspace(const cadd_desc* desc);
+
+/* Grow one CaDDTree per request.
+ *   L       [batch][D][V] logits_dtype   marginal logits, row d-1 for depth d
+ *   anchor  [batch] int32;  ctx_len [batch] int64 (context length l)
+ *   tok, parent, depth [batch][n_max] int32; score [batch][n_max] float (log prefix prob)
+ *   count   [batch] int32  n*;  phi [batch] float  Phi(T)
+ *   dev_status [batch] int32 */
+int32_t cadd_tree_grow(const cadd_desc* desc, const void* L, const int32_t* anchor,
+                       const int64_t* ctx_len, int32_t* tok, int32_t* parent, int32_t* depth,
+                       float* score, int32_t* count, float* phi, int32_t* dev_status,
+                       void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* ------------------------------------------------------------------------ *
+ * Ancestor bitmask for tree attention: bit j of row i (word j / 32, bit
+ * j % 32, least significant first) is set iff j == i or j is an ancestor of
+ * i. Rows at or past count[b] are zero.
+ *   parent [batch][n_stride] int32 (parent[i] < i), count [batch] int32
+ *   mask   [batch][n_stride][ceil(n_stride / 32)] uint32
+ * n_stride in 1..4096. No workspace.
+ * ------------------------------------------------------------------------ */
+int32_t tree_ancestor_mask(int32_t batch, int32_t n_stride, const int32_t* parent,
+                           const int32_t* count, uint32_t* mask, int32_t* dev_status,
+                           void* cuda_stream);
+
+/* ------------------------------------------------------------------------ *
+ * Greedy tree verification.
+ * Source: DSpark explainer (xiaohu-jiedu), section on one round from drafting
+ * to confirmation: drafts are checked from the head, consecutive matches are
+ * kept, checking stops at the first miss, and the target adds its own token
+ * there (four matches give five tokens for one verification).
+ * Here, per node u < count: argmax[u] = argmax_v target[u][v] on the raw
+ * values, ties toward the lower v. From the root, move to the child whose
+ * token equals argmax[u] (the lowest-index such child), stop when none does;
+ * accept_len = nodes moved to, correction = argmax at the last node reached.
+ *   tok, parent [batch][n_stride] int32; count [batch] int32
+ *   target [batch][n_stride][V] target_dtype (rows >= count are not read)
+ *   argmax [batch][n_stride] int32 (-1 at rows >= count)
+ *   accept_len [batch]; accept_path [batch][max_depth] node ids (-1 padded);
+ *   correction [batch]; dev_status [batch]
+ * n_stride in 1..4096, max_depth in 1..4096 (a walk longer than max_depth
+ * stops there and sets PCT_DEV_DEPTH_OVERFLOW).
+ * ------------------------------------------------------------------------ */
+size_t tree_verify_accept_workspace(int32_t batch, int32_t n_stride);
+int32_t tree_verify_accept(int32_t batch, int32_t n_stride, int32_t vocab, int32_t max_depth,
+                           const int32_t* tok, const int32_t* parent, const int32_t* count,
+                           const void* target, int32_t target_dtype, int32_t* argmax,
+                           int32_t* accept_len, int32_t* accept_path, int32_t* correction,
+                           int32_t* dev_status, void* workspace, size_t ws_bytes,
+                           void* cuda_stream);
+
+/* ------------------------------------------------------------------------ *
+ * Kernel trace (off by default; host-side bookkeeping only). While on, every
+ * kernel the library launches is bracketed by two CUDA events on its stream
+ * and the elapsed time is accumulated per kernel name. Not for use inside
+ * CUDA-graph capture.
+ * ------------------------------------------------------------------------ */
+int32_t pct_trace_enable(int32_t on);   /* returns the previous setting */
+int32_t pct_trace_reset(void);
+/* Waits for the recorded events, then writes up to max_entries rows: a
+ * NUL-terminated kernel name in names[i * name_stride], the launch count and
+ * the summed device milliseconds. Returns the number of rows written, or -1. */
+int32_t pct_trace_read(char* names, int32_t name_stride, int64_t* launches,
+                       double* total_ms, int32_t max_entries);
+
+/* Library version string (static storage). */
+const char* pct_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PCTREE_H */

@@ -42,13 +42,13 @@ Parity status of each function (what pins it, other than itself, is in
   parent relation.
 """
 from .numerics import decode_bf16, to_f64, row_log_softmax
-from .pctree import pct_tree_build, PCTreeResult
+from .pctree import pct_tree_build, PCTreeResult, score_parents
 from .caddtree import cadd_tree_grow, CaddResult, cadd_cost
 from .verify import tree_verify_accept, tree_ancestor_mask, VerifyResult
 
 __all__ = [
     "decode_bf16", "to_f64", "row_log_softmax",
-    "pct_tree_build", "PCTreeResult",
+    "pct_tree_build", "PCTreeResult", "score_parents",
     "cadd_tree_grow", "CaddResult", "cadd_cost",
     "tree_verify_accept", "tree_ancestor_mask", "VerifyResult",
 ]

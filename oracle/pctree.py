@@ -69,6 +69,23 @@ class _Node:
         self.tok, self.depth, self.s, self.path, self.vals = tok, depth, s, path, vals
 
 
+def score_parents(L_d, parent_tok, E, W, k):
+    """One depth of batched parent scoring for one request.
+
+    For every parent token p: z = L_d + E[p] . W (all parents in one matrix
+    product), log pi = z - lse(z), and the k + 1 best children in the order
+    (z desc, token asc). Returns (z, markov, log_pi, lse, order) with order
+    holding the first min(k + 1, V) token ids of each row.
+    """
+    toks = np.asarray(parent_tok, dtype=np.int64)
+    markov = E[toks] @ W                                       # [|F|][V]
+    Z = L_d[None, :] + markov                                  # z_d(p)
+    logpi, lse = row_log_softmax(Z)
+    # stable sort of -z keeps the lower token first among equal z
+    order = np.argsort(-Z, axis=1, kind="stable")[:, : min(k + 1, Z.shape[1])]
+    return Z, markov, logpi, lse, order
+
+
 def _build_one(L, anchor, E, W, k, beam, n_nodes, tol):
     D, V = L.shape
     root = _Node(int(anchor), 0, 0.0, (), ())
@@ -78,12 +95,7 @@ def _build_one(L, anchor, E, W, k, beam, n_nodes, tol):
     kk = min(k, V)
     for d in range(1, D + 1):
         # one batched Markov call for every frontier parent: E[tok(p)] . W
-        toks = np.array([p.tok for p in frontier], dtype=np.int64)
-        markov = E[toks] @ W                                   # [|F|][V]
-        Z = L[d - 1][None, :] + markov                         # z_d(p)
-        logpi, lse = row_log_softmax(Z)
-        # stable sort of -z keeps the lower token first among equal z
-        order = np.argsort(-Z, axis=1, kind="stable")
+        Z, markov, logpi, lse, order = score_parents(L[d - 1], [p.tok for p in frontier], E, W, k)
         cands = []
         for i, p in enumerate(frontier):
             for j in range(kk):

@@ -1,0 +1,456 @@
+// C ABI of libpctree: argument checks, workspace planning and the launch
+// sequence of each call. Everything here runs on the host and only enqueues
+// work on the caller's stream; no call synchronises or allocates device memory.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+
+namespace pct {
+
+size_t score_smem_bytes();
+
+// ---------------------------------------------------------------------------
+// device queries
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  n = std::max(n, 1);
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
+bool device_ok() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  return major == 10;
+}
+
+// ---------------------------------------------------------------------------
+// kernel trace
+namespace {
+std::mutex g_mu;
+volatile bool g_on = false;
+struct Rec {
+  int name;
+  cudaEvent_t a, b;
+};
+std::vector<Rec> g_recs;
+std::vector<std::string> g_names;
+std::vector<cudaEvent_t> g_pool;
+
+cudaEvent_t take_event() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+int name_id(const char* n) {
+  for (size_t i = 0; i < g_names.size(); ++i)
+    if (g_names[i] == n) return (int)i;
+  g_names.emplace_back(n);
+  return (int)g_names.size() - 1;
+}
+}  // namespace
+
+TraceScope::TraceScope(cudaStream_t s, const char* name) : stream(s), slot(-1) {
+  if (!g_on) return;
+  std::lock_guard<std::mutex> lk(g_mu);
+  Rec r;
+  r.name = name_id(name);
+  r.a = take_event();
+  r.b = take_event();
+  if (!r.a || !r.b) return;
+  cudaEventRecord(r.a, s);
+  g_recs.push_back(r);
+  slot = (int)g_recs.size() - 1;
+}
+
+TraceScope::~TraceScope() {
+  if (slot < 0) return;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (slot < (int)g_recs.size()) cudaEventRecord(g_recs[slot].b, stream);
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+size_t esize(int dt) { return dt == PCT_BF16 ? 2 : 4; }
+bool dtype_ok(int dt) { return dt == PCT_F32 || dt == PCT_BF16; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---------------------------------------------------------------------------
+// PCTree plan: frontier sizes per depth, V-slices per depth, workspace layout.
+struct PctPlan {
+  int batch, D, V, r, r_pad, k, beam, N, ldt, mdt;
+  int F[66];
+  int S[66];
+  int Mmax, M_pad;
+  size_t max_ps;
+  size_t o_eg, o_ms, o_val, o_idx, o_ltok, o_lppos, o_ls, o_err, total;
+};
+
+int check_build_desc(const pct_build_desc* d) {
+  if (!d) return PCT_EINVAL;
+  if (d->batch < 1 || d->batch > 65535) return PCT_EINVAL;
+  if (d->depth < 1 || d->depth > 64) return PCT_EINVAL;
+  if (d->vocab < 1 || d->k < 1 || d->k > 16 || d->k > d->vocab) return PCT_EINVAL;
+  if (d->rank < 1 || d->rank > 256) return PCT_EINVAL;
+  if (d->beam < 1 || d->beam > 256 || d->beam * d->k > 1024) return PCT_EINVAL;
+  if (d->n_nodes < 1 || d->n_nodes > 4096 || d->depth * d->beam > 4096) return PCT_EINVAL;
+  if (!dtype_ok(d->logits_dtype) || !dtype_ok(d->markov_dtype)) return PCT_EINVAL;
+  if (d->markov_dtype == PCT_BF16 && d->vocab % 8 != 0) return PCT_EUNSUPPORTED;
+  return PCT_OK;
+}
+
+int make_plan(const pct_build_desc* d, PctPlan* P) {
+  const int st = check_build_desc(d);
+  if (st != PCT_OK) return st;
+  P->batch = d->batch; P->D = d->depth; P->V = d->vocab; P->r = d->rank; P->k = d->k;
+  P->beam = d->beam; P->N = d->n_nodes; P->ldt = d->logits_dtype; P->mdt = d->markov_dtype;
+  P->r_pad = P->mdt == PCT_BF16 ? (P->r + 63) / 64 * 64 : P->r;
+  P->F[0] = 1;
+  P->Mmax = 0;
+  P->max_ps = 0;
+  for (int dd = 1; dd <= P->D; ++dd) {
+    P->F[dd] = std::min(P->beam, P->F[dd - 1] * P->k);
+    const int M = P->batch * P->F[dd - 1];
+    P->Mmax = std::max(P->Mmax, M);
+    P->S[dd] = score_slices(M, P->V, P->mdt);
+    P->max_ps = std::max(P->max_ps, (size_t)M * P->S[dd]);
+  }
+  P->M_pad = (P->Mmax + 127) / 128 * 128;
+  const size_t lvl = (size_t)P->D * P->batch * P->beam;
+  size_t o = 0;
+  P->o_eg = o;    o += align_up((size_t)P->M_pad * P->r_pad * esize(P->mdt));
+  P->o_ms = o;    o += align_up(P->max_ps * sizeof(float2));
+  P->o_val = o;   o += align_up(P->max_ps * P->k * sizeof(float));
+  P->o_idx = o;   o += align_up(P->max_ps * P->k * sizeof(int32_t));
+  P->o_ltok = o;  o += align_up(lvl * sizeof(int32_t));
+  P->o_lppos = o; o += align_up(lvl * sizeof(int32_t));
+  P->o_ls = o;    o += align_up(lvl * sizeof(float));
+  P->o_err = o;   o += align_up(sizeof(int32_t));
+  P->total = o;
+  return PCT_OK;
+}
+
+int ws_check(const void* ws, size_t have, size_t need) {
+  if (need == 0) return PCT_OK;
+  if (!ws || !aligned(ws, kAlign) || have < need) return PCT_EWORKSPACE;
+  return PCT_OK;
+}
+
+#define PCT_CU(x)                               \
+  do {                                          \
+    if ((x) != cudaSuccess) return PCT_ECUDA;   \
+  } while (0)
+
+// ---------------------------------------------------------------------------
+// CaDDTree plan
+int check_cadd(const cadd_desc* d) {
+  if (!d) return PCT_EINVAL;
+  if (d->batch < 1 || d->batch > 65535 || d->depth < 1 || d->depth > 63) return PCT_EINVAL;
+  if (d->vocab < 1 || d->vocab > (1 << 24)) return PCT_EINVAL;
+  if (d->n_max < 1 || d->n_max > 1024) return PCT_EINVAL;
+  if (!dtype_ok(d->logits_dtype)) return PCT_EINVAL;
+  if (!(d->c >= 0.f) || !(d->e >= 0.f)) return PCT_EINVAL;   // convex, monotone C_v
+  if (!std::isfinite(d->C_d) || !std::isfinite(d->a) || !std::isfinite(d->b) ||
+      !std::isfinite(d->c) || !std::isfinite(d->e))
+    return PCT_EINVAL;
+  return PCT_OK;
+}
+struct CaddPlan {
+  size_t o_lse, o_cnt, o_q, o_tok, total;
+};
+void cadd_plan(const cadd_desc* d, CaddPlan* P) {
+  const size_t rows = (size_t)d->batch * d->depth;
+  const size_t K1 = (size_t)std::max(d->n_max - 1, 1);
+  size_t o = 0;
+  P->o_lse = o; o += align_up(rows * sizeof(float));
+  P->o_cnt = o; o += align_up(rows * sizeof(int32_t));
+  P->o_q = o;   o += align_up(rows * K1 * sizeof(float));
+  P->o_tok = o; o += align_up(rows * K1 * sizeof(int32_t));
+  P->total = o;
+}
+
+}  // namespace
+}  // namespace pct
+
+using namespace pct;
+
+extern "C" {
+
+const char* pct_version(void) { return "pctree-b200 0.1 (sm_100a)"; }
+
+int32_t pct_trace_enable(int32_t on) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  const int32_t prev = g_on ? 1 : 0;
+  g_on = on != 0;
+  return prev;
+}
+
+int32_t pct_trace_reset(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (auto& r : g_recs) {
+    cudaEventSynchronize(r.b);
+    g_pool.push_back(r.a);
+    g_pool.push_back(r.b);
+  }
+  g_recs.clear();
+  return PCT_OK;
+}
+
+int32_t pct_trace_read(char* names, int32_t name_stride, int64_t* launches, double* total_ms,
+                       int32_t max_entries) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  std::vector<int64_t> cnt(g_names.size(), 0);
+  std::vector<double> ms(g_names.size(), 0.0);
+  for (auto& r : g_recs) {
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return -1;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) return -1;
+    cnt[r.name] += 1;
+    ms[r.name] += t;
+  }
+  int32_t n = 0;
+  for (size_t i = 0; i < g_names.size() && n < max_entries; ++i) {
+    if (cnt[i] == 0) continue;
+    if (names && name_stride > 0) {
+      std::strncpy(names + (size_t)n * name_stride, g_names[i].c_str(), name_stride - 1);
+      names[(size_t)n * name_stride + name_stride - 1] = '\0';
+    }
+    if (launches) launches[n] = cnt[i];
+    if (total_ms) total_ms[n] = ms[i];
+    ++n;
+  }
+  return n;
+}
+
+// ---------------------------------------------------------------------------
+size_t pct_tree_build_workspace(const pct_build_desc* desc) {
+  PctPlan P;
+  if (make_plan(desc, &P) != PCT_OK) return 0;
+  return P.total;
+}
+
+int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t* anchor,
+                       const void* E, const void* W, int32_t* tok, int32_t* parent,
+                       int32_t* depth, float* score, int32_t* count, int32_t* dev_status,
+                       void* workspace, size_t ws_bytes, void* cuda_stream) {
+  PctPlan P;
+  const int st = make_plan(desc, &P);
+  if (st != PCT_OK) return st;
+  if (!L || !anchor || !E || !W || !tok || !parent || !depth || !score || !count || !dev_status)
+    return PCT_EINVAL;
+  if (P.mdt == PCT_BF16 && (!aligned(W, 16) || !aligned(L, 16))) return PCT_EINVAL;
+  if (!device_ok()) return PCT_EDEVICE;
+  const int wst = ws_check(workspace, ws_bytes, P.total);
+  if (wst != PCT_OK) return wst;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  char* ws = static_cast<char*>(workspace);
+  void* Eg = ws + P.o_eg;
+  Partials part{reinterpret_cast<float2*>(ws + P.o_ms), reinterpret_cast<float*>(ws + P.o_val),
+                reinterpret_cast<int32_t*>(ws + P.o_idx)};
+  int32_t* ltok = reinterpret_cast<int32_t*>(ws + P.o_ltok);
+  int32_t* lppos = reinterpret_cast<int32_t*>(ws + P.o_lppos);
+  float* ls = reinterpret_cast<float*>(ws + P.o_ls);
+  int32_t* err = reinterpret_cast<int32_t*>(ws + P.o_err);
+  const size_t lvl = (size_t)P.batch * P.beam;
+
+  PCT_CU(cudaMemsetAsync(dev_status, 0, sizeof(int32_t) * P.batch, s));
+  PCT_CU(cudaMemsetAsync(err, 0, sizeof(int32_t), s));
+  PCT_CU(launch_gather_rows(P.batch, anchor, P.V, P.r, P.r_pad, P.mdt, E, Eg, dev_status, 1, s));
+  for (int d = 1; d <= P.D; ++d) {
+    ScoreArgs a;
+    a.n_req = P.batch; a.n_par = P.F[d - 1]; a.V = P.V; a.r = P.r; a.r_pad = P.r_pad; a.k = P.k;
+    a.logits_dtype = P.ldt; a.markov_dtype = P.mdt;
+    a.L = static_cast<const char*>(L) + (size_t)(d - 1) * P.V * esize(P.ldt);
+    a.L_req_stride = (long long)P.D * P.V;
+    a.Eg = Eg; a.M_pad = P.M_pad; a.W = W; a.part = part; a.S = P.S[d]; a.err = err;
+    PCT_CU(launch_score(a, s));
+    MergeArgs m;
+    m.batch = P.batch; m.F_prev = P.F[d - 1]; m.F_new = P.F[d]; m.k = P.k; m.beam = P.beam;
+    m.S = P.S[d]; m.V = P.V; m.r = P.r; m.r_pad = P.r_pad; m.markov_dtype = P.mdt; m.depth = d;
+    m.part = part;
+    m.prev_tok = nullptr;
+    m.prev_s = d == 1 ? nullptr : ls + (size_t)(d - 2) * lvl;
+    m.prev_stride = P.beam;
+    m.lvl_tok = ltok + (size_t)(d - 1) * lvl;
+    m.lvl_ppos = lppos + (size_t)(d - 1) * lvl;
+    m.lvl_s = ls + (size_t)(d - 1) * lvl;
+    m.E = E;
+    m.Eg_next = d < P.D ? Eg : nullptr;
+    m.err = err;
+    m.status = dev_status;
+    PCT_CU(launch_merge(m, s));
+  }
+  FinalArgs f;
+  f.batch = P.batch; f.D = P.D; f.beam = P.beam; f.N = P.N;
+  for (int d = 0; d <= P.D; ++d) f.F[d] = P.F[d];
+  f.anchor = anchor; f.lvl_tok = ltok; f.lvl_ppos = lppos; f.lvl_s = ls;
+  f.tok = tok; f.parent = parent; f.depth = depth; f.count = count; f.score = score;
+  f.status = dev_status;
+  PCT_CU(launch_final(f, s));
+  return PCT_OK;
+}
+
+// ---------------------------------------------------------------------------
+static int score_parents_plan(const pct_build_desc* d, int32_t n_par, PctPlan* P, size_t* o_eg,
+                              size_t* o_ms, size_t* o_val, size_t* o_idx, size_t* o_err,
+                              size_t* total, int* S) {
+  if (!d) return PCT_EINVAL;
+  if (d->batch < 1 || d->batch > 65535 || n_par < 1 || n_par > 4096) return PCT_EINVAL;
+  if (d->vocab < 1 || d->k < 1 || d->k > 16 || d->k > d->vocab) return PCT_EINVAL;
+  if (d->rank < 1 || d->rank > 256) return PCT_EINVAL;
+  if (!dtype_ok(d->logits_dtype) || !dtype_ok(d->markov_dtype)) return PCT_EINVAL;
+  if (d->markov_dtype == PCT_BF16 && d->vocab % 8 != 0) return PCT_EUNSUPPORTED;
+  P->batch = d->batch; P->V = d->vocab; P->r = d->rank; P->k = d->k;
+  P->ldt = d->logits_dtype; P->mdt = d->markov_dtype;
+  P->r_pad = P->mdt == PCT_BF16 ? (P->r + 63) / 64 * 64 : P->r;
+  const int rows = d->batch * n_par;
+  P->M_pad = (rows + 127) / 128 * 128;
+  *S = score_slices(rows, P->V, P->mdt);
+  const size_t ps = (size_t)rows * *S;
+  size_t o = 0;
+  *o_eg = o;  o += align_up((size_t)P->M_pad * P->r_pad * esize(P->mdt));
+  *o_ms = o;  o += align_up(ps * sizeof(float2));
+  *o_val = o; o += align_up(ps * P->k * sizeof(float));
+  *o_idx = o; o += align_up(ps * P->k * sizeof(int32_t));
+  *o_err = o; o += align_up(sizeof(int32_t));
+  *total = o;
+  return PCT_OK;
+}
+
+size_t pct_score_parents_workspace(const pct_build_desc* desc, int32_t n_par) {
+  PctPlan P;
+  size_t a, b, c, d, e, total;
+  int S;
+  if (score_parents_plan(desc, n_par, &P, &a, &b, &c, &d, &e, &total, &S) != PCT_OK) return 0;
+  return total;
+}
+
+int32_t pct_score_parents(const pct_build_desc* desc, int32_t n_par, const void* L_row,
+                          const int32_t* parent_tok, const void* E, const void* W, float* lse,
+                          int32_t* top_tok, float* top_logpi, int32_t* dev_status,
+                          void* workspace, size_t ws_bytes, void* cuda_stream) {
+  PctPlan P;
+  size_t o_eg, o_ms, o_val, o_idx, o_err, total;
+  int S;
+  const int st = score_parents_plan(desc, n_par, &P, &o_eg, &o_ms, &o_val, &o_idx, &o_err, &total, &S);
+  if (st != PCT_OK) return st;
+  if (!L_row || !parent_tok || !E || !W || !lse || !top_tok || !top_logpi || !dev_status)
+    return PCT_EINVAL;
+  if (P.mdt == PCT_BF16 && (!aligned(W, 16) || !aligned(L_row, 16))) return PCT_EINVAL;
+  if (!device_ok()) return PCT_EDEVICE;
+  const int wst = ws_check(workspace, ws_bytes, total);
+  if (wst != PCT_OK) return wst;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  char* ws = static_cast<char*>(workspace);
+  Partials part{reinterpret_cast<float2*>(ws + o_ms), reinterpret_cast<float*>(ws + o_val),
+                reinterpret_cast<int32_t*>(ws + o_idx)};
+  int32_t* err = reinterpret_cast<int32_t*>(ws + o_err);
+  const int rows = P.batch * n_par;
+  PCT_CU(cudaMemsetAsync(dev_status, 0, sizeof(int32_t) * P.batch, s));
+  PCT_CU(cudaMemsetAsync(err, 0, sizeof(int32_t), s));
+  PCT_CU(launch_gather_rows(rows, parent_tok, P.V, P.r, P.r_pad, P.mdt, E, ws + o_eg, dev_status,
+                            n_par, s));
+  ScoreArgs a;
+  a.n_req = P.batch; a.n_par = n_par; a.V = P.V; a.r = P.r; a.r_pad = P.r_pad; a.k = P.k;
+  a.logits_dtype = P.ldt; a.markov_dtype = P.mdt; a.L = L_row; a.L_req_stride = P.V;
+  a.Eg = ws + o_eg; a.M_pad = P.M_pad; a.W = W; a.part = part; a.S = S; a.err = err;
+  PCT_CU(launch_score(a, s));
+  PCT_CU(launch_rows_finalize(rows, P.k, S, part, lse, top_tok, top_logpi, err, dev_status, n_par, s));
+  return PCT_OK;
+}
+
+// ---------------------------------------------------------------------------
+size_t cadd_tree_grow_workspace(const cadd_desc* desc) {
+  if (check_cadd(desc) != PCT_OK) return 0;
+  CaddPlan P;
+  cadd_plan(desc, &P);
+  return P.total;
+}
+
+int32_t cadd_tree_grow(const cadd_desc* desc, const void* L, const int32_t* anchor,
+                       const int64_t* ctx_len, int32_t* tok, int32_t* parent, int32_t* depth,
+                       float* score, int32_t* count, float* phi, int32_t* dev_status,
+                       void* workspace, size_t ws_bytes, void* cuda_stream) {
+  const int st = check_cadd(desc);
+  if (st != PCT_OK) return st;
+  if (!L || !anchor || !ctx_len || !tok || !parent || !depth || !score || !count || !phi || !dev_status)
+    return PCT_EINVAL;
+  if (!device_ok()) return PCT_EDEVICE;
+  CaddPlan P;
+  cadd_plan(desc, &P);
+  const int wst = ws_check(workspace, ws_bytes, P.total);
+  if (wst != PCT_OK) return wst;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  char* ws = static_cast<char*>(workspace);
+  PCT_CU(cudaMemsetAsync(dev_status, 0, sizeof(int32_t) * desc->batch, s));
+  CaddParams p{desc->batch, desc->depth, desc->vocab, desc->n_max, desc->logits_dtype,
+               desc->C_d, desc->a, desc->b, desc->c, desc->e};
+  PCT_CU(launch_cadd(p, L, anchor, ctx_len, tok, parent, depth, score, count, phi, dev_status,
+                     reinterpret_cast<float*>(ws + P.o_lse), reinterpret_cast<int32_t*>(ws + P.o_cnt),
+                     reinterpret_cast<float*>(ws + P.o_q), reinterpret_cast<int32_t*>(ws + P.o_tok), s));
+  return PCT_OK;
+}
+
+// ---------------------------------------------------------------------------
+int32_t tree_ancestor_mask(int32_t batch, int32_t n_stride, const int32_t* parent,
+                           const int32_t* count, uint32_t* mask, int32_t* dev_status,
+                           void* cuda_stream) {
+  if (batch < 1 || batch > 65535 || n_stride < 1 || n_stride > 4096) return PCT_EINVAL;
+  if (!parent || !count || !mask || !dev_status) return PCT_EINVAL;
+  if (!device_ok()) return PCT_EDEVICE;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  PCT_CU(cudaMemsetAsync(dev_status, 0, sizeof(int32_t) * batch, s));
+  PCT_CU(launch_ancestor_mask(batch, n_stride, parent, count, mask, dev_status, s));
+  return PCT_OK;
+}
+
+size_t tree_verify_accept_workspace(int32_t batch, int32_t n_stride) {
+  if (batch < 1 || batch > 65535 || n_stride < 1 || n_stride > 4096) return 0;
+  return align_up(sizeof(unsigned) * (size_t)batch);
+}
+
+int32_t tree_verify_accept(int32_t batch, int32_t n_stride, int32_t vocab, int32_t max_depth,
+                           const int32_t* tok, const int32_t* parent, const int32_t* count,
+                           const void* target, int32_t target_dtype, int32_t* argmax,
+                           int32_t* accept_len, int32_t* accept_path, int32_t* correction,
+                           int32_t* dev_status, void* workspace, size_t ws_bytes,
+                           void* cuda_stream) {
+  if (batch < 1 || batch > 65535 || n_stride < 1 || n_stride > 4096) return PCT_EINVAL;
+  if (vocab < 1 || max_depth < 1 || max_depth > 4096 || !dtype_ok(target_dtype)) return PCT_EINVAL;
+  if (!tok || !parent || !count || !target || !argmax || !accept_len || !accept_path ||
+      !correction || !dev_status)
+    return PCT_EINVAL;
+  if (!device_ok()) return PCT_EDEVICE;
+  const size_t need = tree_verify_accept_workspace(batch, n_stride);
+  const int wst = ws_check(workspace, ws_bytes, need);
+  if (wst != PCT_OK) return wst;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  unsigned* arrive = static_cast<unsigned*>(workspace);
+  PCT_CU(cudaMemsetAsync(dev_status, 0, sizeof(int32_t) * batch, s));
+  PCT_CU(cudaMemsetAsync(arrive, 0, sizeof(unsigned) * batch, s));
+  PCT_CU(launch_verify(batch, n_stride, vocab, max_depth, tok, parent, count, target, target_dtype,
+                       argmax, accept_len, accept_path, correction, dev_status, arrive, s));
+  return PCT_OK;
+}
+
+}  // extern "C"

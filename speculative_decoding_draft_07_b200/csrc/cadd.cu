@@ -1,0 +1,457 @@
+// CaDDTree: cost-aware best-first draft tree.
+//
+// "Cost-Aware Diffusion Draft Trees for Speculative Decoding" (gist.science
+// summary), technical summary, "Method: CaDDTree": the tree maximises
+// (1 + Phi(T)) / (C_d + C_v(|T|; l)); for a fixed size the best tree takes the
+// nodes of highest prefix probability (greedy best-first); with convex C_v the
+// objective is unimodal, so nodes are added until the marginal gain is
+// non-positive.
+//
+// Two kernels:
+//  * row pass, one 512-thread block per (request, depth) row of marginal
+//    logits: log-sum-exp in one streaming pass, then a second pass (the row was
+//    just read and normally still sits in L2) that keeps only the tokens that
+//    can ever enter the tree. A node is added at size n only if its prefix
+//    probability p satisfies p > (1 + Phi) dC(n) / C(n) >= theta, where
+//    theta = min_n dC(n) / C(n) and dC(n) = C(n + 1) - C(n); since p never
+//    exceeds the marginal q_d of its last token, tokens with q_d <= theta can
+//    be dropped without changing the result. At most n_max - 1 tokens of a row
+//    can ever be used, so the survivors are sorted (value desc, token asc) and
+//    cut to n_max - 1. If more than the buffer survive (theta tiny), an exact
+//    radix select finds the n_max - 1 best instead.
+//  * best-first growth, one warp per request: a pool of candidate (next
+//    sibling, first child) entries packed into 64-bit keys (score, depth,
+//    parent insertion index, rank) so that one warp max-reduction pops the
+//    best node under the library's total order; the stop test is evaluated in
+//    log form, s > log((1 + Phi) dC(n) / C(n)), before each insertion.
+#include <climits>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace pct {
+namespace {
+
+constexpr int kRowThreads = 512;
+constexpr int kCap = 2048;          // candidate buffer per row (power of two)
+constexpr float kThetaSlack = 1e-3f;
+
+__device__ __forceinline__ unsigned long long cand_key(float x, int v) {
+  return ((unsigned long long)f2ord(x) << 32) | (unsigned)(~v);
+}
+
+// Block reduction of online log-sum-exp pairs; result in every thread.
+__device__ void block_lse(float& m, float& s, float* sm, float* ss) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    lse_combine(m, s, m2, s2);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) { sm[warp] = m; ss[warp] = s; }
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    m = lane < nw ? sm[lane] : neg_inf();
+    s = lane < nw ? ss[lane] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
+      lse_combine(m, s, m2, s2);
+    }
+    if (lane == 0) { sm[0] = m; ss[0] = s; }
+  }
+  __syncthreads();
+  m = sm[0]; s = ss[0];
+  __syncthreads();
+}
+
+// Exclusive block scan of one int per thread; returns the prefix, total in *tot.
+__device__ int block_excl_scan(int x, int* sbuf, int* tot) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) sbuf[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    int w = lane < nw ? sbuf[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < nw) sbuf[lane] = w;   // inclusive warp totals
+  }
+  __syncthreads();
+  const int before = (warp > 0 ? sbuf[warp - 1] : 0) + incl - x;
+  *tot = sbuf[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return before;
+}
+
+// Descending bitonic sort of keys[0..P) in shared memory, P a power of two.
+__device__ void bitonic_desc(unsigned long long* keys, int P) {
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = threadIdx.x; t < P / 2; t += blockDim.x) {
+        const int lo = 2 * t - (t & (stride - 1));
+        const int hi = lo + stride;
+        const bool desc = ((lo & size) == 0);
+        unsigned long long a = keys[lo], b = keys[hi];
+        if (desc ? (a < b) : (a > b)) { keys[lo] = b; keys[hi] = a; }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float elem(const T* x, int v) { return load_f(x + v); }
+
+// Visit every value of a row: f(value, index). bf16 rows with 16-byte aligned
+// starts use vector loads of 8 values; everything else is scalar.
+template <typename T, typename F>
+__device__ __forceinline__ void for_row(const T* x, int V, bool vec, F&& f) {
+  if (sizeof(T) == 2 && vec) {
+    const uint4* p = reinterpret_cast<const uint4*>(x);
+    const int nvec = V >> 3;
+    for (int c = threadIdx.x; c < nvec; c += kRowThreads) {
+      const uint4 q = p[c];
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) f((j & 1) ? bf16_hi(w[j >> 1]) : bf16_lo(w[j >> 1]), c * 8 + j);
+    }
+    for (int v = (nvec << 3) + threadIdx.x; v < V; v += kRowThreads) f(elem(x, v), v);
+  } else {
+    for (int v = threadIdx.x; v < V; v += kRowThreads) f(elem(x, v), v);
+  }
+}
+
+template <typename T>
+__global__ __launch_bounds__(kRowThreads) void cadd_rowpass_kernel(
+    CaddParams p, const T* __restrict__ L, const int64_t* __restrict__ ctx,
+    float* __restrict__ row_lse, int32_t* __restrict__ cand_cnt, float* __restrict__ cand_q,
+    int32_t* __restrict__ cand_tok, int32_t* __restrict__ status) {
+  __shared__ unsigned long long keys[kCap];
+  __shared__ float sm[32], ss[32];
+  __shared__ int sbuf[32];
+  __shared__ int hist[256];
+  __shared__ int s_n, s_tot;
+  __shared__ float s_lnth;
+  const int d = blockIdx.x, b = blockIdx.y;
+  const int V = p.V;
+  const size_t row = (size_t)b * p.D + d;
+  const T* x = L + row * (size_t)V;
+  const int K = p.n_max - 1;               // tokens a row can contribute at most
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool vec = (sizeof(T) == 2) && (V % 8 == 0) && ((reinterpret_cast<uintptr_t>(L) & 15u) == 0);
+
+  // theta for this request: min over n in [1, n_max - 1] of dC(n) / C(n)
+  if (warp == 0) {
+    const double ell = (double)ctx[b];
+    const double cb = (double)p.C_d + (double)p.a + (double)p.b * ell;
+    double th = 1e300;
+    int bad = 0, nonpos = 0;
+    for (int n = 1 + lane; n <= p.n_max; n += 32) {
+      const double Cn = cb + (double)p.c * n + (double)p.e * (double)n * n;
+      if (Cn <= 0.0) bad = 1;
+      if (n < p.n_max) {
+        const double dC = (double)p.c + (double)p.e * (2.0 * n + 1.0);
+        if (dC <= 0.0) nonpos = 1; else if (Cn > 0.0) th = fmin(th, dC / Cn);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      th = fmin(th, __shfl_xor_sync(0xffffffffu, th, o));
+      bad |= __shfl_xor_sync(0xffffffffu, bad, o);
+      nonpos |= __shfl_xor_sync(0xffffffffu, nonpos, o);
+    }
+    if (lane == 0) {
+      if (bad && d == 0) atomicOr(&status[b], PCT_DEV_BAD_COST);
+      s_lnth = (nonpos || th >= 1e299) ? neg_inf() : (float)log(th);
+      s_n = 0;
+    }
+  }
+
+  // pass 1: log-sum-exp
+  float m = neg_inf(), s = 0.f;
+  if (vec) {
+    const uint4* pv = reinterpret_cast<const uint4*>(x);
+    const int nvec = V >> 3;
+    for (int c = threadIdx.x; c < nvec; c += kRowThreads) {
+      const uint4 q = ld_stream16(pv + c);
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+      float cm = neg_inf();
+#pragma unroll
+      for (int j = 0; j < 4; ++j) cm = fmaxf(cm, fmaxf(bf16_lo(w[j]), bf16_hi(w[j])));
+      if (cm > m) { s = (m == neg_inf()) ? 0.f : s * ex2((m - cm) * kLog2e); m = cm; }
+      if (m != neg_inf()) {
+        const float mb = m * kLog2e;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          s += ex2(fmaf(bf16_lo(w[j]), kLog2e, -mb));
+          s += ex2(fmaf(bf16_hi(w[j]), kLog2e, -mb));
+        }
+      }
+    }
+    for (int v = (nvec << 3) + threadIdx.x; v < V; v += kRowThreads) {
+      const float z = elem(x, v);
+      lse_combine(m, s, z, 1.f);
+    }
+  } else {
+    for (int v = threadIdx.x; v < V; v += kRowThreads) lse_combine(m, s, elem(x, v), 1.f);
+  }
+  block_lse(m, s, sm, ss);
+  const float lse = (m == neg_inf()) ? neg_inf() : m + logf(s);
+  // s_lnth was written before the block_lse barriers
+  const float t = (K <= 0) ? __int_as_float(0x7f800000) : lse + s_lnth - kThetaSlack;
+
+  // pass 2: survivors above the threshold (normally served from L2)
+  if (K > 0) {
+    for_row(x, V, vec, [&](float z, int v) {
+      if (z > t) {
+        const int pos = atomicAdd(&s_n, 1);
+        if (pos < kCap) keys[pos] = cand_key(z, v);
+      }
+    });
+  }
+  __syncthreads();
+  int n = s_n;
+  if (n > kCap) {
+    // exact radix select of the K best (value desc, token asc) over the row
+    unsigned prefix = 0, pmask = 0;
+    int need = K;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int j = threadIdx.x; j < 256; j += kRowThreads) hist[j] = 0;
+      __syncthreads();
+      for_row(x, V, vec, [&](float z, int v) {
+        const unsigned kk = f2ord(z);
+        if ((kk & pmask) == prefix) atomicAdd(&hist[(kk >> shift) & 255], 1);
+      });
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int cum = 0, bsel = 0;
+        for (int j = 255; j >= 0; --j) {
+          if (cum + hist[j] >= need) { bsel = j; break; }
+          cum += hist[j];
+        }
+        need -= cum;
+        sbuf[0] = bsel; sbuf[1] = need;
+      }
+      __syncthreads();
+      prefix |= (unsigned)sbuf[0] << shift;
+      pmask |= 255u << shift;
+      need = sbuf[1];
+      __syncthreads();
+    }
+    // prefix is the exact key of the K-th value; take every larger value and
+    // the `need` lowest-index values equal to it (contiguous segments per thread
+    // keep index order)
+    if (threadIdx.x == 0) s_n = 0;
+    __syncthreads();
+    const int seg = (V + kRowThreads - 1) / kRowThreads;
+    const int v0 = threadIdx.x * seg, v1 = min(V, v0 + seg);
+    int ties = 0;
+    for (int v = v0; v < v1; ++v) {
+      const float z = elem(x, v);
+      const unsigned kk = f2ord(z);
+      if (kk > prefix) { const int pos = atomicAdd(&s_n, 1); keys[pos] = cand_key(z, v); }
+      else if (kk == prefix) ++ties;
+    }
+    int tot;
+    int rank = block_excl_scan(ties, sbuf, &tot);
+    const int above = s_n;    // stable after the scan's barriers
+    for (int v = v0; v < v1 && rank < need; ++v) {
+      const float z = elem(x, v);
+      if (f2ord(z) == prefix) { keys[above + rank] = cand_key(z, v); ++rank; }
+    }
+    __syncthreads();
+    n = K;
+  }
+  int P = 1;
+  while (P < n) P <<= 1;
+  for (int j = n + threadIdx.x; j < P; j += kRowThreads) keys[j] = 0ull;
+  __syncthreads();
+  if (P > 1) bitonic_desc(keys, P);
+  const int keep = min(n, max(K, 0));
+  const size_t cbase = row * (size_t)max(K, 1);
+  for (int j = threadIdx.x; j < keep; j += kRowThreads) {
+    const unsigned long long kk = keys[j];
+    const float z = ord2f((unsigned)(kk >> 32));
+    cand_q[cbase + j] = z - lse;
+    cand_tok[cbase + j] = (int)(~(unsigned)(kk & 0xffffffffu));
+  }
+  if (threadIdx.x == 0) {
+    cand_cnt[row] = keep;
+    row_lse[row] = lse;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// best-first growth, one warp per request
+
+__device__ __forceinline__ unsigned long long pool_key(float s, int depth, int pidx, int rank) {
+  return ((unsigned long long)f2ord(s) << 32) | ((unsigned long long)(63 - depth) << 20) |
+         ((unsigned long long)(1023 - pidx) << 10) | (unsigned long long)(1023 - rank);
+}
+
+__global__ __launch_bounds__(32) void cadd_bestfirst_kernel(
+    CaddParams p, const int32_t* __restrict__ anchor, const int64_t* __restrict__ ctx,
+    const int32_t* __restrict__ cand_cnt, const float* __restrict__ cand_q,
+    const int32_t* __restrict__ cand_tok, int32_t* __restrict__ otok, int32_t* __restrict__ opar,
+    int32_t* __restrict__ odep, float* __restrict__ oscore, int32_t* __restrict__ ocount,
+    float* __restrict__ ophi, int32_t* __restrict__ status) {
+  extern __shared__ unsigned long long pool[];          // [n_max + 1]
+  const int nmax = p.n_max;
+  int* ntok = reinterpret_cast<int*>(pool + nmax + 1);  // [n_max] each
+  int* npar = ntok + nmax;
+  int* ndep = npar + nmax;
+  float* ns = reinterpret_cast<float*>(ndep + nmax);
+  int* canon = reinterpret_cast<int*>(ns + nmax);
+  int* order = canon + nmax;
+  __shared__ int dstart[66], dfill[66];
+
+  const int b = blockIdx.x, lane = threadIdx.x;
+  const int D = p.D, K1 = max(nmax - 1, 1);
+  const size_t row0 = (size_t)b * D;
+  const int a0 = anchor[b];
+  if (lane == 0 && (a0 < 0 || a0 >= p.V)) atomicOr(&status[b], PCT_DEV_BAD_TOKEN);
+  if (lane == 0) { ntok[0] = a0; npar[0] = -1; ndep[0] = 0; ns[0] = 0.f; }
+
+  auto cnt_at = [&](int depth) { return cand_cnt[row0 + depth - 1]; };
+  auto q_at = [&](int depth, int rank) { return cand_q[(row0 + depth - 1) * K1 + rank]; };
+  int pool_n = 0;
+  if (D >= 1 && nmax > 1 && cnt_at(1) > 0) {
+    if (lane == 0) pool[0] = pool_key(q_at(1, 0), 1, 0, 0);
+    pool_n = 1;
+  }
+  __syncwarp();
+
+  const float ell = (float)ctx[b];
+  const float cbase = p.C_d + p.a + p.b * ell;
+  int n = 1;
+  float phi = 0.f;
+  while (n < nmax) {
+    unsigned long long best = 0ull;
+    int bslot = -1;
+    for (int j = lane; j < pool_n; j += 32) {
+      const unsigned long long k = pool[j];
+      if (k > best) { best = k; bslot = j; }
+    }
+    const unsigned long long wbest = warp_max_u64(best);
+    if (wbest == 0ull) break;                                     // no candidate left
+    const unsigned own = __ballot_sync(0xffffffffu, best == wbest);
+    bslot = __shfl_sync(0xffffffffu, bslot, __ffs(own) - 1);
+    const float s = ord2f((unsigned)(wbest >> 32));
+    const int depth = 63 - (int)((wbest >> 20) & 63);
+    const int pidx = 1023 - (int)((wbest >> 10) & 1023);
+    const int rank = 1023 - (int)(wbest & 1023);
+    // stop test: add only if f(n + 1) > f(n)  <=>  s > log((1 + Phi) dC(n) / C(n))
+    const float fn = (float)n;
+    const float Cn = cbase + p.c * fn + p.e * fn * fn;
+    const float dC = p.c + p.e * (2.f * fn + 1.f);
+    const float thr = dC > 0.f ? logf((1.f + phi) * dC / Cn) : neg_inf();
+    if (!(s > thr)) break;
+    const int tk = cand_tok[(row0 + depth - 1) * K1 + rank];
+    const int np = pidx;
+    unsigned long long sib = 0ull, child = 0ull;
+    if (rank + 1 < cnt_at(depth)) sib = pool_key(ns[np] + q_at(depth, rank + 1), depth, np, rank + 1);
+    if (depth < D && cnt_at(depth + 1) > 0) child = pool_key(s + q_at(depth + 1, 0), depth + 1, n, 0);
+    __syncwarp();
+    if (lane == 0) {
+      ntok[n] = tk; npar[n] = np; ndep[n] = depth; ns[n] = s;
+      pool[bslot] = sib;
+      if (child) pool[pool_n] = child;
+    }
+    if (child) ++pool_n;
+    phi += expf(s);
+    ++n;
+    __syncwarp();
+  }
+
+  // canonical BFS order: by depth, then (parent's canonical index, token)
+  for (int j = lane; j < 66; j += 32) { dstart[j] = 0; dfill[j] = 0; }
+  __syncwarp();
+  for (int j = lane; j < n; j += 32) atomicAdd(&dstart[ndep[j] + 1], 1);
+  __syncwarp();
+  if (lane == 0) for (int j = 1; j < 66; ++j) dstart[j] += dstart[j - 1];
+  __syncwarp();
+  for (int j = lane; j < n; j += 32) {
+    const int dd = ndep[j];
+    order[dstart[dd] + atomicAdd(&dfill[dd], 1)] = j;
+  }
+  __syncwarp();
+  if (lane == 0) canon[0] = 0;
+  __syncwarp();
+  for (int dd = 1; dd <= D && dd < 64; ++dd) {
+    const int s0 = dstart[dd], s1 = dstart[dd + 1];
+    if (s0 == s1) break;
+    for (int jj = s0 + lane; jj < s1; jj += 32) {
+      const int j = order[jj];
+      const unsigned long long kj = ((unsigned long long)canon[npar[j]] << 32) | (unsigned)ntok[j];
+      int r = 0;
+      for (int ii = s0; ii < s1; ++ii) {
+        const int i2 = order[ii];
+        const unsigned long long ki = ((unsigned long long)canon[npar[i2]] << 32) | (unsigned)ntok[i2];
+        r += ki < kj;
+      }
+      canon[j] = s0 + r;
+    }
+    __syncwarp();
+  }
+  const size_t ob = (size_t)b * nmax;
+  for (int j = lane; j < n; j += 32) {
+    const int o = canon[j];
+    otok[ob + o] = ntok[j];
+    opar[ob + o] = j == 0 ? -1 : canon[npar[j]];
+    odep[ob + o] = ndep[j];
+    oscore[ob + o] = ns[j];
+  }
+  for (int o = n + lane; o < nmax; o += 32) {
+    otok[ob + o] = -1; opar[ob + o] = -1; odep[ob + o] = -1; oscore[ob + o] = neg_inf();
+  }
+  if (lane == 0) { ocount[b] = n; ophi[b] = phi; }
+}
+
+}  // namespace
+
+size_t cadd_rowpass_bytes_per_row(int n_max) {
+  const size_t K1 = (size_t)(n_max > 1 ? n_max - 1 : 1);
+  return K1 * (sizeof(float) + sizeof(int32_t)) + sizeof(float) + sizeof(int32_t);
+}
+
+cudaError_t launch_cadd(const CaddParams& p, const void* L, const int32_t* anchor,
+                        const int64_t* ctx, int32_t* tok, int32_t* parent, int32_t* depth,
+                        float* score, int32_t* count, float* phi, int32_t* status,
+                        float* row_lse, int32_t* cand_cnt, float* cand_q, int32_t* cand_tok,
+                        cudaStream_t s) {
+  {
+    dim3 grid(p.D, p.batch);
+    TraceScope t(s, "cadd_rowpass");
+    if (p.dtype == PCT_BF16)
+      cadd_rowpass_kernel<__nv_bfloat16><<<grid, kRowThreads, 0, s>>>(
+          p, static_cast<const __nv_bfloat16*>(L), ctx, row_lse, cand_cnt, cand_q, cand_tok, status);
+    else
+      cadd_rowpass_kernel<float><<<grid, kRowThreads, 0, s>>>(
+          p, static_cast<const float*>(L), ctx, row_lse, cand_cnt, cand_q, cand_tok, status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const size_t smem = (size_t)(p.n_max + 1) * 8 + (size_t)p.n_max * 4 * 6;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(cadd_bestfirst_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  TraceScope t(s, "cadd_bestfirst");
+  cadd_bestfirst_kernel<<<p.batch, 32, smem, s>>>(p, anchor, ctx, cand_cnt, cand_q, cand_tok, tok,
+                                                  parent, depth, score, count, phi, status);
+  return cudaGetLastError();
+}
+
+}  // namespace pct

@@ -1,0 +1,140 @@
+// Device helpers shared by the kernels of libpctree (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pctree.h"
+
+namespace pct {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
+
+// 2^x on the special-function unit (hardware approximation, flushes subnormal
+// results to zero; relative error a few ulp), used for the softmax sums.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Order-preserving map float -> uint32 (larger float -> larger key). -0 is
+// folded onto +0 first so that equal values give equal keys.
+__device__ __forceinline__ uint32_t f2ord(float f) {
+  uint32_t u = __float_as_uint(f + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ord2f(uint32_t o) {
+  uint32_t u = (o & 0x80000000u) ? (o & 0x7fffffffu) : ~o;
+  return __uint_as_float(u);
+}
+
+// Exact bf16 -> fp32 widening of a raw 16-bit pattern.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+template <typename T> __device__ __forceinline__ float load_f(const T* p);
+template <> __device__ __forceinline__ float load_f<float>(const float* p) { return *p; }
+template <> __device__ __forceinline__ float load_f<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return bf16_lo(*reinterpret_cast<const uint16_t*>(p));
+}
+
+// Streaming 16-byte load that does not allocate in L1.
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+// Key order used by every top-k in this library: larger value first, then
+// lower index. Returns true when (va, ia) goes before (vb, ib).
+__device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+// Sorted (descending by `better`) top-K list kept in registers; K is a
+// compile-time capacity, the live length is the runtime k <= K. Slots start
+// at (-inf, INT_MAX) so that -inf values still enter in index order.
+template <int K>
+struct TopK {
+  float v[K];
+  int i[K];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int j = 0; j < K; ++j) { v[j] = neg_inf(); i[j] = 0x7fffffff; }
+  }
+  // k-th entry (the admission threshold), k in 1..K.
+  __device__ __forceinline__ void kth(int k, float& tv, int& ti) const {
+    tv = v[0]; ti = i[0];
+#pragma unroll
+    for (int j = 1; j < K; ++j) if (j == k - 1) { tv = v[j]; ti = i[j]; }
+  }
+  // Bubble the new element through the sorted list; the last one falls out.
+  __device__ __forceinline__ void insert(float z, int idx) {
+    float cz = z; int ci = idx;
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+      bool sw = better(cz, ci, v[j], i[j]);
+      float tv = v[j]; int ti = i[j];
+      v[j] = sw ? cz : tv; i[j] = sw ? ci : ti;
+      cz = sw ? tv : cz; ci = sw ? ti : ci;
+    }
+  }
+  // Remove the head (shift left).
+  __device__ __forceinline__ void pop() {
+#pragma unroll
+    for (int j = 0; j + 1 < K; ++j) { v[j] = v[j + 1]; i[j] = i[j + 1]; }
+    v[K - 1] = neg_inf(); i[K - 1] = 0x7fffffff;
+  }
+};
+
+// Online log-sum-exp state: sum = sum_j exp(z_j - m).
+struct LseState {
+  float m, s;
+  __device__ __forceinline__ void init() { m = neg_inf(); s = 0.f; }
+};
+__device__ __forceinline__ void lse_combine(float& m, float& s, float m2, float s2) {
+  if (m2 == neg_inf()) return;
+  if (m == neg_inf()) { m = m2; s = s2; return; }
+  if (m2 > m) { s = s * ex2((m - m2) * kLog2e) + s2; m = m2; }
+  else        { s = s + s2 * ex2((m2 - m) * kLog2e); }
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ int warp_min_i(int x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = min(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ int warp_sum_i(int x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    unsigned long long y = __shfl_xor_sync(0xffffffffu, x, o);
+    x = y > x ? y : x;
+  }
+  return x;
+}
+// Warp-wide best (value desc, index asc).
+__device__ __forceinline__ void warp_best(float& v, int& i) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+    int i2 = __shfl_xor_sync(0xffffffffu, i, o);
+    if (better(v2, i2, v, i)) { v = v2; i = i2; }
+  }
+}
+
+}  // namespace pct

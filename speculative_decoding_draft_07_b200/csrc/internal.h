@@ -1,0 +1,113 @@
+// Host-side interfaces between the translation units of libpctree.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/pctree.h"
+
+namespace pct {
+
+// ---- kernel trace (api.cu) ------------------------------------------------
+// Brackets one launch with events when the trace is on. Usage:
+//   { TraceScope t(stream, "name"); kernel<<<...>>>(...); }
+struct TraceScope {
+  TraceScope(cudaStream_t s, const char* name);
+  ~TraceScope();
+  cudaStream_t stream;
+  int slot;
+};
+
+// ---- device queries (api.cu) ----------------------------------------------
+int num_sms();          // SMs of the current device (cached per device)
+bool device_ok();       // compute capability 10.x
+
+// ---- verify.cu --------------------------------------------------------------
+cudaError_t launch_ancestor_mask(int batch, int n_stride, const int32_t* parent,
+                                 const int32_t* count, uint32_t* mask, int32_t* status,
+                                 cudaStream_t s);
+cudaError_t launch_verify(int batch, int n_stride, int vocab, int max_depth, const int32_t* tok,
+                          const int32_t* parent, const int32_t* count, const void* target,
+                          int dtype, int32_t* argmax, int32_t* alen, int32_t* apath,
+                          int32_t* corr, int32_t* status, unsigned* arrive, cudaStream_t s);
+
+// ---- cadd.cu ----------------------------------------------------------------
+struct CaddParams {
+  int batch, D, V, n_max, dtype;
+  float C_d, a, b, c, e;
+};
+size_t cadd_rowpass_bytes_per_row(int n_max);
+cudaError_t launch_cadd(const CaddParams& p, const void* L, const int32_t* anchor,
+                        const int64_t* ctx, int32_t* tok, int32_t* parent, int32_t* depth,
+                        float* score, int32_t* count, float* phi, int32_t* status,
+                        float* row_lse, int32_t* cand_cnt, float* cand_q, int32_t* cand_tok,
+                        cudaStream_t s);
+
+// ---- PCTree (pct_*.cu) ------------------------------------------------------
+// Partial results of one (row, V-slice): online log-sum-exp state and the
+// slice's top-k (value desc, token asc).
+struct Partials {
+  float2* ms;      // [rows][S]    (max, sum exp(z - max))
+  float* val;      // [rows][S][k] z values
+  int32_t* idx;    // [rows][S][k] token ids
+};
+
+// One depth of batched parent scoring: rows = n_req * n_par; row r belongs
+// to request r / n_par and its parent embedding row is Eg[r].
+struct ScoreArgs {
+  int n_req, n_par, V, r, r_pad, k;
+  int logits_dtype, markov_dtype;
+  const void* L;          // logits base for request 0
+  long long L_req_stride; // elements between consecutive requests' rows
+  const void* Eg;         // [M_pad][r_pad] (bf16) or [M_pad][r] (f32)
+  int M_pad;
+  const void* W;          // [r][V]
+  Partials part;
+  int S;                  // V-slices (partials per row)
+  int32_t* err;           // device word, set on a timed-out wait
+};
+// Slices the scoring kernel will use for `rows` rows (deterministic per device).
+int score_slices(int rows, int V, int markov_dtype);
+cudaError_t launch_score(const ScoreArgs& a, cudaStream_t s);
+
+// Gather E rows of tokens into Eg (zero padded to r_pad for bf16).
+cudaError_t launch_gather_rows(int rows, const int32_t* toks, int V, int r, int r_pad,
+                               int markov_dtype, const void* E, void* Eg, int32_t* status,
+                               int status_div, cudaStream_t s);
+
+struct MergeArgs {
+  int batch, F_prev, F_new, k, beam, S, V, r, r_pad, markov_dtype, depth;
+  Partials part;
+  const int32_t* prev_tok;   // [batch][F_prev] (depth 1: anchors, stride 1)
+  const float* prev_s;       // [batch][F_prev] (depth 1: null -> 0)
+  int prev_stride;           // elements between requests in prev arrays
+  int32_t* lvl_tok;          // [batch][beam] this depth
+  int32_t* lvl_ppos;
+  float* lvl_s;
+  const void* E;
+  void* Eg_next;             // null at the last depth
+  const int32_t* err;
+  int32_t* status;
+};
+cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s);
+
+struct FinalArgs {
+  int batch, D, beam, N;
+  int F[65];                 // F[d] for d = 1..D
+  const int32_t* anchor;
+  const int32_t* lvl_tok;    // [D][batch][beam]
+  const int32_t* lvl_ppos;
+  const float* lvl_s;
+  int32_t *tok, *parent, *depth, *count;
+  float* score;
+  int32_t* status;
+};
+cudaError_t launch_final(const FinalArgs& a, cudaStream_t s);
+
+// pct_score_parents: per-row merge of partials into lse + top-k.
+cudaError_t launch_rows_finalize(int rows, int k, int S, Partials part, float* lse,
+                                 int32_t* top_tok, float* top_logpi, const int32_t* err,
+                                 int32_t* status, int n_par, cudaStream_t s);
+
+}  // namespace pct

@@ -1,0 +1,329 @@
+// PCTree selection kernels: partial merge, per-depth beam, global top-N.
+//
+// PCTree article (qiita), section on the chain draft's weakness and the tree
+// built in its place: after every frontier parent p has been scored,
+// z_d(p) = L_d + Markov(p), each parent keeps its local top-k children,
+// candidates are ranked by s(c) = s(p) + log pi(c|p), each depth is pruned to
+// the beam, and a final global top-N keeps the tree inside the verification
+// budget.
+//
+//  * gather:  Eg[row] = E[token of the row's parent] (the batched Markov call's
+//             A operand for the next depth), zero-padded to the MMA's K tile.
+//  * merge:   one 1024-thread block per request and depth. A warp per parent
+//             row folds the V-slice partials into the row's log-sum-exp and
+//             top-k; the |F| * k candidates are ranked by counting under the
+//             total order (score desc, parent position asc, token asc), the
+//             best `beam` kept and re-ranked into canonical order (parent
+//             position, token), which within one depth is the lexicographic
+//             order of the token paths.
+//  * final:   one block per request; the kept nodes of all depths are ranked
+//             by (score desc, depth asc, canonical position asc), the best N-1
+//             selected, and an exclusive scan over the depth-major flattening
+//             gives every selected node its canonical BFS index; parents are
+//             remapped through the same scan.
+#include <climits>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace pct {
+namespace {
+
+template <typename TE>
+__global__ void gather_rows_kernel(int rows, const int32_t* __restrict__ toks, int V, int r,
+                                   int r_pad, const TE* __restrict__ E, TE* __restrict__ Eg,
+                                   int32_t* __restrict__ status, int status_div) {
+  const int row = blockIdx.x;
+  if (row >= rows) return;
+  int t = toks[row];
+  if (t < 0 || t >= V) {
+    if (threadIdx.x == 0) atomicOr(&status[row / status_div], PCT_DEV_BAD_TOKEN);
+    t = 0;
+  }
+  const TE* src = E + (size_t)t * r;
+  TE* dst = Eg + (size_t)row * r_pad;
+  for (int j = threadIdx.x; j < r_pad; j += blockDim.x) dst[j] = j < r ? src[j] : TE(0.f);
+}
+
+// Fold the S partials of one row (warp-cooperative). Returns lse and writes
+// the row's k best (value desc, token asc) to out_v / out_i (lane 0 holds the
+// full lists after the call; every lane returns the same lse).
+template <int KMAX>
+__device__ __forceinline__ float merge_row(const Partials& part, size_t row, int S, int k,
+                                           float* out_v, int* out_i) {
+  const int lane = threadIdx.x & 31;
+  float m = neg_inf(), s = 0.f;
+  TopK<KMAX> tk;
+  tk.init();
+  for (int sl = lane; sl < S; sl += 32) {
+    const size_t ps = row * S + sl;
+    const float2 ms = part.ms[ps];
+    lse_combine(m, s, ms.x, ms.y);
+    for (int j = 0; j < k; ++j) {
+      const float v = part.val[ps * k + j];
+      const int i = part.idx[ps * k + j];
+      float tv; int ti;
+      tk.kth(k, tv, ti);
+      if (better(v, i, tv, ti)) tk.insert(v, i);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    lse_combine(m, s, m2, s2);
+  }
+  const float lse = (m == neg_inf()) ? neg_inf() : m + logf(s);
+  for (int j = 0; j < k; ++j) {
+    float v = tk.v[0];
+    int i = tk.i[0];
+    warp_best(v, i);
+    if (tk.v[0] == v && tk.i[0] == i) tk.pop();
+    if (lane == 0) { out_v[j] = v; out_i[j] = i; }
+  }
+  return lse;
+}
+
+constexpr int kMergeThreads = 1024;
+constexpr int kMaxCand = 1024;
+
+template <int KMAX, typename TE>
+__global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
+  __shared__ float cs[kMaxCand];
+  __shared__ int cp[kMaxCand], ct[kMaxCand], cpos[kMaxCand];
+  __shared__ float wv[32][16];
+  __shared__ int wi[32][16];
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int F = a.F_prev, k = a.k, C = F * k;
+  if (threadIdx.x == 0 && *a.err) atomicOr(&a.status[b], PCT_DEV_TIMEOUT);
+
+  for (int i = warp; i < F; i += 32) {
+    const size_t row = (size_t)b * F + i;
+    const float lse = merge_row<KMAX>(a.part, row, a.S, k, wv[warp], wi[warp]);
+    __syncwarp();
+    const float sp = a.prev_s ? a.prev_s[(size_t)b * a.prev_stride + i] : 0.f;
+    for (int j = lane; j < k; j += 32) {
+      cs[i * k + j] = sp + (wv[warp][j] - lse);
+      cp[i * k + j] = i;
+      ct[i * k + j] = wi[warp][j];
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+
+  // beam: rank by counting under (score desc, parent position asc, token asc)
+  for (int t = threadIdx.x; t < C; t += blockDim.x) {
+    const float st = cs[t];
+    const int pt = cp[t], tt = ct[t];
+    int rank = 0;
+    for (int u = 0; u < C; ++u) {
+      const float su = cs[u];
+      rank += (su > st) || (su == st && (cp[u] < pt || (cp[u] == pt && ct[u] < tt)));
+    }
+    cpos[t] = rank;
+  }
+  __syncthreads();
+  // canonical order among the kept: (parent position, token)
+  for (int t = threadIdx.x; t < C; t += blockDim.x) {
+    if (cpos[t] >= a.beam) continue;
+    const int pt = cp[t], tt = ct[t];
+    int pos = 0;
+    for (int u = 0; u < C; ++u)
+      pos += cpos[u] < a.beam && (cp[u] < pt || (cp[u] == pt && ct[u] < tt));
+    const size_t o = (size_t)b * a.beam + pos;
+    a.lvl_tok[o] = tt;
+    a.lvl_ppos[o] = pt;
+    a.lvl_s[o] = cs[t];
+  }
+  if (a.Eg_next == nullptr) return;
+  __syncthreads();
+  // next depth's Markov operand rows: Eg[b * F_new + pos] = E[token]
+  const int Fn = a.F_new;
+  const TE* E = static_cast<const TE*>(a.E);
+  TE* Eg = static_cast<TE*>(a.Eg_next);
+  for (int idx = threadIdx.x; idx < Fn * a.r_pad; idx += blockDim.x) {
+    const int pos = idx / a.r_pad, j = idx - pos * a.r_pad;
+    int t = a.lvl_tok[(size_t)b * a.beam + pos];
+    t = (t < 0 || t >= a.V) ? 0 : t;
+    Eg[((size_t)b * Fn + pos) * a.r_pad + j] = j < a.r ? E[(size_t)t * a.r + j] : TE(0.f);
+  }
+}
+
+constexpr int kFinalThreads = 1024;
+constexpr int kMaxUnion = 4096;
+
+__global__ __launch_bounds__(kFinalThreads) void final_kernel(FinalArgs a) {
+  __shared__ float us[kMaxUnion];
+  __shared__ int oidx[kMaxUnion];
+  __shared__ int off[66];
+  __shared__ int sbuf[32];
+  const int b = blockIdx.x;
+  if (threadIdx.x == 0) {
+    off[0] = 0;
+    for (int d = 1; d <= a.D; ++d) off[d] = off[d - 1] + a.F[d];
+  }
+  __syncthreads();
+  const int U = off[a.D];
+  const int keepN = a.N - 1;
+  const size_t lvl_stride = (size_t)a.batch * a.beam;
+  auto depth_of = [&](int u) {
+    int d = 1;
+    while (u >= off[d]) ++d;
+    return d;
+  };
+  for (int u = threadIdx.x; u < U; u += blockDim.x) {
+    const int d = depth_of(u), pos = u - off[d - 1];
+    us[u] = a.lvl_s[(d - 1) * lvl_stride + (size_t)b * a.beam + pos];
+  }
+  __syncthreads();
+  // selection flag: rank under (score desc, depth asc, position asc) < N - 1;
+  // the flattened index u is depth-major, so (depth, position) order is u order
+  constexpr int PER = kMaxUnion / kFinalThreads;
+  int flag[PER];
+  int mine = 0;
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    const int u = threadIdx.x * PER + q;
+    int f = 0;
+    if (u < U) {
+      if (U <= keepN) {
+        f = 1;
+      } else {
+        const float su = us[u];
+        int rank = 0;
+        for (int v = 0; v < U; ++v) rank += (us[v] > su) || (us[v] == su && v < u);
+        f = rank < keepN;
+      }
+    }
+    flag[q] = f;
+    mine += f;
+  }
+  // exclusive scan of the per-thread counts (threads own consecutive u)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) sbuf[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = sbuf[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    sbuf[lane] = w;
+  }
+  __syncthreads();
+  int run = (warp > 0 ? sbuf[warp - 1] : 0) + incl - mine;
+  const int total = sbuf[31];
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    const int u = threadIdx.x * PER + q;
+    if (u < U) oidx[u] = flag[q] ? 1 + run : -1;
+    run += flag[q];
+  }
+  __syncthreads();
+  const size_t ob = (size_t)b * a.N;
+  int bad = 0;
+  for (int u = threadIdx.x; u < U; u += blockDim.x) {
+    const int o = oidx[u];
+    if (o < 0) continue;
+    const int d = depth_of(u), pos = u - off[d - 1];
+    const size_t li = (d - 1) * lvl_stride + (size_t)b * a.beam + pos;
+    int par = 0;
+    if (d > 1) {
+      par = oidx[off[d - 2] + a.lvl_ppos[li]];
+      if (par < 0) { bad = 1; par = 0; }
+    }
+    a.tok[ob + o] = a.lvl_tok[li];
+    a.parent[ob + o] = par;
+    a.depth[ob + o] = d;
+    a.score[ob + o] = us[u];
+  }
+  const int cnt = 1 + total;
+  for (int o = cnt + threadIdx.x; o < a.N; o += blockDim.x) {
+    a.tok[ob + o] = -1; a.parent[ob + o] = -1; a.depth[ob + o] = -1; a.score[ob + o] = neg_inf();
+  }
+  if (threadIdx.x == 0) {
+    a.tok[ob] = a.anchor[b]; a.parent[ob] = -1; a.depth[ob] = 0; a.score[ob] = 0.f;
+    a.count[b] = cnt;
+  }
+  if (bad) atomicOr(&a.status[b], PCT_DEV_BAD_PARENT);
+}
+
+template <int KMAX>
+__global__ void rows_finalize_kernel(int rows, int k, int S, Partials part, float* lse_out,
+                                     int32_t* top_tok, float* top_logpi, const int32_t* err,
+                                     int32_t* status, int n_par) {
+  __shared__ float wv[8][16];
+  __shared__ int wi[8][16];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= rows) return;
+  const float lse = merge_row<KMAX>(part, row, S, k, wv[warp], wi[warp]);
+  __syncwarp();
+  for (int j = lane; j < k; j += 32) {
+    top_tok[(size_t)row * k + j] = wi[warp][j];
+    top_logpi[(size_t)row * k + j] = wv[warp][j] - lse;
+  }
+  if (lane == 0) {
+    lse_out[row] = lse;
+    if (*err) atomicOr(&status[row / n_par], PCT_DEV_TIMEOUT);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gather_rows(int rows, const int32_t* toks, int V, int r, int r_pad,
+                               int markov_dtype, const void* E, void* Eg, int32_t* status,
+                               int status_div, cudaStream_t s) {
+  TraceScope t(s, "gather_rows");
+  if (markov_dtype == PCT_BF16)
+    gather_rows_kernel<__nv_bfloat16><<<rows, 128, 0, s>>>(
+        rows, toks, V, r, r_pad, static_cast<const __nv_bfloat16*>(E),
+        static_cast<__nv_bfloat16*>(Eg), status, status_div);
+  else
+    gather_rows_kernel<float><<<rows, 128, 0, s>>>(rows, toks, V, r, r_pad,
+                                                   static_cast<const float*>(E),
+                                                   static_cast<float*>(Eg), status, status_div);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s) {
+  TraceScope t(s, "pct_merge_beam");
+  const bool bf = a.markov_dtype == PCT_BF16;
+#define PCT_MERGE(KM)                                                                  \
+  (bf ? (merge_kernel<KM, __nv_bfloat16><<<a.batch, kMergeThreads, 0, s>>>(a), 0)      \
+      : (merge_kernel<KM, float><<<a.batch, kMergeThreads, 0, s>>>(a), 0))
+  if (a.k <= 4) PCT_MERGE(4);
+  else if (a.k <= 8) PCT_MERGE(8);
+  else PCT_MERGE(16);
+#undef PCT_MERGE
+  return cudaGetLastError();
+}
+
+cudaError_t launch_final(const FinalArgs& a, cudaStream_t s) {
+  TraceScope t(s, "pct_global_topn");
+  final_kernel<<<a.batch, kFinalThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rows_finalize(int rows, int k, int S, Partials part, float* lse,
+                                 int32_t* top_tok, float* top_logpi, const int32_t* err,
+                                 int32_t* status, int n_par, cudaStream_t s) {
+  TraceScope t(s, "pct_rows_finalize");
+  const int grid = (rows + 7) / 8;
+  if (k <= 4)
+    rows_finalize_kernel<4><<<grid, 256, 0, s>>>(rows, k, S, part, lse, top_tok, top_logpi, err, status, n_par);
+  else if (k <= 8)
+    rows_finalize_kernel<8><<<grid, 256, 0, s>>>(rows, k, S, part, lse, top_tok, top_logpi, err, status, n_par);
+  else
+    rows_finalize_kernel<16><<<grid, 256, 0, s>>>(rows, k, S, part, lse, top_tok, top_logpi, err, status, n_par);
+  return cudaGetLastError();
+}
+
+}  // namespace pct

@@ -1,0 +1,65 @@
+"""Helpers shared by the GPU parity tests (comparison rules, host copies)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+
+SCORE_TOL = 1e-4      # absolute, path scores and log-probabilities
+PHI_RTOL = 1e-4       # relative, Phi(T)
+
+
+def host(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().numpy()
+
+
+def f64(t) -> np.ndarray:
+    return oracle.to_f64(t)
+
+
+def compare_trees(gpu, ref, excluded=None, rows=None, label=""):
+    """Bit-exact node tables and count on non-excluded requests; scores within SCORE_TOL.
+
+    gpu: object with tok/parent/depth/score/count tensors; ref: oracle result.
+    rows: which gpu rows correspond to ref rows (default: all, in order).
+    Returns the number of compared requests.
+    """
+    tok, par, dep, sc, cnt = (host(gpu.tok), host(gpu.parent), host(gpu.depth),
+                              host(gpu.score), host(gpu.count))
+    n_ref = ref.tok.shape[0]
+    rows = list(range(n_ref)) if rows is None else list(rows)
+    excluded = ref.excluded if excluded is None else excluded
+    compared = 0
+    for j, b in enumerate(rows):
+        if excluded[j]:
+            continue
+        n = int(ref.count[j])
+        msg = f"{label} request {b}"
+        assert int(cnt[b]) == n, f"{msg}: count {cnt[b]} != {n}"
+        np.testing.assert_array_equal(tok[b], ref.tok[j], err_msg=msg + " tok")
+        np.testing.assert_array_equal(par[b], ref.parent[j], err_msg=msg + " parent")
+        np.testing.assert_array_equal(dep[b], ref.depth[j], err_msg=msg + " depth")
+        np.testing.assert_allclose(sc[b, :n], ref.score[j, :n], rtol=0, atol=SCORE_TOL,
+                                   err_msg=msg + " score")
+        assert np.isneginf(sc[b, n:]).all(), msg + " padding score"
+        compared += 1
+    return compared
+
+
+def check_tree_invariants(gpu, anchor, n_nodes, label=""):
+    """Properties of any valid output: root, canonical order, parent < child, scores."""
+    tok, par, dep, sc, cnt = (host(gpu.tok), host(gpu.parent), host(gpu.depth),
+                              host(gpu.score), host(gpu.count))
+    anchor = np.asarray(anchor)
+    for b in range(tok.shape[0]):
+        n = int(cnt[b])
+        assert 1 <= n <= n_nodes, label
+        assert tok[b, 0] == anchor[b] and par[b, 0] == -1 and dep[b, 0] == 0 and sc[b, 0] == 0
+        p = par[b, 1:n]
+        assert (p >= 0).all() and (p < np.arange(1, n)).all(), f"{label} parent order {b}"
+        assert (dep[b, 1:n] == dep[b, p] + 1).all()
+        assert (sc[b, 1:n] <= sc[b, p] + 1e-6).all()
+        keys = list(zip(dep[b, 1:n], p, tok[b, 1:n]))
+        assert keys == sorted(keys) and len(set(keys)) == len(keys), f"{label} canonical {b}"
+        assert (tok[b, n:] == -1).all() and (par[b, n:] == -1).all() and (dep[b, n:] == -1).all()

@@ -1,0 +1,109 @@
+"""GPU parity: CaDDTree best-first growth with the greedy stop against the oracle.
+
+"Cost-Aware Diffusion Draft Trees for Speculative Decoding" (gist.science),
+"Method: CaDDTree".
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import speculative_decoding_draft_07_b200 as pct
+import workloads
+from gpu_util import PHI_RTOL, compare_trees, f64, host
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda")
+COST = dict(C_d=1.0, a=2.0, b=1e-4, c=5e-3, e=1e-5)
+
+
+def _sharp_logits(batch, D, V, seed, dtype="bf16", sigma=1.0, peak=(8.0, 16.0)):
+    g = torch.Generator().manual_seed(seed)
+    L = torch.randn((batch, D, V), generator=g) * sigma
+    tok = torch.randint(0, V, (batch, D), generator=g)
+    h = torch.rand((batch, D), generator=g) * (peak[1] - peak[0]) + peak[0]
+    L.scatter_add_(2, tok[..., None], h[..., None])
+    return L.to(torch.bfloat16 if dtype == "bf16" else torch.float32)
+
+
+def _run(L, anchor, ctx, n_max, cost, max_excluded=0.1, label=""):
+    out = pct.cadd_tree_grow(L.to(DEV), torch.as_tensor(anchor, dtype=torch.int32, device=DEV),
+                             torch.as_tensor(ctx, dtype=torch.int64, device=DEV), n_max, **cost)
+    torch.cuda.synchronize()
+    ref = oracle.cadd_tree_grow(f64(L), np.asarray(anchor), np.asarray(ctx), n_max, **cost)
+    n = compare_trees(out, ref, label=label)
+    assert n >= (1 - max_excluded) * len(anchor), f"{label}: {len(anchor) - n} excluded"
+    keep = ~ref.excluded
+    np.testing.assert_allclose(host(out.phi)[keep], ref.phi[keep], rtol=PHI_RTOL, atol=1e-7)
+    assert (host(out.status) == 0).all()
+    return out, ref
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("V,D,n_max", [(512, 6, 64), (1000, 15, 512), (64, 4, 200), (3000, 8, 32)])
+def test_sharp_marginals_deep_trees(dtype, V, D, n_max):
+    batch = 8
+    L = _sharp_logits(batch, D, V, seed=V + D, dtype=dtype)
+    anchor = np.arange(batch) % V
+    ctx = np.array([512, 4096, 32768, 0, 100, 2000, 50000, 7] * (batch // 8 + 1))[:batch]
+    out, ref = _run(L, anchor, ctx, n_max, COST, label=f"sharp V={V}")
+    assert ref.count.max() > 3      # trees actually grow
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_random_convex_costs(seed):
+    rng = np.random.default_rng(seed)
+    batch, D, V = 12, 10, 2048
+    L = _sharp_logits(batch, D, V, seed=100 + seed, sigma=float(rng.uniform(0.5, 2)),
+                      peak=(float(rng.uniform(0, 6)), float(rng.uniform(6, 20))))
+    cost = dict(C_d=float(rng.uniform(0.2, 2)), a=float(rng.uniform(0, 3)), b=float(rng.uniform(0, 1e-3)),
+                c=float(rng.uniform(0, 0.02)), e=float(rng.uniform(0, 1e-4)))
+    _run(L, np.arange(batch), rng.integers(0, 40000, batch), 256, cost, label=f"cost{seed}")
+
+
+def test_stop_disabled_uses_exact_selection_fallback():
+    """c = e = 0: no threshold applies, every token survives the filter (more than the
+    2048-entry buffer), so the exact radix selection of the n_max - 1 best runs."""
+    batch, D, V = 4, 5, 6000
+    L = _sharp_logits(batch, D, V, seed=7, sigma=1.0, peak=(0.0, 3.0))
+    L[0, 0, :] = 0.25          # a row of identical values: ties resolved by token id
+    cost = dict(C_d=1.0, a=1.0, b=0.0, c=0.0, e=0.0)
+    out, ref = _run(L, np.arange(batch), np.zeros(batch), 40, cost, label="fallback")
+    assert (ref.count == 40).all()
+
+
+def test_exhausted_small_vocab():
+    L = _sharp_logits(3, 2, 3, seed=3, sigma=0.5, peak=(0.0, 0.1))
+    cost = dict(C_d=1.0, a=0.0, b=0.0, c=0.0, e=0.0)
+    out, ref = _run(L, [0, 1, 2], [0, 0, 0], 100, cost, label="exhausted")
+    assert (ref.count == 13).all()
+
+
+def test_bad_cost_flagged():
+    L = _sharp_logits(2, 3, 256, seed=4)
+    cost = dict(C_d=-10.0, a=0.0, b=0.0, c=0.01, e=0.0)     # C(n) <= 0 for small n
+    out = pct.cadd_tree_grow(L.to(DEV), torch.tensor([0, 1], dtype=torch.int32, device=DEV),
+                             torch.zeros(2, dtype=torch.int64, device=DEV), 16, **cost)
+    torch.cuda.synchronize()
+    assert (host(out.status) & pct.DEV_BAD_COST).all()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("ell", workloads.CADDTREE.ells)
+def test_caddtree_workload_full_size(ell):
+    """64 requests, V = 151936, D = 15, n_max = 512; the oracle checks 16 of them."""
+    w = workloads.CADDTREE
+    d = workloads.cadd_inputs(w, ell, device=DEV)
+    cost = dict(C_d=w.C_d, a=w.a, b=w.b, c=w.c, e=w.e)
+    out = pct.cadd_tree_grow(d["L"], d["anchor"], d["ctx_len"], w.n_max, **cost)
+    torch.cuda.synchronize()
+    sample = list(range(0, w.batch, 4))
+    Ls = d["L"][sample]
+    ref = oracle.cadd_tree_grow(f64(Ls), host(d["anchor"])[sample], host(d["ctx_len"])[sample],
+                                w.n_max, **cost)
+    n = compare_trees(out, ref, rows=sample, label=f"caddtree l={ell}")
+    assert n >= len(sample) - 1
+    keep = ~ref.excluded
+    np.testing.assert_allclose(host(out.phi)[sample][keep], ref.phi[keep], rtol=PHI_RTOL)
+    counts = host(out.count)
+    assert (counts >= 2).all() and (counts <= w.n_max).all()

@@ -1,0 +1,160 @@
+"""GPU parity: PCTree (batched parent scoring, log-softmax, local top-k, beam,
+global top-N) against the oracle.
+
+PCTree article (qiita), section on the chain draft's weakness and the tree
+built in its place.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import speculative_decoding_draft_07_b200 as pct
+import workloads
+from gpu_util import SCORE_TOL, check_tree_invariants, compare_trees, f64, host
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda")
+
+
+def _problem(batch, D, V, r, seed, dtype="bf16", sigma=2.0, peak=(2.0, 10.0), ew=0.3):
+    g = torch.Generator().manual_seed(seed)
+    L = torch.randn((batch, D, V), generator=g) * sigma
+    pt = torch.randint(0, V, (batch, D), generator=g)
+    ph = torch.rand((batch, D), generator=g) * (peak[1] - peak[0]) + peak[0]
+    L.scatter_add_(2, pt[..., None], ph[..., None])
+    E = torch.randn((V, r), generator=g) * ew
+    W = torch.randn((r, V), generator=g) * ew
+    anchor = torch.randint(0, V, (batch,), generator=g, dtype=torch.int64).to(torch.int32)
+    t = torch.bfloat16 if dtype == "bf16" else torch.float32
+    return L.to(t), anchor, E.to(t), W.to(t)
+
+
+def _score_ref(L_row, ptok, E, W, k):
+    """Oracle per-parent scoring for every request; returns lse, top tokens, log pi,
+    and a mask of rows whose k-th / (k+1)-th values are closer than the tolerance."""
+    Lf, Ef, Wf = f64(L_row), f64(E), f64(W)
+    lse_all, tok_all, lp_all, near_all = [], [], [], []
+    for b in range(Lf.shape[0]):
+        Z, markov, logpi, lse, order = oracle.score_parents(Lf[b], ptok[b], Ef, Wf, k)
+        rows = np.arange(Z.shape[0])[:, None]
+        top = order[:, :k]
+        lse_all.append(lse)
+        tok_all.append(top)
+        lp_all.append(logpi[rows, top])
+        if order.shape[1] > k:
+            zk, zk1 = Z[rows[:, 0], order[:, k - 1]], Z[rows[:, 0], order[:, k]]
+            near = (np.abs(zk - zk1) < SCORE_TOL)
+        else:
+            near = np.zeros(Z.shape[0], bool)
+        # near ties inside the top-k permute tokens too; compare those rows as sets
+        zs = Z[rows, order[:, :k]]
+        near_in = (np.abs(np.diff(zs, axis=1)) < SCORE_TOL).any(axis=1) if k > 1 else np.zeros_like(near)
+        near_all.append((near, near_in))
+    return (np.stack(lse_all), np.stack(tok_all), np.stack(lp_all), near_all)
+
+
+@pytest.mark.parametrize("dtype,V,r,k,batch,n_par", [
+    ("bf16", 1024, 64, 4, 1, 1), ("bf16", 1024, 16, 8, 3, 40), ("bf16", 2048, 100, 8, 2, 200),
+    ("bf16", 4096, 256, 16, 3, 100), ("bf16", 64, 64, 1, 2, 5), ("bf16", 1000, 256, 8, 1, 130),
+    ("f32", 1000, 16, 4, 2, 7), ("f32", 777, 33, 8, 3, 20)])
+def test_score_parents_matches_oracle(dtype, V, r, k, batch, n_par):
+    L, _, E, W = _problem(batch, 1, V, r, seed=V + r + k, dtype=dtype)
+    L = L[:, 0, :].contiguous()
+    g = torch.Generator().manual_seed(k)
+    ptok = torch.randint(0, V, (batch, n_par), generator=g, dtype=torch.int64).to(torch.int32)
+    lse, tt, tl, st = pct.pct_score_parents(L.to(DEV), ptok.to(DEV), E.to(DEV), W.to(DEV), k)
+    torch.cuda.synchronize()
+    rl, rt, rlp, near = _score_ref(L, ptok.numpy(), E, W, k)
+    np.testing.assert_allclose(host(lse), rl, rtol=0, atol=SCORE_TOL)
+    gt, gl = host(tt), host(tl)
+    skipped = 0
+    for b in range(batch):
+        nb, nin = near[b]
+        for p in range(n_par):
+            if nb[p]:
+                skipped += 1
+                continue
+            if nin[p]:
+                assert sorted(gt[b, p]) == sorted(rt[b, p])
+            else:
+                np.testing.assert_array_equal(gt[b, p], rt[b, p], err_msg=f"row {b},{p}")
+            np.testing.assert_allclose(gl[b, p], rlp[b, p], rtol=0, atol=SCORE_TOL)
+    assert skipped <= max(1, batch * n_par // 50)
+    assert (host(st) == 0).all()
+
+
+def _build_and_compare(L, anchor, E, W, k, beam, N, sample=None, max_excluded=0.2, label=""):
+    out = pct.pct_tree_build(L.to(DEV), anchor.to(DEV), E.to(DEV), W.to(DEV), k, beam, N)
+    torch.cuda.synchronize()
+    check_tree_invariants(out, anchor.numpy(), N, label)
+    rows = list(range(L.shape[0])) if sample is None else list(sample)
+    ref = oracle.pct_tree_build(f64(L[rows]), anchor.numpy()[rows], f64(E), f64(W), k, beam, N)
+    n = compare_trees(out, ref, rows=rows, label=label)
+    assert n >= (1 - max_excluded) * len(rows), f"{label}: {len(rows) - n} excluded of {len(rows)}"
+    assert (host(out.status) == 0).all()
+    return out, ref
+
+
+def test_tiny_workload_fp32():
+    w = workloads.WORKLOADS["tiny"]
+    d = workloads.drafter_inputs(w)
+    out, ref = _build_and_compare(d["L"], d["anchor"], d["E"], d["W"], w.k, w.beam, w.n_nodes,
+                                  max_excluded=0.0, label="tiny")
+    assert host(out.count)[0] == 25
+
+
+@pytest.mark.parametrize("dtype,V,D,r,k,beam,N,batch", [
+    ("bf16", 2048, 4, 64, 4, 8, 32, 4), ("bf16", 1024, 6, 256, 8, 16, 64, 3),
+    ("bf16", 4096, 5, 100, 8, 32, 128, 5), ("bf16", 512, 8, 32, 2, 5, 40, 6),
+    ("bf16", 3000, 3, 16, 16, 64, 200, 2), ("f32", 1500, 5, 24, 4, 8, 40, 4),
+    ("f32", 1000, 6, 16, 3, 6, 30, 3)])
+def test_small_builds_match_oracle(dtype, V, D, r, k, beam, N, batch):
+    L, anchor, E, W = _problem(batch, D, V, r, seed=V + D + r, dtype=dtype)
+    _build_and_compare(L, anchor, E, W, k, beam, N, label=f"{dtype} V={V}")
+
+
+def test_k1_is_the_greedy_chain_on_gpu():
+    L, anchor, E, W = _problem(4, 6, 1024, 64, seed=9)
+    out, ref = _build_and_compare(L, anchor, E, W, 1, 4, 7, label="chain")
+    assert (host(out.count) == 7).all()
+    assert (host(out.parent)[:, 1:] == np.arange(6)).all()
+
+
+def test_zero_markov_exact_ties():
+    """W = 0: every parent of a depth sees the same row, many exact ties in bf16."""
+    L, anchor, E, W = _problem(3, 5, 1024, 64, seed=11, sigma=1.0)
+    W = torch.zeros_like(W)
+    L[0, 1, 10:20] = 6.0          # ten identical peaks
+    _build_and_compare(L, anchor, E, W, 8, 16, 64, max_excluded=0.0, label="w0")
+
+
+def test_repeated_builds_are_bit_identical():
+    L, anchor, E, W = _problem(4, 6, 2048, 64, seed=13)
+    Ld, ad, Ed, Wd = L.to(DEV), anchor.to(DEV), E.to(DEV), W.to(DEV)
+    first = pct.pct_tree_build(Ld, ad, Ed, Wd, 8, 16, 64)
+    ref = [host(x).copy() for x in (first.tok, first.parent, first.score, first.count)]
+    for _ in range(10):
+        o = pct.pct_tree_build(Ld, ad, Ed, Wd, 8, 16, 64)
+        for x, y in zip(ref, (o.tok, o.parent, o.score, o.count)):
+            np.testing.assert_array_equal(x, host(y))
+
+
+@pytest.mark.slow
+def test_qwen3_4b_scale_workload():
+    """V = 151936, B = 7, r = 256, k = 8, beam 16, N = 64, one request: full oracle."""
+    w = workloads.WORKLOADS["qwen3_4b_scale"]
+    d = workloads.drafter_inputs(w, device=DEV)
+    L, a, E, W = (d[x].cpu() for x in ("L", "anchor", "E", "W"))
+    _build_and_compare(L, a, E, W, w.k, w.beam, w.n_nodes, max_excluded=0.0, label="qwen3_4b")
+
+
+@pytest.mark.slow
+def test_long_block_workload_sampled():
+    """V = 151936, B = 16, r = 256, k = 8, beam 32, N = 128, 32 requests; the oracle
+    checks 4 sampled requests, every request is checked for the output invariants."""
+    w = workloads.WORKLOADS["long_block"]
+    d = workloads.drafter_inputs(w, device=DEV)
+    L, a, E, W = (d[x].cpu() for x in ("L", "anchor", "E", "W"))
+    _build_and_compare(L, a, E, W, w.k, w.beam, w.n_nodes, sample=[0, 9, 18, 31],
+                       max_excluded=0.25, label="long_block")

@@ -13,7 +13,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 MUTATIONS = [
     # (file, original text, planted mistake, pin file)
-    ("pctree.py", "Z = L[d - 1][None, :] + markov", "Z = L[d - 1][None, :] - markov",
+    ("pctree.py", "Z = L_d[None, :] + markov", "Z = L_d[None, :] - markov",
      "test_oracle_pctree.py"),                                     # wrong sign
     ("pctree.py", "markov = E[toks] @ W", "markov = E[toks * 0] @ W",
      "test_oracle_pctree.py"),                                     # wrong parent index
@@ -23,7 +23,7 @@ MUTATIONS = [
      "test_oracle_pctree.py"),                                     # top-k from the wrong end
     ("pctree.py", "key=lambda c: (-c.s, c.depth, c.path)", "key=lambda c: (c.s, c.depth, c.path)",
      "test_oracle_pctree.py"),                                     # global top-N reversed
-    ("pctree.py", "Z = L[d - 1][None, :]", "Z = L[(d) % D][None, :]",
+    ("pctree.py", "score_parents(L[d - 1],", "score_parents(L[d % D],",
      "test_oracle_pctree.py"),                                     # depth off by one
     ("numerics.py", "lse = m_safe + np.log(", "lse = np.log(",
      "test_oracle_numerics.py"),                                   # dropped max shift

@@ -208,6 +208,34 @@ int32_t tree_verify_accept(int32_t batch, int32_t n_stride, int32_t vocab, int32
                            void* cuda_stream);
 
 /* ------------------------------------------------------------------------ *
+ * Allocation-free variant of tree_verify_accept. The pages have no
+ * counterpart to this call: it exists for users of the library whose code
+ * cannot allocate device memory -- for example a component inside a serving
+ * runtime that reserves all device memory up front and hands its parts only
+ * their input and output buffers, or code on a latency-critical path where a
+ * cudaMalloc (which may synchronise the device) is not acceptable.
+ *
+ * Same arguments, results and errors as tree_verify_accept, minus the
+ * workspace. The scratch it needs (one 32-bit arrival counter per request)
+ * lives in a file-scope device array of PCT_NOALLOC_MAX_BATCH counters
+ * (16 KB), which every GPU that loads the library holds until the process
+ * exits. batch > PCT_NOALLOC_MAX_BATCH returns PCT_EUNSUPPORTED before
+ * anything is launched. The call allocates nothing; it clears the counters it
+ * uses on its stream before the kernel runs.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls share the one array: two calls that can run at the same time on
+ *     the GPU (for example on different streams) race on it and give undefined
+ *     results. Order them on one stream or with events.
+ * ------------------------------------------------------------------------ */
+#define PCT_NOALLOC_MAX_BATCH 4096
+int32_t tree_verify_accept_noalloc(int32_t batch, int32_t n_stride, int32_t vocab,
+                                   int32_t max_depth, const int32_t* tok, const int32_t* parent,
+                                   const int32_t* count, const void* target, int32_t target_dtype,
+                                   int32_t* argmax, int32_t* accept_len, int32_t* accept_path,
+                                   int32_t* correction, int32_t* dev_status, void* cuda_stream);
+
+/* ------------------------------------------------------------------------ *
  * Kernel trace (off by default; host-side bookkeeping only). While on, every
  * kernel the library launches is bracketed by two CUDA events on its stream
  * and the elapsed time is accumulated per kernel name. Not for use inside

@@ -28,7 +28,7 @@ EXPORTED = [
     "pct_tree_build_workspace", "pct_tree_build", "pct_score_parents_workspace",
     "pct_score_parents", "cadd_tree_grow_workspace", "cadd_tree_grow", "tree_ancestor_mask",
     "tree_verify_accept_workspace", "tree_verify_accept", "pct_trace_enable", "pct_trace_reset",
-    "pct_trace_read", "pct_version",
+    "pct_trace_read", "pct_version", "tree_verify_accept_noalloc",
 ]
 
 
@@ -81,6 +81,8 @@ def lib() -> ctypes.CDLL:
         "pct_trace_reset": (i32, []),
         "pct_trace_read": (i32, [ctypes.c_char_p, i32, vp, vp, i32]),
         "pct_version": (ctypes.c_char_p, []),
+        "tree_verify_accept_noalloc": (i32, [i32, i32, i32, i32, vp, vp, vp, vp, i32, vp, vp, vp,
+                                             vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)

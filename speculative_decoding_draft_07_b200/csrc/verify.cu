@@ -16,6 +16,7 @@
 // (arrival counter) performs that request's accept walk, so no second launch
 // and no grid-wide wait is needed.
 #include <climits>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -306,3 +307,67 @@ cudaError_t launch_verify(int batch, int n_stride, int vocab, int max_depth, con
 }
 
 }  // namespace pct
+
+// ---------------------------------------------------------------------------
+// Allocation-free verification entry point.
+//
+// For callers that cannot allocate device memory (see the header): the only
+// scratch the verification kernel needs, one arrival counter per request,
+// lives in this file-scope device array instead of a caller workspace. Every
+// GPU that loads the library holds it (16 KB) until the process exits, and
+// every call shares it.
+namespace pct {
+namespace {
+
+__device__ __align__(256) unsigned g_noalloc_arrive[PCT_NOALLOC_MAX_BATCH];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of the counters on the current device, looked up once per
+// device (host code may not use the array's name as a device pointer).
+int noalloc_counters(unsigned** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PCT_ECUDA;
+  if (dev < 0 || dev >= 64) return PCT_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_arrive) != cudaSuccess || p == nullptr) return PCT_ECUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = static_cast<unsigned*>(g_noalloc_ptr[dev]);
+  return PCT_OK;
+}
+
+}  // namespace
+}  // namespace pct
+
+extern "C" int32_t tree_verify_accept_noalloc(int32_t batch, int32_t n_stride, int32_t vocab,
+                                              int32_t max_depth, const int32_t* tok,
+                                              const int32_t* parent, const int32_t* count,
+                                              const void* target, int32_t target_dtype,
+                                              int32_t* argmax, int32_t* accept_len,
+                                              int32_t* accept_path, int32_t* correction,
+                                              int32_t* dev_status, void* cuda_stream) {
+  if (batch < 1 || n_stride < 1 || n_stride > 4096) return PCT_EINVAL;
+  if (batch > PCT_NOALLOC_MAX_BATCH) return PCT_EUNSUPPORTED;
+  if (vocab < 1 || max_depth < 1 || max_depth > 4096) return PCT_EINVAL;
+  if (target_dtype != PCT_F32 && target_dtype != PCT_BF16) return PCT_EINVAL;
+  if (!tok || !parent || !count || !target || !argmax || !accept_len || !accept_path ||
+      !correction || !dev_status)
+    return PCT_EINVAL;
+  if (!pct::device_ok()) return PCT_EDEVICE;
+  unsigned* arrive = nullptr;
+  const int st = pct::noalloc_counters(&arrive);
+  if (st != PCT_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  // the counters keep the previous call's contents: clear the ones this call uses
+  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t) * batch, s) != cudaSuccess) return PCT_ECUDA;
+  if (cudaMemsetAsync(arrive, 0, sizeof(unsigned) * batch, s) != cudaSuccess) return PCT_ECUDA;
+  if (pct::launch_verify(batch, n_stride, vocab, max_depth, tok, parent, count, target,
+                         target_dtype, argmax, accept_len, accept_path, correction, dev_status,
+                         arrive, s) != cudaSuccess)
+    return PCT_ECUDA;
+  return PCT_OK;
+}

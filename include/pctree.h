@@ -86,7 +86,7 @@ enum {
 typedef struct {
   int32_t batch;        /* independent requests, >= 1                          */
   int32_t depth;        /* D, drafted depths (block size B = D + 1), 1..64      */
-  int32_t vocab;        /* V, >= k                                              */
+  int32_t vocab;        /* V, k..4194304 (2^22)                                  */
   int32_t rank;         /* r of E [V][r] and W [r][V], 1..256                   */
   int32_t k;            /* local top-k children per parent, 1..16              */
   int32_t beam;         /* frontier width kept per depth, 1..256, beam*k <= 1024 */

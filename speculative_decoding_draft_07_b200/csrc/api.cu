@@ -116,6 +116,7 @@ int check_build_desc(const pct_build_desc* d) {
   if (d->n_nodes < 1 || d->n_nodes > 4096 || d->depth * d->beam > 4096) return PCT_EINVAL;
   if (!dtype_ok(d->logits_dtype) || !dtype_ok(d->markov_dtype)) return PCT_EINVAL;
   if (d->markov_dtype == PCT_BF16 && d->vocab % 8 != 0) return PCT_EUNSUPPORTED;
+  if (d->vocab > (1 << 22)) return PCT_EUNSUPPORTED;   // token ids packed into 22-bit key fields
   return PCT_OK;
 }
 

@@ -8,10 +8,12 @@
 // non-positive.
 //
 // Two kernels:
-//  * row pass, one 512-thread block per (request, depth) row of marginal
-//    logits: log-sum-exp in one streaming pass, then a second pass (the row was
-//    just read and normally still sits in L2) that keeps only the tokens that
-//    can ever enter the tree. A node is added at size n only if its prefix
+//  * row pass, one 256-thread block per (request, depth) row of marginal
+//    logits, streamed once from HBM in 32 KB register chunks: a running
+//    log-sum-exp of the block (a lower bound of the row's) gives after every
+//    chunk a threshold with which the chunk's survivors are taken straight from
+//    registers; a final exact filter keeps only the tokens that can ever enter
+//    the tree. A node is added at size n only if its prefix
 //    probability p satisfies p > (1 + Phi) dC(n) / C(n) >= theta, where
 //    theta = min_n dC(n) / C(n) and dC(n) = C(n + 1) - C(n); since p never
 //    exceeds the marginal q_d of its last token, tokens with q_d <= theta can
@@ -32,7 +34,8 @@
 namespace pct {
 namespace {
 
-constexpr int kRowThreads = 512;
+constexpr int kRowThreads = 256;
+constexpr int kChunk = 8;             // 16-byte loads per thread per chunk (32 KB per block)
 constexpr int kCap = 2048;          // candidate buffer per row (power of two)
 constexpr float kThetaSlack = 1e-3f;
 
@@ -132,6 +135,39 @@ __device__ __forceinline__ void for_row(const T* x, int V, bool vec, F&& f) {
   }
 }
 
+// theta = min over n in [1, n_max - 1] of dC(n) / C(n) for request b, computed
+// by one warp in double; returns ln(theta) (-inf when some dC(n) <= 0, i.e. no
+// token can be excluded) and reports C(n) <= 0 in the status word.
+__device__ float cadd_ln_theta(const CaddParams& p, double ell, int lane, bool report,
+                               int32_t* status_b) {
+  const double cb = (double)p.C_d + (double)p.a + (double)p.b * ell;
+  double th = 1e300;
+  int bad = 0, nonpos = 0;
+  for (int n = 1 + lane; n <= p.n_max; n += 32) {
+    const double Cn = cb + (double)p.c * n + (double)p.e * (double)n * n;
+    if (Cn <= 0.0) bad = 1;
+    if (n < p.n_max) {
+      const double dC = (double)p.c + (double)p.e * (2.0 * n + 1.0);
+      if (dC <= 0.0) nonpos = 1; else if (Cn > 0.0) th = fmin(th, dC / Cn);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    th = fmin(th, __shfl_xor_sync(0xffffffffu, th, o));
+    bad |= __shfl_xor_sync(0xffffffffu, bad, o);
+    nonpos |= __shfl_xor_sync(0xffffffffu, nonpos, o);
+  }
+  if (report && lane == 0 && bad) atomicOr(status_b, PCT_DEV_BAD_COST);
+  return (nonpos || th >= 1e299) ? neg_inf() : (float)log(th);
+}
+
+// Keep (value, token) in the candidate buffer; the counter keeps counting past
+// the capacity so that an overflow is detected.
+__device__ __forceinline__ void cadd_keep(unsigned long long* keys, int* n, float z, int v) {
+  const int pos = atomicAdd(n, 1);
+  if (pos < kCap) keys[pos] = cand_key(z, v);
+}
+
 template <typename T>
 __global__ __launch_bounds__(kRowThreads) void cadd_rowpass_kernel(
     CaddParams p, const T* __restrict__ L, const int64_t* __restrict__ ctx,
@@ -141,7 +177,7 @@ __global__ __launch_bounds__(kRowThreads) void cadd_rowpass_kernel(
   __shared__ float sm[32], ss[32];
   __shared__ int sbuf[32];
   __shared__ int hist[256];
-  __shared__ int s_n, s_tot;
+  __shared__ int s_n, s_n2;
   __shared__ float s_lnth;
   const int d = blockIdx.x, b = blockIdx.y;
   const int V = p.V;
@@ -151,79 +187,117 @@ __global__ __launch_bounds__(kRowThreads) void cadd_rowpass_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool vec = (sizeof(T) == 2) && (V % 8 == 0) && ((reinterpret_cast<uintptr_t>(L) & 15u) == 0);
 
-  // theta for this request: min over n in [1, n_max - 1] of dC(n) / C(n)
   if (warp == 0) {
-    const double ell = (double)ctx[b];
-    const double cb = (double)p.C_d + (double)p.a + (double)p.b * ell;
-    double th = 1e300;
-    int bad = 0, nonpos = 0;
-    for (int n = 1 + lane; n <= p.n_max; n += 32) {
-      const double Cn = cb + (double)p.c * n + (double)p.e * (double)n * n;
-      if (Cn <= 0.0) bad = 1;
-      if (n < p.n_max) {
-        const double dC = (double)p.c + (double)p.e * (2.0 * n + 1.0);
-        if (dC <= 0.0) nonpos = 1; else if (Cn > 0.0) th = fmin(th, dC / Cn);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      th = fmin(th, __shfl_xor_sync(0xffffffffu, th, o));
-      bad |= __shfl_xor_sync(0xffffffffu, bad, o);
-      nonpos |= __shfl_xor_sync(0xffffffffu, nonpos, o);
-    }
-    if (lane == 0) {
-      if (bad && d == 0) atomicOr(&status[b], PCT_DEV_BAD_COST);
-      s_lnth = (nonpos || th >= 1e299) ? neg_inf() : (float)log(th);
-      s_n = 0;
-    }
+    const float lt = cadd_ln_theta(p, (double)ctx[b], lane, d == 0, &status[b]);
+    if (lane == 0) { s_lnth = lt; s_n = 0; }
   }
+  __syncthreads();
+  const float lnth = s_lnth - kThetaSlack;
 
-  // pass 1: log-sum-exp
+  // One pass over the row in chunks held in registers. After each chunk the
+  // block's running log-sum-exp (a lower bound of the row's, which only grows)
+  // gives a threshold that every final candidate already passes, so the
+  // chunk's survivors are taken from registers without a second read.
   float m = neg_inf(), s = 0.f;
   if (vec) {
     const uint4* pv = reinterpret_cast<const uint4*>(x);
     const int nvec = V >> 3;
-    for (int c = threadIdx.x; c < nvec; c += kRowThreads) {
-      const uint4 q = ld_stream16(pv + c);
-      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-      float cm = neg_inf();
+    // uniform trip count: block_lse below synchronises the whole block
+    for (int c0 = 0; c0 < nvec; c0 += kRowThreads * kChunk) {
+      const int base = c0 + threadIdx.x;
+      uint4 q[kChunk];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) cm = fmaxf(cm, fmaxf(bf16_lo(w[j]), bf16_hi(w[j])));
-      if (cm > m) { s = (m == neg_inf()) ? 0.f : s * ex2((m - cm) * kLog2e); m = cm; }
-      if (m != neg_inf()) {
-        const float mb = m * kLog2e;
+      for (int u = 0; u < kChunk; ++u) {
+        const int c = base + u * kRowThreads;
+        q[u] = c < nvec ? ld_stream16(pv + c)
+                        : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+      }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          s += ex2(fmaf(bf16_lo(w[j]), kLog2e, -mb));
-          s += ex2(fmaf(bf16_hi(w[j]), kLog2e, -mb));
+      for (int u = 0; u < kChunk; ++u) {
+        const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+        float cm = neg_inf();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cm = fmaxf(cm, fmaxf(bf16_lo(w[j]), bf16_hi(w[j])));
+        if (cm > m) { s = (m == neg_inf()) ? 0.f : s * ex2((m - cm) * kLog2e); m = cm; }
+        if (m != neg_inf()) {
+          const float mb = m * kLog2e;
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            s0 += ex2(fmaf(bf16_lo(w[j]), kLog2e, -mb));
+            s1 += ex2(fmaf(bf16_hi(w[j]), kLog2e, -mb));
+          }
+          s += s0 + s1;
+        }
+      }
+      // running block log-sum-exp -> chunk threshold
+      float bm = m, bs = s;
+      block_lse(bm, bs, sm, ss);
+      const float t = (K <= 0 || bm == neg_inf()) ? __int_as_float(0x7f800000)
+                                                  : bm + logf(bs) + lnth;
+#pragma unroll
+      for (int u = 0; u < kChunk; ++u) {
+        const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+        float cm = neg_inf();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cm = fmaxf(cm, fmaxf(bf16_lo(w[j]), bf16_hi(w[j])));
+        if (cm > t) {
+          const int v0 = (base + u * kRowThreads) * 8;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float z = (j & 1) ? bf16_hi(w[j >> 1]) : bf16_lo(w[j >> 1]);
+            if (z > t) cadd_keep(keys, &s_n, z, v0 + j);
+          }
         }
       }
     }
-    for (int v = (nvec << 3) + threadIdx.x; v < V; v += kRowThreads) {
-      const float z = elem(x, v);
-      lse_combine(m, s, z, 1.f);
-    }
+    // tail (V % 8 values): scalar, folded into the totals below
+    for (int v = (nvec << 3) + threadIdx.x; v < V; v += kRowThreads) lse_combine(m, s, elem(x, v), 1.f);
   } else {
     for (int v = threadIdx.x; v < V; v += kRowThreads) lse_combine(m, s, elem(x, v), 1.f);
   }
   block_lse(m, s, sm, ss);
   const float lse = (m == neg_inf()) ? neg_inf() : m + logf(s);
-  // s_lnth was written before the block_lse barriers
-  const float t = (K <= 0) ? __int_as_float(0x7f800000) : lse + s_lnth - kThetaSlack;
-
-  // pass 2: survivors above the threshold (normally served from L2)
+  const float t = (K <= 0) ? __int_as_float(0x7f800000) : lse + lnth;
+  // scalar paths (tail or non-vector rows) collect against the exact threshold
   if (K > 0) {
-    for_row(x, V, vec, [&](float z, int v) {
-      if (z > t) {
-        const int pos = atomicAdd(&s_n, 1);
-        if (pos < kCap) keys[pos] = cand_key(z, v);
+    if (vec) {
+      for (int v = ((V >> 3) << 3) + threadIdx.x; v < V; v += kRowThreads) {
+        const float z = elem(x, v);
+        if (z > t) cadd_keep(keys, &s_n, z, v);
       }
-    });
+    } else {
+      for (int v = threadIdx.x; v < V; v += kRowThreads) {
+        const float z = elem(x, v);
+        if (z > t) cadd_keep(keys, &s_n, z, v);
+      }
+    }
   }
   __syncthreads();
   int n = s_n;
-  if (n > kCap) {
-    // exact radix select of the K best (value desc, token asc) over the row
+  if (n <= kCap) {
+    // exact filter of the chunk survivors against the final threshold
+    if (threadIdx.x == 0) s_n2 = 0;
+    __syncthreads();
+    unsigned long long mine[kCap / kRowThreads];
+    int cntm = 0;
+#pragma unroll
+    for (int u = 0; u < kCap / kRowThreads; ++u) {
+      const int j = threadIdx.x + u * kRowThreads;
+      if (j < n) {
+        const unsigned long long kk = keys[j];
+        if (ord2f((unsigned)(kk >> 32)) > t) mine[cntm++] = kk;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kCap / kRowThreads; ++u)
+      if (u < cntm) keys[atomicAdd(&s_n2, 1)] = mine[u];
+    __syncthreads();
+    n = s_n2;
+  } else {
+    // more than the buffer survived (theta tiny): exact radix select of the K
+    // best (value desc, token asc) over the row
     unsigned prefix = 0, pmask = 0;
     int need = K;
     for (int shift = 24; shift >= 0; shift -= 8) {

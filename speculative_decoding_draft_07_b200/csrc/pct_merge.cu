@@ -9,13 +9,13 @@
 //
 //  * gather:  Eg[row] = E[token of the row's parent] (the batched Markov call's
 //             A operand for the next depth), zero-padded to the MMA's K tile.
-//  * merge:   one 1024-thread block per request and depth. A warp per parent
+//  * merge:   one 512-thread block per request and depth. A warp per parent
 //             row folds the V-slice partials into the row's log-sum-exp and
-//             top-k; the |F| * k candidates are ranked by counting under the
-//             total order (score desc, parent position asc, token asc), the
-//             best `beam` kept and re-ranked into canonical order (parent
-//             position, token), which within one depth is the lexicographic
-//             order of the token paths.
+//             top-k; the |F| * k candidates become 64-bit keys ordered by the
+//             total order (score desc, parent position asc, token asc) and are
+//             bitonic-sorted; the best `beam` are re-sorted into canonical
+//             order (parent position, token), which within one depth is the
+//             lexicographic order of the token paths.
 //  * final:   one block per request; the kept nodes of all depths are ranked
 //             by (score desc, depth asc, canonical position asc), the best N-1
 //             selected, and an exclusive scan over the depth-major flattening
@@ -46,8 +46,10 @@ __global__ void gather_rows_kernel(int rows, const int32_t* __restrict__ toks, i
 }
 
 // Fold the S partials of one row (warp-cooperative). Returns lse and writes
-// the row's k best (value desc, token asc) to out_v / out_i (lane 0 holds the
-// full lists after the call; every lane returns the same lse).
+// the row's k best (value desc, token asc) to out_v / out_i. Every slice's
+// list is already sorted, so with S <= 32 each lane holds one slice's list and
+// the merge is k rounds of "take the best head, the owner pops"; with S > 32 a
+// lane first folds its slices by insertion.
 template <int KMAX>
 __device__ __forceinline__ float merge_row(const Partials& part, size_t row, int S, int k,
                                            float* out_v, int* out_i) {
@@ -59,12 +61,23 @@ __device__ __forceinline__ float merge_row(const Partials& part, size_t row, int
     const size_t ps = row * S + sl;
     const float2 ms = part.ms[ps];
     lse_combine(m, s, ms.x, ms.y);
-    for (int j = 0; j < k; ++j) {
-      const float v = part.val[ps * k + j];
-      const int i = part.idx[ps * k + j];
-      float tv; int ti;
-      tk.kth(k, tv, ti);
-      if (better(v, i, tv, ti)) tk.insert(v, i);
+    float v[KMAX];
+    int id[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      v[j] = j < k ? part.val[ps * k + j] : neg_inf();
+      id[j] = j < k ? part.idx[ps * k + j] : 0x7fffffff;
+    }
+    if (sl == lane) {          // first slice of this lane: already sorted
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) { tk.v[j] = v[j]; tk.i[j] = id[j]; }
+    } else {
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        float tv; int ti;
+        tk.kth(k, tv, ti);
+        if (j < k && better(v[j], id[j], tv, ti)) tk.insert(v[j], id[j]);
+      }
     }
   }
 #pragma unroll
@@ -73,7 +86,9 @@ __device__ __forceinline__ float merge_row(const Partials& part, size_t row, int
     lse_combine(m, s, m2, s2);
   }
   const float lse = (m == neg_inf()) ? neg_inf() : m + logf(s);
-  for (int j = 0; j < k; ++j) {
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    if (j >= k) break;
     float v = tk.v[0];
     int i = tk.i[0];
     warp_best(v, i);
@@ -83,69 +98,112 @@ __device__ __forceinline__ float merge_row(const Partials& part, size_t row, int
   return lse;
 }
 
-constexpr int kMergeThreads = 1024;
+constexpr int kMergeThreads = 512;
 constexpr int kMaxCand = 1024;
+
+// Descending bitonic sort of keys[0..P) (P a power of two) by the block.
+__device__ void bitonic_desc_block(unsigned long long* keys, int P) {
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = threadIdx.x; t < P / 2; t += blockDim.x) {
+        const int lo = 2 * t - (t & (stride - 1));
+        const int hi = lo + stride;
+        const bool desc = ((lo & size) == 0);
+        const unsigned long long x = keys[lo], y = keys[hi];
+        if (desc ? (x < y) : (x > y)) { keys[lo] = y; keys[hi] = x; }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// Candidate key: larger = better under (score desc, parent position asc,
+// token asc); tokens < 2^22, parent positions < 1024.
+__device__ __forceinline__ unsigned long long cand_key(float s, int ppos, int tok) {
+  return ((unsigned long long)f2ord(s) << 32) | ((unsigned long long)(1023 - ppos) << 22) |
+         (unsigned long long)(0x3fffff - tok);
+}
 
 template <int KMAX, typename TE>
 __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
-  __shared__ float cs[kMaxCand];
-  __shared__ int cp[kMaxCand], ct[kMaxCand], cpos[kMaxCand];
-  __shared__ float wv[32][16];
-  __shared__ int wi[32][16];
+  __shared__ unsigned long long keys[kMaxCand];
+  __shared__ unsigned long long ck[256];
+  __shared__ float kept_s[256];
+  __shared__ float wv[kMergeThreads / 32][16];
+  __shared__ int wi[kMergeThreads / 32][16];
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = kMergeThreads / 32;
   const int F = a.F_prev, k = a.k, C = F * k;
   if (threadIdx.x == 0 && *a.err) atomicOr(&a.status[b], PCT_DEV_TIMEOUT);
 
-  for (int i = warp; i < F; i += 32) {
+  // candidates (score, parent position, token) as ordered keys, a warp per parent row
+  for (int i = warp; i < F; i += nwarps) {
     const size_t row = (size_t)b * F + i;
     const float lse = merge_row<KMAX>(a.part, row, a.S, k, wv[warp], wi[warp]);
     __syncwarp();
     const float sp = a.prev_s ? a.prev_s[(size_t)b * a.prev_stride + i] : 0.f;
-    for (int j = lane; j < k; j += 32) {
-      cs[i * k + j] = sp + (wv[warp][j] - lse);
-      cp[i * k + j] = i;
-      ct[i * k + j] = wi[warp][j];
-    }
+    for (int j = lane; j < k; j += 32) keys[i * k + j] = cand_key(sp + (wv[warp][j] - lse), i, wi[warp][j]);
     __syncwarp();
   }
+  int P = 1;
+  while (P < C) P <<= 1;
+  for (int t = C + threadIdx.x; t < P; t += blockDim.x) keys[t] = 0ull;
   __syncthreads();
-
-  // beam: rank by counting under (score desc, parent position asc, token asc)
-  for (int t = threadIdx.x; t < C; t += blockDim.x) {
-    const float st = cs[t];
-    const int pt = cp[t], tt = ct[t];
-    int rank = 0;
-    for (int u = 0; u < C; ++u) {
-      const float su = cs[u];
-      rank += (su > st) || (su == st && (cp[u] < pt || (cp[u] == pt && ct[u] < tt)));
+  // beam: the best `beam` candidates under (score desc, parent position asc, token asc)
+  bitonic_desc_block(keys, P);
+  const int kept = min(a.beam, C);
+  // canonical order of the kept: ascending (parent position, token); the beam
+  // rank rides along in the low bits to find the score again
+  int Q = 1;
+  while (Q < kept) Q <<= 1;
+  for (int t = threadIdx.x; t < Q; t += blockDim.x) {
+    if (t < kept) {
+      const unsigned long long x = keys[t];
+      const unsigned long long ppos = 1023ull - ((x >> 22) & 1023ull);
+      const unsigned long long tok = 0x3fffffull - (x & 0x3fffffull);
+      kept_s[t] = ord2f((unsigned)(x >> 32));
+      ck[t] = ~((ppos << 42) | (tok << 10) | (unsigned long long)t);   // descending sort -> ascending
+    } else {
+      ck[t] = 0ull;
     }
-    cpos[t] = rank;
   }
   __syncthreads();
-  // canonical order among the kept: (parent position, token)
-  for (int t = threadIdx.x; t < C; t += blockDim.x) {
-    if (cpos[t] >= a.beam) continue;
-    const int pt = cp[t], tt = ct[t];
-    int pos = 0;
-    for (int u = 0; u < C; ++u)
-      pos += cpos[u] < a.beam && (cp[u] < pt || (cp[u] == pt && ct[u] < tt));
-    const size_t o = (size_t)b * a.beam + pos;
-    a.lvl_tok[o] = tt;
-    a.lvl_ppos[o] = pt;
-    a.lvl_s[o] = cs[t];
+  bitonic_desc_block(ck, Q);
+  for (int t = threadIdx.x; t < kept; t += blockDim.x) {
+    const unsigned long long x = ~ck[t];
+    const size_t o = (size_t)b * a.beam + t;
+    a.lvl_tok[o] = (int)((x >> 10) & 0x3fffffull);
+    a.lvl_ppos[o] = (int)(x >> 42);
+    a.lvl_s[o] = kept_s[x & 1023ull];
   }
   if (a.Eg_next == nullptr) return;
-  __syncthreads();
-  // next depth's Markov operand rows: Eg[b * F_new + pos] = E[token]
+  // next depth's Markov operand rows: Eg[b * F_new + pos] = E[token], 16-byte copies
   const int Fn = a.F_new;
   const TE* E = static_cast<const TE*>(a.E);
   TE* Eg = static_cast<TE*>(a.Eg_next);
-  for (int idx = threadIdx.x; idx < Fn * a.r_pad; idx += blockDim.x) {
-    const int pos = idx / a.r_pad, j = idx - pos * a.r_pad;
-    int t = a.lvl_tok[(size_t)b * a.beam + pos];
-    t = (t < 0 || t >= a.V) ? 0 : t;
-    Eg[((size_t)b * Fn + pos) * a.r_pad + j] = j < a.r ? E[(size_t)t * a.r + j] : TE(0.f);
+  constexpr int per16 = 16 / (int)sizeof(TE);
+  const bool vec = (a.r % per16 == 0) && (a.r_pad % per16 == 0) &&
+                   ((reinterpret_cast<uintptr_t>(E) & 15u) == 0);
+  if (vec) {
+    const int rv = a.r / per16, rpv = a.r_pad / per16;
+    for (int idx = threadIdx.x; idx < kept * rpv; idx += blockDim.x) {
+      const int t = idx / rpv, j = idx - t * rpv;
+      const unsigned long long x = ~ck[t];
+      int tok = (int)((x >> 10) & 0x3fffffull);
+      tok = (tok < 0 || tok >= a.V) ? 0 : tok;
+      const uint4 val = j < rv ? reinterpret_cast<const uint4*>(E + (size_t)tok * a.r)[j]
+                               : make_uint4(0u, 0u, 0u, 0u);
+      reinterpret_cast<uint4*>(Eg + ((size_t)b * Fn + t) * a.r_pad)[j] = val;
+    }
+  } else {
+    for (int idx = threadIdx.x; idx < kept * a.r_pad; idx += blockDim.x) {
+      const int t = idx / a.r_pad, j = idx - t * a.r_pad;
+      const unsigned long long x = ~ck[t];
+      int tok = (int)((x >> 10) & 0x3fffffull);
+      tok = (tok < 0 || tok >= a.V) ? 0 : tok;
+      Eg[((size_t)b * Fn + t) * a.r_pad + j] = j < a.r ? E[(size_t)tok * a.r + j] : TE(0.f);
+    }
   }
 }
 

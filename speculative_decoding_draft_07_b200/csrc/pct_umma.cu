@@ -51,8 +51,10 @@ constexpr int B_STAGE_BYTES = BK * BN * 2;       // 16 KB
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int THREADS = 64 + 32 * NUM_EPI_WARPS; // 320
 constexpr int TMEM_COLS = 512;
-constexpr size_t SMEM_BYTES =
-    1024 + (size_t)NSUBMAX * KBMAX * A_TILE_BYTES + (size_t)STAGES * B_STAGE_BYTES + 256;
+constexpr int LBMAX = 64;                        // request rows of L_d staged per N-tile
+constexpr int L_SLOT_BYTES = 2 * 64 * LBMAX * 2; // two [LB][64] bf16 boxes = 16 KB
+constexpr size_t SMEM_BYTES = 1024 + (size_t)NSUBMAX * KBMAX * A_TILE_BYTES +
+                              (size_t)STAGES * B_STAGE_BYTES + 2 * (size_t)L_SLOT_BYTES + 256;
 constexpr long long kTimeoutCycles = 4000000000ll;   // ~2 s at 2 GHz
 
 // Instruction descriptor, kind::f16: D = f32, A = B = bf16, A K-major,
@@ -62,6 +64,7 @@ constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u
 
 struct UmmaParams {
   int M, nsub, rows_per_cta, n_par, V, kblocks, S, tiles_total, k;
+  int LB;          // L_d rows staged per N-tile (requests a CTA touches, <= LBMAX)
   const void* L;
   long long L_req_stride;
   float2* pms;
@@ -174,6 +177,13 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ uint4 ld_shared16(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr));
+  return r;
+}
+
 // 32 drafter logits of one row starting at column col0 (col0 % 32 == 0).
 // Columns at or past V read as -inf.
 template <typename TL>
@@ -206,21 +216,27 @@ __device__ __forceinline__ void load_logits32<float>(const float* row, int col0,
   }
 }
 
-template <typename TL, int KMAX>
+// STAGE: the drafter logits of each N-tile arrive in shared memory by TMA
+// (bf16 logits, every CTA touching at most LBMAX requests); otherwise the
+// epilogue reads them from global memory (L2) itself.
+template <typename TL, int KMAX, bool STAGE>
 __global__ void __launch_bounds__(THREADS, 1)
     score_umma_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const UmmaParams p) {
+                      const __grid_constant__ CUtensorMap tmL, const UmmaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + NSUBMAX * KBMAX * A_TILE_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE_BYTES);
+  uint8_t* sL = sB + STAGES * B_STAGE_BYTES;                     // [2] L_d slots
+  uint64_t* full = reinterpret_cast<uint64_t*>(sL + 2 * L_SLOT_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* afull = empty + STAGES;
   uint64_t* tfull = afull + 1;      // [2]
   uint64_t* tempty = tfull + 2;     // [2]
-  uint64_t* drain = tempty + 2;
+  uint64_t* lfull = tempty + 2;     // [2]
+  uint64_t* lempty = lfull + 2;     // [2]
+  uint64_t* drain = lempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -234,7 +250,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     mbar_init(afull, 1);
-    for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], NUM_EPI_WARPS * 32); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], NUM_EPI_WARPS * 32);
+      mbar_init(&lfull[i], 1);
+      mbar_init(&lempty[i], NUM_EPI_WARPS * 32);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -262,8 +283,19 @@ __global__ void __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      const int req0 = row0 / p.n_par;
+      uint32_t larmed = 0;
       for (int it = 0; it < ntiles && ok; ++it) {
         const int n0 = (t_begin + it) * BN;
+        if (STAGE) {
+          const int slot = it & 1;
+          if (!wait_bar(&lempty[slot], (((uint32_t)it >> 1) & 1u) ^ 1u, abort_flag, p.err)) { ok = false; break; }
+          mbar_expect_tx(&lfull[slot], (uint32_t)(2 * 64 * p.LB * 2));
+          uint8_t* dst = sL + slot * L_SLOT_BYTES;
+          tma_load_2d(dst, &tmL, n0, req0, &lfull[slot]);
+          tma_load_2d(dst + 64 * p.LB * 2, &tmL, n0 + 64, req0, &lfull[slot]);
+          larmed = (uint32_t)it + 1;
+        }
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!wait_bar(&empty[stage], phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
           mbar_expect_tx(&full[stage], B_STAGE_BYTES);
@@ -280,6 +312,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int i = 0; i < STAGES; ++i)
         if (armed & (1u << i)) drain_wait(&full[i], (armed_par >> i) & 1u);
+      // the last one or two L_d slots armed (tiles larmed-1 and larmed-2)
+      for (int t = (int)larmed - 2; t < (int)larmed; ++t)
+        if (t >= 0) drain_wait(&lfull[t & 1], ((uint32_t)t >> 1) & 1u);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -327,8 +362,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int r_in = st * BM + quad * 32 + lane;
     const int row = row0 + r_in;
     const bool valid = (st < p.nsub) && (row < p.M);
-    const int req = valid ? row / p.n_par : 0;
+    const int req = valid ? row / p.n_par : row0 / p.n_par;
+    const int req_local = req - row0 / p.n_par;       // < LB when STAGE
     const TL* Lr = static_cast<const TL*>(p.L) + (size_t)req * p.L_req_stride;
+    const uint32_t sL_row = smem_u32(sL) + (uint32_t)(req_local * 128);
     const int k = p.k, V = p.V;
     float m = neg_inf(), s = 0.f;
     TopK<KMAX> tk;
@@ -337,7 +374,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     int ti = INT_MAX;
     for (int it = 0; it < ntiles; ++it) {
       const int buf = it & 1;
-      if (!wait_bar(&tfull[buf], (uint32_t)((it >> 1) & 1), abort_flag, p.err)) break;
+      const uint32_t par = (uint32_t)((it >> 1) & 1);
+      if (!wait_bar(&tfull[buf], par, abort_flag, p.err)) break;
+      if (STAGE && !wait_bar(&lfull[buf], par, abort_flag, p.err)) break;
       tc_fence_after();
       const int n0 = (t_begin + it) * BN;
       const uint32_t tbase =
@@ -346,33 +385,56 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int c = 0; c < BN / 32; ++c) {
         const int col0 = n0 + c * 32;
         float x[32];
-        if (valid) load_logits32<TL>(Lr, col0, V, x);
+        if (STAGE) {
+          // [LB][64] box (c >> 1), columns (c & 1) * 32 .. +31 of this request's row
+          const uint32_t a = sL_row + (uint32_t)(buf * L_SLOT_BYTES + (c >> 1) * (64 * p.LB * 2) +
+                                                 (c & 1) * 64);
+          uint4 w[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) w[q] = ld_shared16(a + 16 * q);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            x[q * 8 + 0] = bf16_lo(w[q].x); x[q * 8 + 1] = bf16_hi(w[q].x);
+            x[q * 8 + 2] = bf16_lo(w[q].y); x[q * 8 + 3] = bf16_hi(w[q].y);
+            x[q * 8 + 4] = bf16_lo(w[q].z); x[q * 8 + 5] = bf16_hi(w[q].z);
+            x[q * 8 + 6] = bf16_lo(w[q].w); x[q * 8 + 7] = bf16_hi(w[q].w);
+          }
+        } else if (valid) {
+          load_logits32<TL>(Lr, col0, V, x);
+        }
         uint32_t acc[32];
         tmem_ld32(tbase + (uint32_t)(c * 32), acc);
         if (valid) {
-          float cm = neg_inf();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            x[j] += __uint_as_float(acc[j]);
-            cm = fmaxf(cm, x[j]);
+          for (int j = 0; j < 32; ++j) x[j] += __uint_as_float(acc[j]);
+          if (col0 + 32 > V) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = (col0 + j < V) ? x[j] : neg_inf();
           }
+          // chunk max as a tree (short dependency chains)
+          float t16[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) t16[j] = fmaxf(x[j], x[j + 16]);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) t16[j] = fmaxf(t16[j], t16[j + 8]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) t16[j] = fmaxf(t16[j], t16[j + 4]);
+          const float cm = fmaxf(fmaxf(t16[0], t16[2]), fmaxf(t16[1], t16[3]));
           if (cm > m) { s = (m == neg_inf()) ? 0.f : s * ex2((m - cm) * kLog2e); m = cm; }
           if (m != neg_inf()) {
             const float mb = m * kLog2e;
-            float s0 = 0.f, s1 = 0.f;
+            float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              s0 += ex2(fmaf(x[j], kLog2e, -mb));
-              s1 += ex2(fmaf(x[j + 1], kLog2e, -mb));
-            }
-            s += s0 + s1;
+            for (int j = 0; j < 32; ++j) s4[j & 3] += ex2(fmaf(x[j], kLog2e, -mb));
+            s += (s4[0] + s4[1]) + (s4[2] + s4[3]);
           }
           if (cm >= tv) {
-            // positions that beat the current k-th entry; the threshold only
-            // rises, so positions outside the mask never need a second look
+            // superset gate (x >= k-th value); the exact order test runs per
+            // candidate. The threshold only rises, so positions outside the
+            // mask never need a second look.
             uint32_t cand = 0;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) cand |= (uint32_t)better(x[j], col0 + j, tv, ti) << j;
+            for (int j = 0; j < 32; ++j) cand |= (uint32_t)(x[j] >= tv) << j;
             while (cand) {
               const int j = __ffs(cand) - 1;
               cand &= cand - 1;
@@ -386,6 +448,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
+      if (STAGE) mbar_arrive(&lempty[buf]);
     }
     if (valid) {
       const size_t ps = (size_t)row * p.S + sl;
@@ -425,16 +488,20 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// 2D bf16 tensor map: `inner` contiguous elements per row, rows `row_bytes`
+// apart (0: dense), 128-byte swizzle or none.
 bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                    uint32_t box_inner, uint32_t box_outer) {
+                    uint32_t box_inner, uint32_t box_outer, uint64_t row_bytes = 0,
+                    bool swizzle128 = true) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint64_t strides[1] = {row_bytes ? row_bytes : inner * 2};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -479,20 +546,39 @@ cudaError_t launch_score(const ScoreArgs& a, cudaStream_t s) {
   p.pval = a.part.val;
   p.pidx = a.part.idx;
   p.err = a.err;
-  dim3 grid(a.S, (rows + p.rows_per_cta - 1) / p.rows_per_cta);
+  const int mtiles = (rows + p.rows_per_cta - 1) / p.rows_per_cta;
+  // requests any CTA's rows span: stage L_d by TMA when that fits a slot
+  int span = 0;
+  for (int mt = 0; mt < mtiles; ++mt) {
+    const int r0 = mt * p.rows_per_cta, r1 = std::min(rows, r0 + p.rows_per_cta) - 1;
+    span = std::max(span, r1 / a.n_par - r0 / a.n_par + 1);
+  }
+  const bool stage = a.logits_dtype == PCT_BF16 && span <= LBMAX;
+  p.LB = stage ? (span + 7) / 8 * 8 : 0;
+  CUtensorMap tmL;
+  if (stage) {
+    if (!encode_2d_bf16(&tmL, a.L, (uint64_t)a.V, (uint64_t)a.n_req, 64, (uint32_t)p.LB,
+                        (uint64_t)a.L_req_stride * 2, false))
+      return cudaErrorInvalidValue;
+  } else {
+    tmL = tmB;   // unused
+  }
+  dim3 grid(a.S, mtiles);
   TraceScope t(s, "pct_score_umma");
-#define PCT_UMMA(TL, KM)                                                                        \
+#define PCT_UMMA(TL, KM, ST)                                                                    \
   do {                                                                                          \
-    auto kern = score_umma_kernel<TL, KM>;                                                      \
+    auto kern = score_umma_kernel<TL, KM, ST>;                                                  \
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,     \
                                          (int)SMEM_BYTES);                                      \
     if (e != cudaSuccess) return e;                                                             \
-    kern<<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, p);                                        \
+    kern<<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, tmL, p);                                   \
   } while (0)
-  if (a.logits_dtype == PCT_BF16) {
-    if (a.k <= 4) PCT_UMMA(__nv_bfloat16, 4); else if (a.k <= 8) PCT_UMMA(__nv_bfloat16, 8); else PCT_UMMA(__nv_bfloat16, 16);
+  if (stage) {
+    if (a.k <= 4) PCT_UMMA(__nv_bfloat16, 4, true); else if (a.k <= 8) PCT_UMMA(__nv_bfloat16, 8, true); else PCT_UMMA(__nv_bfloat16, 16, true);
+  } else if (a.logits_dtype == PCT_BF16) {
+    if (a.k <= 4) PCT_UMMA(__nv_bfloat16, 4, false); else if (a.k <= 8) PCT_UMMA(__nv_bfloat16, 8, false); else PCT_UMMA(__nv_bfloat16, 16, false);
   } else {
-    if (a.k <= 4) PCT_UMMA(float, 4); else if (a.k <= 8) PCT_UMMA(float, 8); else PCT_UMMA(float, 16);
+    if (a.k <= 4) PCT_UMMA(float, 4, false); else if (a.k <= 8) PCT_UMMA(float, 8, false); else PCT_UMMA(float, 16, false);
   }
 #undef PCT_UMMA
   return cudaGetLastError();

@@ -57,6 +57,13 @@ def test_bf16_markov_needs_vocab_multiple_of_8():
     assert pct.lib().pct_tree_build_workspace(ctypes.byref(d)) > 0
 
 
+def test_vocab_above_2_pow_22_unsupported():
+    d = _desc(vocab=(1 << 22) + 8)
+    dummy = ctypes.c_void_p(256)
+    rc = pct.lib().pct_tree_build(ctypes.byref(d), *([dummy] * 10), dummy, 1 << 30, None)
+    assert rc == pct.PCT_EUNSUPPORTED
+
+
 def test_null_pointers_rejected_before_device_check():
     d = _desc()
     rc = pct.lib().pct_tree_build(ctypes.byref(d), *([None] * 10), None, 0, None)

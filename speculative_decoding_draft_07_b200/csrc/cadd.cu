@@ -169,7 +169,7 @@ __device__ __forceinline__ void cadd_keep(unsigned long long* keys, int* n, floa
 }
 
 template <typename T>
-__global__ __launch_bounds__(kRowThreads) void cadd_rowpass_kernel(
+__global__ __launch_bounds__(kRowThreads, 3) void cadd_rowpass_kernel(
     CaddParams p, const T* __restrict__ L, const int64_t* __restrict__ ctx,
     float* __restrict__ row_lse, int32_t* __restrict__ cand_cnt, float* __restrict__ cand_q,
     int32_t* __restrict__ cand_tok, int32_t* __restrict__ status) {
@@ -179,6 +179,7 @@ __global__ __launch_bounds__(kRowThreads) void cadd_rowpass_kernel(
   __shared__ int hist[256];
   __shared__ int s_n, s_n2;
   __shared__ float s_lnth;
+  __shared__ float2 s_pub[kRowThreads / 32];   // per-warp running (max, sum)
   const int d = blockIdx.x, b = blockIdx.y;
   const int V = p.V;
   const size_t row = (size_t)b * p.D + d;
@@ -191,18 +192,22 @@ __global__ __launch_bounds__(kRowThreads) void cadd_rowpass_kernel(
     const float lt = cadd_ln_theta(p, (double)ctx[b], lane, d == 0, &status[b]);
     if (lane == 0) { s_lnth = lt; s_n = 0; }
   }
+  if (lane == 0) s_pub[warp] = make_float2(neg_inf(), 0.f);
   __syncthreads();
   const float lnth = s_lnth - kThetaSlack;
 
-  // One pass over the row in chunks held in registers. After each chunk the
-  // block's running log-sum-exp (a lower bound of the row's, which only grows)
-  // gives a threshold that every final candidate already passes, so the
-  // chunk's survivors are taken from registers without a second read.
+  // One pass over the row in chunks held in registers. After each chunk a
+  // warp publishes its running (max, sum) to shared memory and combines every
+  // warp's latest snapshot: partial sums over disjoint parts of the row, so the
+  // combination is a lower bound of the row's log-sum-exp whatever the other
+  // warps' progress. That bound gives a threshold every final candidate
+  // already passes, and the chunk's survivors are taken straight from
+  // registers: no second read of the row and no block barrier in the loop.
   float m = neg_inf(), s = 0.f;
   if (vec) {
     const uint4* pv = reinterpret_cast<const uint4*>(x);
     const int nvec = V >> 3;
-    // uniform trip count: block_lse below synchronises the whole block
+    // uniform trip count: the warp shuffles below need every lane
     for (int c0 = 0; c0 < nvec; c0 += kRowThreads * kChunk) {
       const int base = c0 + threadIdx.x;
       uint4 q[kChunk];
@@ -230,9 +235,20 @@ __global__ __launch_bounds__(kRowThreads) void cadd_rowpass_kernel(
           s += s0 + s1;
         }
       }
-      // running block log-sum-exp -> chunk threshold
-      float bm = m, bs = s;
-      block_lse(bm, bs, sm, ss);
+      // warp total -> published snapshot -> bound over all warps' snapshots
+      float wm = m, ws = s;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, wm, o), s2 = __shfl_xor_sync(0xffffffffu, ws, o);
+        lse_combine(wm, ws, m2, s2);
+      }
+      if (lane == 0) st_shared_vol2(&s_pub[warp], wm, ws);
+      float bm = neg_inf(), bs = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < kRowThreads / 32; ++w2) {
+        const float2 o = w2 == warp ? make_float2(wm, ws) : ld_shared_vol2(&s_pub[w2]);
+        lse_combine(bm, bs, o.x, o.y);
+      }
       const float t = (K <= 0 || bm == neg_inf()) ? __int_as_float(0x7f800000)
                                                   : bm + logf(bs) + lnth;
 #pragma unroll

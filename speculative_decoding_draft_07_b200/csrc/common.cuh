@@ -50,38 +50,62 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
   return r;
 }
 
+// 8-byte shared-memory store/load that other warps observe as one unit.
+__device__ __forceinline__ void st_shared_vol2(float2* p, float a, float b) {
+  asm volatile("st.volatile.shared.v2.f32 [%0], {%1, %2};" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(p))),
+               "f"(a), "f"(b)
+               : "memory");
+}
+__device__ __forceinline__ float2 ld_shared_vol2(const float2* p) {
+  float2 r;
+  asm volatile("ld.volatile.shared.v2.f32 {%0, %1}, [%2];"
+               : "=f"(r.x), "=f"(r.y)
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p)))
+               : "memory");
+  return r;
+}
+
 // Key order used by every top-k in this library: larger value first, then
 // lower index. Returns true when (va, ia) goes before (vb, ib).
 __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
   return va > vb || (va == vb && ia < ib);
 }
 
-// Sorted (descending by `better`) top-K list kept in registers; K is a
-// compile-time capacity, the live length is the runtime k <= K. Slots start
-// at (-inf, INT_MAX) so that -inf values still enter in index order.
+// Sorted (descending by `better`) top-k list kept in registers. K is the
+// compile-time capacity and k <= K the live length: the k live entries sit in
+// the LAST k slots, behind K - k (+inf, -1) markers that nothing displaces, so
+// the admission threshold is always slot K - 1. Every index is a compile-time
+// constant (a runtime k-th index would force the array into local memory).
+// Empty live slots hold (-inf, INT_MAX) so that -inf values still enter in
+// index order. finish(k) moves the live entries to slots 0..k-1.
 template <int K>
 struct TopK {
   float v[K];
   int i[K];
-  __device__ __forceinline__ void init() {
+  __device__ __forceinline__ void init(int k) {
 #pragma unroll
-    for (int j = 0; j < K; ++j) { v[j] = neg_inf(); i[j] = 0x7fffffff; }
+    for (int j = 0; j < K; ++j) {
+      const bool marker = j < K - k;
+      v[j] = marker ? __int_as_float(0x7f800000) : neg_inf();
+      i[j] = marker ? -1 : 0x7fffffff;
+    }
   }
-  // k-th entry (the admission threshold), k in 1..K.
-  __device__ __forceinline__ void kth(int k, float& tv, int& ti) const {
-    tv = v[0]; ti = i[0];
-#pragma unroll
-    for (int j = 1; j < K; ++j) if (j == k - 1) { tv = v[j]; ti = i[j]; }
+  // admission threshold: the k-th live entry
+  __device__ __forceinline__ float tv() const { return v[K - 1]; }
+  __device__ __forceinline__ int ti() const { return i[K - 1]; }
+  __device__ __forceinline__ bool admits(float z, int idx) const {
+    return better(z, idx, v[K - 1], i[K - 1]);
   }
   // Bubble the new element through the sorted list; the last one falls out.
   __device__ __forceinline__ void insert(float z, int idx) {
     float cz = z; int ci = idx;
 #pragma unroll
     for (int j = 0; j < K; ++j) {
-      bool sw = better(cz, ci, v[j], i[j]);
-      float tv = v[j]; int ti = i[j];
-      v[j] = sw ? cz : tv; i[j] = sw ? ci : ti;
-      cz = sw ? tv : cz; ci = sw ? ti : ci;
+      const bool sw = better(cz, ci, v[j], i[j]);
+      const float tv_ = v[j]; const int ti_ = i[j];
+      v[j] = sw ? cz : tv_; i[j] = sw ? ci : ti_;
+      cz = sw ? tv_ : cz; ci = sw ? ti_ : ci;
     }
   }
   // Remove the head (shift left).
@@ -89,6 +113,9 @@ struct TopK {
 #pragma unroll
     for (int j = 0; j + 1 < K; ++j) { v[j] = v[j + 1]; i[j] = i[j + 1]; }
     v[K - 1] = neg_inf(); i[K - 1] = 0x7fffffff;
+  }
+  __device__ __forceinline__ void finish(int k) {
+    for (int s = 0; s < K - k; ++s) pop();
   }
 };
 

@@ -46,17 +46,16 @@ __global__ void gather_rows_kernel(int rows, const int32_t* __restrict__ toks, i
 }
 
 // Fold the S partials of one row (warp-cooperative). Returns lse and writes
-// the row's k best (value desc, token asc) to out_v / out_i. Every slice's
-// list is already sorted, so with S <= 32 each lane holds one slice's list and
-// the merge is k rounds of "take the best head, the owner pops"; with S > 32 a
-// lane first folds its slices by insertion.
+// the row's k best (value desc, token asc) to out_v / out_i: each lane folds
+// its slices' lists into a register top-k, then k rounds of "take the best
+// head across the warp, the owner pops".
 template <int KMAX>
 __device__ __forceinline__ float merge_row(const Partials& part, size_t row, int S, int k,
                                            float* out_v, int* out_i) {
   const int lane = threadIdx.x & 31;
   float m = neg_inf(), s = 0.f;
   TopK<KMAX> tk;
-  tk.init();
+  tk.init(k);
   for (int sl = lane; sl < S; sl += 32) {
     const size_t ps = row * S + sl;
     const float2 ms = part.ms[ps];
@@ -68,18 +67,11 @@ __device__ __forceinline__ float merge_row(const Partials& part, size_t row, int
       v[j] = j < k ? part.val[ps * k + j] : neg_inf();
       id[j] = j < k ? part.idx[ps * k + j] : 0x7fffffff;
     }
-    if (sl == lane) {          // first slice of this lane: already sorted
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j) { tk.v[j] = v[j]; tk.i[j] = id[j]; }
-    } else {
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        float tv; int ti;
-        tk.kth(k, tv, ti);
-        if (j < k && better(v[j], id[j], tv, ti)) tk.insert(v[j], id[j]);
-      }
-    }
+    for (int j = 0; j < KMAX; ++j)
+      if (j < k && tk.admits(v[j], id[j])) tk.insert(v[j], id[j]);
   }
+  tk.finish(k);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);

@@ -37,16 +37,15 @@ __global__ __launch_bounds__(kSimtThreads) void score_simt_kernel(ScoreArgs a, i
 
   float m = neg_inf(), s = 0.f;
   TopK<KMAX> tk;
-  tk.init();
-  float tv = neg_inf();
-  int ti = INT_MAX;
+  tk.init(k);
   for (int v = c0 + threadIdx.x; v < c1; v += blockDim.x) {
     float acc = 0.f;
     for (int j = 0; j < r; ++j) acc = fmaf(eg[j], W[(size_t)j * V + v], acc);
     const float z = load_f(Lr + v) + acc;
     lse_combine(m, s, z, 1.f);
-    if (better(z, v, tv, ti)) { tk.insert(z, v); tk.kth(k, tv, ti); }
+    if (tk.admits(z, v)) tk.insert(z, v);
   }
+  tk.finish(k);
   // fold the block: log-sum-exp pairs, then k rounds of block-wide best head
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll

@@ -17,7 +17,9 @@
 //    x 2 buffers x 128 columns = all 512 columns), commits each ring slot back
 //    to the producer and each finished accumulator to the epilogue.
 //  * warps 2..9: epilogue. Warp w reads TMEM lane quarter (w % 4), so every
-//    thread owns one parent row; it loads 32 accumulator columns at a time,
+//    thread owns one parent row (with 16 epilogue warps two warps share a
+//    quarter, each taking half of every N-tile's columns, and the halves are
+//    folded at the end; 8 measured faster); it loads 32 accumulator columns at a time,
 //    adds the row's drafter logits L_d (bf16, shared by the request's parents,
 //    served from L2), and keeps an online log-sum-exp (chunk max, one rescale,
 //    32 exp2 on the SFU) and a register top-k admitted by a threshold test.
@@ -48,8 +50,9 @@ constexpr int KBMAX = 4;                 // r_pad <= 256
 constexpr int NSUBMAX = 2;               // row tiles per CTA
 constexpr int A_TILE_BYTES = BM * BK * 2;        // 16 KB
 constexpr int B_STAGE_BYTES = BK * BN * 2;       // 16 KB
-constexpr int NUM_EPI_WARPS = 8;
-constexpr int THREADS = 64 + 32 * NUM_EPI_WARPS; // 320
+constexpr int NUM_EPI_WARPS = 8;                 // 1 or 2 per (row tile, TMEM lane quarter)
+constexpr int SPLIT = NUM_EPI_WARPS / 8;         // warps sharing a lane quarter: column parts
+constexpr int THREADS = 64 + 32 * NUM_EPI_WARPS; // producer + MMA warps + epilogue
 constexpr int TMEM_COLS = 512;
 constexpr int LBMAX = 64;                        // request rows of L_d staged per N-tile
 constexpr int L_SLOT_BYTES = 2 * 64 * LBMAX * 2; // two [LB][64] bf16 boxes = 16 KB
@@ -356,8 +359,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ---------------- epilogue ----------------
+    // warp group g = (warp - 2) / 4 covers TMEM lane quarters 0..3 once:
+    // row tile st = g / 2, column half h = g % 2 of every N-tile
     const int e = warp - 2;
-    const int st = e >> 2;
+    const int g = e >> 2;
+    const int st = g / SPLIT, h = g % SPLIT;
     const int quad = warp & 3;
     const int r_in = st * BM + quad * 32 + lane;
     const int row = row0 + r_in;
@@ -369,9 +375,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int k = p.k, V = p.V;
     float m = neg_inf(), s = 0.f;
     TopK<KMAX> tk;
-    tk.init();
-    float tv = neg_inf();
-    int ti = INT_MAX;
+    tk.init(k);
     for (int it = 0; it < ntiles; ++it) {
       const int buf = it & 1;
       const uint32_t par = (uint32_t)((it >> 1) & 1);
@@ -382,11 +386,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t tbase =
           tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)((buf * NSUBMAX + st) * BN);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = h * (4 / SPLIT); c < (h + 1) * (4 / SPLIT); ++c) {
         const int col0 = n0 + c * 32;
         float x[32];
         if (STAGE) {
-          // [LB][64] box (c >> 1), columns (c & 1) * 32 .. +31 of this request's row
+          // [LB][64] box (c >> 1) = h, columns (c & 1) * 32 .. +31 of this request's row
           const uint32_t a = sL_row + (uint32_t)(buf * L_SLOT_BYTES + (c >> 1) * (64 * p.LB * 2) +
                                                  (c & 1) * 64);
           uint4 w[4];
@@ -428,20 +432,20 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int j = 0; j < 32; ++j) s4[j & 3] += ex2(fmaf(x[j], kLog2e, -mb));
             s += (s4[0] + s4[1]) + (s4[2] + s4[3]);
           }
-          if (cm >= tv) {
+          if (cm >= tk.tv()) {
             // superset gate (x >= k-th value); the exact order test runs per
             // candidate. The threshold only rises, so positions outside the
             // mask never need a second look.
             uint32_t cand = 0;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) cand |= (uint32_t)(x[j] >= tv) << j;
+            for (int j = 0; j < 32; ++j) cand |= (uint32_t)(x[j] >= tk.tv()) << j;
             while (cand) {
               const int j = __ffs(cand) - 1;
               cand &= cand - 1;
               float z = x[0];
 #pragma unroll
               for (int jj = 1; jj < 32; ++jj) z = (j == jj) ? x[jj] : z;
-              if (better(z, col0 + j, tv, ti)) { tk.insert(z, col0 + j); tk.kth(k, tv, ti); }
+              if (tk.admits(z, col0 + j)) tk.insert(z, col0 + j);
             }
           }
         }
@@ -450,7 +454,38 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive(&tempty[buf]);
       if (STAGE) mbar_arrive(&lempty[buf]);
     }
-    if (valid) {
+    // fold the two column halves of each row through shared memory (the Eg
+    // tile region is idle once the last MMA has completed)
+    wait_bar(afull, 0, abort_flag, p.err);
+    float2* xms = reinterpret_cast<float2*>(sA);                       // [256]
+    float* xv = reinterpret_cast<float*>(sA + 256 * sizeof(float2));   // [256][KMAX]
+    int* xi = reinterpret_cast<int*>(xv + 256 * KMAX);                 // [256][KMAX]
+    if (SPLIT == 1) {
+      if (valid) {
+        tk.finish(k);
+        const size_t ps = (size_t)row * p.S + sl;
+        p.pms[ps] = make_float2(m, s);
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+          if (j < k) { p.pval[ps * k + j] = tk.v[j]; p.pidx[ps * k + j] = tk.i[j]; }
+      }
+    } else if (h == 1) {
+      tk.finish(k);
+      xms[r_in] = make_float2(m, s);
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) { xv[r_in * KMAX + j] = tk.v[j]; xi[r_in * KMAX + j] = tk.i[j]; }
+    }
+    if (SPLIT > 1) asm volatile("bar.sync 1, %0;" ::"n"(NUM_EPI_WARPS * 32) : "memory");
+    if (SPLIT > 1 && h == 0 && valid) {
+      const float2 o = xms[r_in];
+      lse_combine(m, s, o.x, o.y);
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        const float v = xv[r_in * KMAX + j];
+        const int i = xi[r_in * KMAX + j];
+        if (j < k && tk.admits(v, i)) tk.insert(v, i);
+      }
+      tk.finish(k);
       const size_t ps = (size_t)row * p.S + sl;
       p.pms[ps] = make_float2(m, s);
 #pragma unroll

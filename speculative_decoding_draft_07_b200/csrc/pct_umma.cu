@@ -322,30 +322,41 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
+      // The issue loop is kept to a few instructions per MMA: a 128x128x16
+      // MMA lasts 64 cycles, and a longer dependent instruction chain here
+      // (descriptor assembly, runtime loops) leaves the tensor pipe idle.
+      // Descriptors are built once; the start-address field holds addr >> 4
+      // in the low 14 bits and shared addresses stay below 256 KB, so adding
+      // (offset >> 4) to a descriptor never carries out of the field.
       bool ok = wait_bar(afull, 0, abort_flag, p.err);
       tc_fence_after();
       int stage = 0;
       uint32_t phase = 0;
-      const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+      const uint64_t a_desc0 = make_desc(smem_u32(sA), 16, 1024);      // row tile 0, K block 0
+      const uint64_t b_desc0 = make_desc(smem_u32(sB), 8192, 1024);    // ring slot 0
+      const bool two = p.nsub == 2;
       for (int it = 0; it < ntiles && ok; ++it) {
         const int buf = it & 1;
         const uint32_t use = (uint32_t)(it >> 1);
         if (!wait_bar(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.err)) break;
         tc_fence_after();
+        const uint32_t d0 = tmem_base + (uint32_t)(buf * NSUBMAX * BN);
+        const uint32_t d1 = d0 + BN;
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!wait_bar(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
-          tc_fence_after();
+          const uint64_t bd = b_desc0 + (uint64_t)((stage * B_STAGE_BYTES) >> 4);
+          const uint64_t ad = a_desc0 + (uint64_t)((kb * A_TILE_BYTES) >> 4);
+          const uint32_t acc0 = kb != 0;
+          // B: [64 K][2 x 64 V] V-major, +2048 bytes per 16 K rows;
+          // A: [128 rows][64 K] K-major, +32 bytes per 16 K columns
+          umma_f16(d0, ad, bd, IDESC, acc0);
+          if (two) umma_f16(d1, ad + (KBMAX * A_TILE_BYTES >> 4), bd, IDESC, acc0);
 #pragma unroll
-          for (int k4 = 0; k4 < BK / 16; ++k4) {
-            // B: [64 K][2 x 64 V] V-major; +2048 bytes = 16 K rows
-            const uint64_t bdesc = make_desc(b_base + stage * B_STAGE_BYTES + k4 * 2048, 8192, 1024);
-            for (int st = 0; st < p.nsub; ++st) {
-              // A: [128 rows][64 K] K-major; +32 bytes = 16 K columns
-              const uint64_t adesc =
-                  make_desc(a_base + (st * KBMAX + kb) * A_TILE_BYTES + k4 * 32, 16, 1024);
-              umma_f16(tmem_base + (uint32_t)((buf * NSUBMAX + st) * BN), adesc, bdesc, IDESC,
-                       (kb | k4) != 0);
-            }
+          for (int k4 = 1; k4 < BK / 16; ++k4) {
+            umma_f16(d0, ad + (uint64_t)(k4 * 2), bd + (uint64_t)(k4 * 128), IDESC, 1u);
+            if (two)
+              umma_f16(d1, ad + (uint64_t)((KBMAX * A_TILE_BYTES >> 4) + k4 * 2),
+                       bd + (uint64_t)(k4 * 128), IDESC, 1u);
           }
           umma_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }

@@ -103,7 +103,7 @@ struct PctPlan {
   int S[66];
   int Mmax, M_pad;
   size_t max_ps;
-  size_t o_eg, o_ms, o_val, o_idx, o_ltok, o_lppos, o_ls, o_err, total;
+  size_t o_eg, o_ms, o_val, o_idx, o_ltok, o_lppos, o_ls, o_err, o_thr, total;
 };
 
 int check_build_desc(const pct_build_desc* d) {
@@ -147,6 +147,7 @@ int make_plan(const pct_build_desc* d, PctPlan* P) {
   P->o_lppos = o; o += align_up(lvl * sizeof(int32_t));
   P->o_ls = o;    o += align_up(lvl * sizeof(float));
   P->o_err = o;   o += align_up(sizeof(int32_t));
+  P->o_thr = o;   o += align_up((size_t)P->Mmax * sizeof(uint32_t));
   P->total = o;
   return PCT_OK;
 }
@@ -284,6 +285,7 @@ int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t*
     a.L = static_cast<const char*>(L) + (size_t)(d - 1) * P.V * esize(P.ldt);
     a.L_req_stride = (long long)P.D * P.V;
     a.Eg = Eg; a.M_pad = P.M_pad; a.W = W; a.part = part; a.S = P.S[d]; a.err = err;
+    a.row_thr = reinterpret_cast<uint32_t*>(ws + P.o_thr);
     PCT_CU(launch_score(a, s));
     MergeArgs m;
     m.batch = P.batch; m.F_prev = P.F[d - 1]; m.F_new = P.F[d]; m.k = P.k; m.beam = P.beam;
@@ -314,7 +316,7 @@ int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t*
 // ---------------------------------------------------------------------------
 static int score_parents_plan(const pct_build_desc* d, int32_t n_par, PctPlan* P, size_t* o_eg,
                               size_t* o_ms, size_t* o_val, size_t* o_idx, size_t* o_err,
-                              size_t* total, int* S) {
+                              size_t* o_thr, size_t* total, int* S) {
   if (!d) return PCT_EINVAL;
   if (d->batch < 1 || d->batch > 65535 || n_par < 1 || n_par > 4096) return PCT_EINVAL;
   if (d->vocab < 1 || d->k < 1 || d->k > 16 || d->k > d->vocab) return PCT_EINVAL;
@@ -334,15 +336,16 @@ static int score_parents_plan(const pct_build_desc* d, int32_t n_par, PctPlan* P
   *o_val = o; o += align_up(ps * P->k * sizeof(float));
   *o_idx = o; o += align_up(ps * P->k * sizeof(int32_t));
   *o_err = o; o += align_up(sizeof(int32_t));
+  *o_thr = o; o += align_up((size_t)rows * sizeof(uint32_t));
   *total = o;
   return PCT_OK;
 }
 
 size_t pct_score_parents_workspace(const pct_build_desc* desc, int32_t n_par) {
   PctPlan P;
-  size_t a, b, c, d, e, total;
+  size_t a, b, c, d, e, f, total;
   int S;
-  if (score_parents_plan(desc, n_par, &P, &a, &b, &c, &d, &e, &total, &S) != PCT_OK) return 0;
+  if (score_parents_plan(desc, n_par, &P, &a, &b, &c, &d, &e, &f, &total, &S) != PCT_OK) return 0;
   return total;
 }
 
@@ -351,9 +354,10 @@ int32_t pct_score_parents(const pct_build_desc* desc, int32_t n_par, const void*
                           int32_t* top_tok, float* top_logpi, int32_t* dev_status,
                           void* workspace, size_t ws_bytes, void* cuda_stream) {
   PctPlan P;
-  size_t o_eg, o_ms, o_val, o_idx, o_err, total;
+  size_t o_eg, o_ms, o_val, o_idx, o_err, o_thr, total;
   int S;
-  const int st = score_parents_plan(desc, n_par, &P, &o_eg, &o_ms, &o_val, &o_idx, &o_err, &total, &S);
+  const int st = score_parents_plan(desc, n_par, &P, &o_eg, &o_ms, &o_val, &o_idx, &o_err, &o_thr,
+                                    &total, &S);
   if (st != PCT_OK) return st;
   if (!L_row || !parent_tok || !E || !W || !lse || !top_tok || !top_logpi || !dev_status)
     return PCT_EINVAL;
@@ -375,6 +379,7 @@ int32_t pct_score_parents(const pct_build_desc* desc, int32_t n_par, const void*
   a.n_req = P.batch; a.n_par = n_par; a.V = P.V; a.r = P.r; a.r_pad = P.r_pad; a.k = P.k;
   a.logits_dtype = P.ldt; a.markov_dtype = P.mdt; a.L = L_row; a.L_req_stride = P.V;
   a.Eg = ws + o_eg; a.M_pad = P.M_pad; a.W = W; a.part = part; a.S = S; a.err = err;
+  a.row_thr = reinterpret_cast<uint32_t*>(ws + o_thr);
   PCT_CU(launch_score(a, s));
   PCT_CU(launch_rows_finalize(rows, P.k, S, part, lse, top_tok, top_logpi, err, dev_status, n_par, s));
   return PCT_OK;

@@ -32,6 +32,29 @@ __device__ __forceinline__ float ord2f(uint32_t o) {
   return __uint_as_float(u);
 }
 
+// Packed fp32 pairs (sm_100: add/fma on .f32x2, each lane IEEE round to
+// nearest even) and the three-input max.
+__device__ __forceinline__ float2 f2_add(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 a_, b_, r_;\n\tmov.b64 a_, {%2, %3};\n\tmov.b64 b_, {%4, %5};\n\t"
+      "add.rn.f32x2 r_, a_, b_;\n\tmov.b64 {%0, %1}, r_;\n\t}"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c) {
+  float2 r;
+  asm("{\n\t.reg .b64 a_, b_, c_, r_;\n\tmov.b64 a_, {%2, %3};\n\tmov.b64 b_, {%4, %5};\n\t"
+      "mov.b64 c_, {%6, %7};\n\tfma.rn.f32x2 r_, a_, b_, c_;\n\tmov.b64 {%0, %1}, r_;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Exact bf16 -> fp32 widening of a raw 16-bit pattern.
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }

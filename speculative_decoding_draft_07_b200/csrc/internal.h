@@ -66,6 +66,8 @@ struct ScoreArgs {
   Partials part;
   int S;                  // V-slices (partials per row)
   int32_t* err;           // device word, set on a timed-out wait
+  uint32_t* row_thr;      // [rows] best published k-th value per row (ordered key,
+                          // 0 = none); cleared by launch_score
 };
 // Slices the scoring kernel will use for `rows` rows (deterministic per device).
 int score_slices(int rows, int V, int markov_dtype);

@@ -50,8 +50,9 @@ constexpr int KBMAX = 4;                 // r_pad <= 256
 constexpr int NSUBMAX = 2;               // row tiles per CTA
 constexpr int A_TILE_BYTES = BM * BK * 2;        // 16 KB
 constexpr int B_STAGE_BYTES = BK * BN * 2;       // 16 KB
-constexpr int NUM_EPI_WARPS = 8;                 // 1 or 2 per (row tile, TMEM lane quarter)
+constexpr int NUM_EPI_WARPS = 16;                // 1 or 2 per (row tile, TMEM lane quarter)
 constexpr int SPLIT = NUM_EPI_WARPS / 8;         // warps sharing a lane quarter: column parts
+constexpr int CH = SPLIT == 2 ? 16 : 32;         // accumulator columns per TMEM load
 constexpr int THREADS = 64 + 32 * NUM_EPI_WARPS; // producer + MMA warps + epilogue
 constexpr int TMEM_COLS = 512;
 constexpr int LBMAX = 64;                        // request rows of L_d staged per N-tile
@@ -74,6 +75,7 @@ struct UmmaParams {
   float* pval;
   int32_t* pidx;
   int32_t* err;
+  uint32_t* row_thr;   // [M] best published k-th value per row (ordered key, 0 = none)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -162,6 +164,21 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
+// 16 consecutive fp32 accumulator columns of this thread's TMEM lane (load
+// and wait in one asm statement).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[16]) { tmem_ld16(taddr, r); }
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[32]);
+
 // 32 consecutive fp32 accumulator columns of this thread's TMEM lane. The
 // load and its wait sit in one asm statement so that no use of the outputs can
 // be scheduled before the data has arrived.
@@ -187,15 +204,61 @@ __device__ __forceinline__ uint4 ld_shared16(uint32_t addr) {
   return r;
 }
 
-// 32 drafter logits of one row starting at column col0 (col0 % 32 == 0).
-// Columns at or past V read as -inf.
-template <typename TL>
-__device__ __forceinline__ void load_logits32(const TL* row, int col0, int V, float (&x)[32]);
-template <>
-__device__ __forceinline__ void load_logits32<__nv_bfloat16>(const __nv_bfloat16* row, int col0,
-                                                             int V, float (&x)[32]) {
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[32]) { tmem_ld32(taddr, r); }
+
+// sum_j 2^(x_j log2 e - m log2 e) over N values, arguments and partial sums
+// in fp32 pairs.
+template <int N>
+__device__ __forceinline__ float chunk_exp_sum(const float (&x)[N], float m) {
+  const float2 l2e = make_float2(kLog2e, kLog2e);
+  const float2 nmb = make_float2(-m * kLog2e, -m * kLog2e);
+  float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int j = 0; j < N; j += 4) {
+    const float2 a0 = f2_fma(make_float2(x[j], x[j + 1]), l2e, nmb);
+    const float2 a1 = f2_fma(make_float2(x[j + 2], x[j + 3]), l2e, nmb);
+    sa = f2_add(sa, make_float2(ex2(a0.x), ex2(a0.y)));
+    sb = f2_add(sb, make_float2(ex2(a1.x), ex2(a1.y)));
+  }
+  const float2 t = f2_add(sa, sb);
+  return t.x + t.y;
+}
+
+// max of N values as a tree of three-input maxima
+template <int N>
+__device__ __forceinline__ float chunk_max(const float (&x)[N]) {
+  float t[(N + 2) / 3];
+#pragma unroll
+  for (int j = 0; j < N / 3; ++j) t[j] = fmax3(x[3 * j], x[3 * j + 1], x[3 * j + 2]);
+  if (N % 3 == 1) t[N / 3] = x[N - 1];
+  if (N % 3 == 2) t[N / 3] = fmaxf(x[N - 2], x[N - 1]);
+  constexpr int T = (N + 2) / 3;
+  float u[(T + 2) / 3];
+#pragma unroll
+  for (int j = 0; j < T / 3; ++j) u[j] = fmax3(t[3 * j], t[3 * j + 1], t[3 * j + 2]);
+  if (T % 3 == 1) u[T / 3] = t[T - 1];
+  if (T % 3 == 2) u[T / 3] = fmaxf(t[T - 2], t[T - 1]);
+  constexpr int U = (T + 2) / 3;
+  float r = u[0];
+#pragma unroll
+  for (int j = 1; j < U; ++j) r = fmaxf(r, u[j]);
+  return r;
+}
+
+// N drafter logits of one row starting at column col0 (col0 % N == 0, N a
+// multiple of 8). Columns at or past V read as -inf.
+template <typename TL, int N>
+__device__ __forceinline__ void load_logits(const TL* row, int col0, int V, float (&x)[N]) {
+  if (sizeof(TL) == 4) {
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      const int c = col0 + j;
+      x[j] = c < V ? load_f(row + c) : neg_inf();
+    }
+    return;
+  }
+#pragma unroll
+  for (int q = 0; q < N / 8; ++q) {
     const int c = col0 + q * 8;
     if (c < V) {   // V % 8 == 0: a 16-byte group is entirely in or out
       const uint4 w = __ldg(reinterpret_cast<const uint4*>(row + c));
@@ -207,15 +270,6 @@ __device__ __forceinline__ void load_logits32<__nv_bfloat16>(const __nv_bfloat16
 #pragma unroll
       for (int j = 0; j < 8; ++j) x[q * 8 + j] = neg_inf();
     }
-  }
-}
-template <>
-__device__ __forceinline__ void load_logits32<float>(const float* row, int col0, int V,
-                                                     float (&x)[32]) {
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const int c = col0 + j;
-    x[j] = c < V ? __ldg(row + c) : neg_inf();
   }
 }
 
@@ -387,6 +441,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     float m = neg_inf(), s = 0.f;
     TopK<KMAX> tk;
     tk.init(k);
+    // admission gate: max(own k-th value, best k-th value any slice of this
+    // row has published). Every slice's k-th value is a lower bound of the
+    // row's k-th, so values below the gate cannot be in the row's top-k.
+    float gth = neg_inf();
+    uint32_t* thr = p.row_thr + (valid ? row : 0);
+    uint32_t pub_prev = 0;   // loaded at the end of the previous tile, used one tile later
     for (int it = 0; it < ntiles; ++it) {
       const int buf = it & 1;
       const uint32_t par = (uint32_t)((it >> 1) & 1);
@@ -397,69 +457,82 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t tbase =
           tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)((buf * NSUBMAX + st) * BN);
 #pragma unroll 1
-      for (int c = h * (4 / SPLIT); c < (h + 1) * (4 / SPLIT); ++c) {
-        const int col0 = n0 + c * 32;
-        float x[32];
+      for (int c = h * (BN / CH / SPLIT); c < (h + 1) * (BN / CH / SPLIT); ++c) {
+        const int col0 = n0 + c * CH;
+        float x[CH];
         if (STAGE) {
-          // [LB][64] box (c >> 1) = h, columns (c & 1) * 32 .. +31 of this request's row
-          const uint32_t a = sL_row + (uint32_t)(buf * L_SLOT_BYTES + (c >> 1) * (64 * p.LB * 2) +
-                                                 (c & 1) * 64);
-          uint4 w[4];
+          // [LB][64] box (c * CH) / 64, columns (c * CH) % 64 .. of this request's row
+          const uint32_t a = sL_row + (uint32_t)(buf * L_SLOT_BYTES + ((c * CH) >> 6) * (64 * p.LB * 2) +
+                                                 ((c * CH) & 63) * 2);
+          uint4 w[CH / 8];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) w[q] = ld_shared16(a + 16 * q);
+          for (int q = 0; q < CH / 8; ++q) w[q] = ld_shared16(a + 16 * q);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < CH / 8; ++q) {
             x[q * 8 + 0] = bf16_lo(w[q].x); x[q * 8 + 1] = bf16_hi(w[q].x);
             x[q * 8 + 2] = bf16_lo(w[q].y); x[q * 8 + 3] = bf16_hi(w[q].y);
             x[q * 8 + 4] = bf16_lo(w[q].z); x[q * 8 + 5] = bf16_hi(w[q].z);
             x[q * 8 + 6] = bf16_lo(w[q].w); x[q * 8 + 7] = bf16_hi(w[q].w);
           }
         } else if (valid) {
-          load_logits32<TL>(Lr, col0, V, x);
+          load_logits<TL, CH>(Lr, col0, V, x);
         }
-        uint32_t acc[32];
-        tmem_ld32(tbase + (uint32_t)(c * 32), acc);
+        uint32_t acc[CH];
+        tmem_ld(tbase + (uint32_t)(c * CH), acc);
         if (valid) {
+          // z = L + E[p].W in fp32 pairs
 #pragma unroll
-          for (int j = 0; j < 32; ++j) x[j] += __uint_as_float(acc[j]);
-          if (col0 + 32 > V) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) x[j] = (col0 + j < V) ? x[j] : neg_inf();
+          for (int j = 0; j < CH; j += 2) {
+            const float2 z2 = f2_add(make_float2(x[j], x[j + 1]),
+                                     make_float2(__uint_as_float(acc[j]), __uint_as_float(acc[j + 1])));
+            x[j] = z2.x;
+            x[j + 1] = z2.y;
           }
-          // chunk max as a tree (short dependency chains)
-          float t16[16];
+          if (col0 + CH > V) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) t16[j] = fmaxf(x[j], x[j + 16]);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) t16[j] = fmaxf(t16[j], t16[j + 8]);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) t16[j] = fmaxf(t16[j], t16[j + 4]);
-          const float cm = fmaxf(fmaxf(t16[0], t16[2]), fmaxf(t16[1], t16[3]));
-          if (cm > m) { s = (m == neg_inf()) ? 0.f : s * ex2((m - cm) * kLog2e); m = cm; }
-          if (m != neg_inf()) {
-            const float mb = m * kLog2e;
-            float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int j = 0; j < 32; ++j) s4[j & 3] += ex2(fmaf(x[j], kLog2e, -mb));
-            s += (s4[0] + s4[1]) + (s4[2] + s4[3]);
+            for (int j = 0; j < CH; ++j) x[j] = (col0 + j < V) ? x[j] : neg_inf();
           }
-          if (cm >= tk.tv()) {
-            // superset gate (x >= k-th value); the exact order test runs per
-            // candidate. The threshold only rises, so positions outside the
-            // mask never need a second look.
+          const float cm = chunk_max<CH>(x);
+          // sum of 2^(z log2 e - m log2 e) against the running reference m,
+          // computed before (and independent of) this chunk's max; m moves
+          // only when a value exceeds it by more than 64 (exp(64) keeps the
+          // fp32 sum far from overflow), which recomputes the chunk
+          float csum = 0.f;
+          if (m != neg_inf()) csum = chunk_exp_sum<CH>(x, m);
+          if (cm > m + 64.f) {
+            s = (m == neg_inf()) ? 0.f : s * ex2((m - cm) * kLog2e);
+            m = cm;
+            csum = chunk_exp_sum<CH>(x, m);
+          }
+          s += csum;
+          if (cm >= gth) {
+            // superset gate (x >= gate); the exact order test runs per
+            // candidate. The gate only rises, so positions outside the mask
+            // never need a second look.
             uint32_t cand = 0;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) cand |= (uint32_t)(x[j] >= tk.tv()) << j;
+            for (int j = 0; j < CH; ++j) cand |= (uint32_t)(x[j] >= gth) << j;
             while (cand) {
               const int j = __ffs(cand) - 1;
               cand &= cand - 1;
               float z = x[0];
 #pragma unroll
-              for (int jj = 1; jj < 32; ++jj) z = (j == jj) ? x[jj] : z;
-              if (tk.admits(z, col0 + j)) tk.insert(z, col0 + j);
+              for (int jj = 1; jj < CH; ++jj) z = (j == jj) ? x[jj] : z;
+              if (z >= gth && tk.admits(z, col0 + j)) {
+                tk.insert(z, col0 + j);
+                gth = fmaxf(gth, tk.tv());
+              }
             }
           }
         }
+      }
+      // publish this slice's k-th value for the row and pick up the best one
+      // published by any slice (stale values are still valid lower bounds)
+      if (valid) {
+        if (pub_prev > f2ord(neg_inf())) gth = fmaxf(gth, ord2f(pub_prev));
+        const float own = tk.tv();
+        if (own != neg_inf()) atomicMax(thr, f2ord(own));
+        pub_prev = *reinterpret_cast<volatile uint32_t*>(thr);
       }
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
@@ -592,6 +665,9 @@ cudaError_t launch_score(const ScoreArgs& a, cudaStream_t s) {
   p.pval = a.part.val;
   p.pidx = a.part.idx;
   p.err = a.err;
+  p.row_thr = a.row_thr;
+  if (cudaMemsetAsync(a.row_thr, 0, sizeof(uint32_t) * (size_t)rows, s) != cudaSuccess)
+    return cudaErrorInvalidValue;
   const int mtiles = (rows + p.rows_per_cta - 1) / p.rows_per_cta;
   // requests any CTA's rows span: stage L_d by TMA when that fits a slot
   int span = 0;

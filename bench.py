@@ -83,13 +83,19 @@ def frontier_sizes():
     return F
 
 
+# The library scores depths of more than 128 parent rows with the CTA-pair
+# kernel and smaller ones with the single-CTA kernel.
+PAIR_ROWS_MIN = 129
+
+
 def algorithmic_work():
     F = frontier_sizes()
     rows = [W.batch * F[d - 1] for d in range(1, W.depth + 1)]
-    markov_flop = sum(2.0 * W.rank * W.vocab * m for m in rows)
+    flop = lambda ms: sum(2.0 * W.rank * W.vocab * m for m in ms)
     return {
-        # tensor-core contraction E_g[M_d][r] . W[r][V] per depth
-        "pct_score_umma": {"bound": "tensor", "flop": markov_flop},
+        # tensor-core contraction E_g[M_d][r] . W[r][V] per depth, by the kernel that runs it
+        "pct_score_pair": {"bound": "tensor", "flop": flop([m for m in rows if m >= PAIR_ROWS_MIN])},
+        "pct_score_umma": {"bound": "tensor", "flop": flop([m for m in rows if m < PAIR_ROWS_MIN])},
         # every node row of target logits read once (bf16)
         "verify_argmax_walk": {"bound": "hbm", "bytes": float(W.batch * W.n_nodes * W.vocab * 2)},
         # every marginal row read once (bf16)
@@ -102,7 +108,8 @@ def source_sha(fname):
     return hashlib.sha256(open(p, "rb").read()).hexdigest()[:12] if os.path.exists(p) else None
 
 
-KERNEL_SOURCE = {"pct_score_umma": "pct_umma.cu", "verify_argmax_walk": "verify.cu",
+KERNEL_SOURCE = {"pct_score_pair": "pct_umma2.cu", "pct_score_umma": "pct_umma.cu",
+                 "verify_argmax_walk": "verify.cu",
                  "cadd_rowpass": "cadd.cu"}
 
 

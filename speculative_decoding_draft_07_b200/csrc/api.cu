@@ -103,7 +103,7 @@ struct PctPlan {
   int S[66];
   int Mmax, M_pad;
   size_t max_ps;
-  size_t o_eg, o_ms, o_val, o_idx, o_ltok, o_lppos, o_ls, o_err, o_thr, total;
+  size_t o_eg, o_ms, o_val, o_idx, o_ltok, o_lppos, o_ls, o_err, o_thr, o_scol, o_slval, o_swmax, o_swcol, total;
 };
 
 int check_build_desc(const pct_build_desc* d) {
@@ -148,6 +148,11 @@ int make_plan(const pct_build_desc* d, PctPlan* P) {
   P->o_ls = o;    o += align_up(lvl * sizeof(float));
   P->o_err = o;   o += align_up(sizeof(int32_t));
   P->o_thr = o;   o += align_up((size_t)P->Mmax * sizeof(uint32_t));
+  const size_t seeds = (size_t)P->batch * P->D * P->k;   // seed entries (request, depth, column)
+  P->o_scol = o;  o += align_up(seeds * sizeof(int32_t));
+  P->o_slval = o; o += align_up(seeds * sizeof(float));
+  P->o_swmax = o; o += align_up(seeds * sizeof(float));
+  P->o_swcol = o; o += P->mdt == PCT_BF16 ? align_up(seeds * P->r_pad * 2) : 0;
   P->total = o;
   return PCT_OK;
 }
@@ -277,7 +282,32 @@ int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t*
 
   PCT_CU(cudaMemsetAsync(dev_status, 0, sizeof(int32_t) * P.batch, s));
   PCT_CU(cudaMemsetAsync(err, 0, sizeof(int32_t), s));
-  PCT_CU(launch_gather_rows(P.batch, anchor, P.V, P.r, P.r_pad, P.mdt, E, Eg, dev_status, 1, s));
+  // tensor-core scoring: every row's top-k gate starts from a seed (k exact
+  // values of the row at the request's best drafter columns of that depth)
+  const bool seeded = P.mdt == PCT_BF16;
+  uint32_t* row_thr = reinterpret_cast<uint32_t*>(ws + P.o_thr);
+  int32_t* scol = reinterpret_cast<int32_t*>(ws + P.o_scol);
+  float* slval = reinterpret_cast<float*>(ws + P.o_slval);
+  float* swmax = reinterpret_cast<float*>(ws + P.o_swmax);
+  char* swcol = ws + P.o_swcol;
+  auto seed_for = [&](int di) {   // seeds of the rows scored against L index di
+    SeedArgs sd{};
+    if (!seeded || di >= P.D) return sd;
+    const size_t e = (size_t)di * P.k;
+    sd.cols = scol + e;
+    sd.lval = slval + e;
+    sd.wmax = swmax + e;
+    sd.wcol = swcol + e * P.r_pad * 2;
+    sd.req_stride = (long long)P.D * P.k;
+    sd.ks = P.k;
+    sd.thr = row_thr;
+    return sd;
+  };
+  if (seeded)
+    PCT_CU(launch_drafter_topk(P.batch * P.D, P.V, P.k, P.ldt, L, W, P.r, P.r_pad, scol, slval,
+                               swmax, swcol, s));
+  PCT_CU(launch_gather_rows(P.batch, anchor, P.V, P.r, P.r_pad, P.mdt, E, Eg, dev_status, 1,
+                            seed_for(0), s));
   for (int d = 1; d <= P.D; ++d) {
     ScoreArgs a;
     a.n_req = P.batch; a.n_par = P.F[d - 1]; a.V = P.V; a.r = P.r; a.r_pad = P.r_pad; a.k = P.k;
@@ -285,7 +315,8 @@ int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t*
     a.L = static_cast<const char*>(L) + (size_t)(d - 1) * P.V * esize(P.ldt);
     a.L_req_stride = (long long)P.D * P.V;
     a.Eg = Eg; a.M_pad = P.M_pad; a.W = W; a.part = part; a.S = P.S[d]; a.err = err;
-    a.row_thr = reinterpret_cast<uint32_t*>(ws + P.o_thr);
+    a.row_thr = row_thr;
+    a.thr_seeded = seeded;
     PCT_CU(launch_score(a, s));
     MergeArgs m;
     m.batch = P.batch; m.F_prev = P.F[d - 1]; m.F_new = P.F[d]; m.k = P.k; m.beam = P.beam;
@@ -301,6 +332,7 @@ int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t*
     m.Eg_next = d < P.D ? Eg : nullptr;
     m.err = err;
     m.status = dev_status;
+    m.seed = seed_for(d);
     PCT_CU(launch_merge(m, s));
   }
   FinalArgs f;
@@ -374,12 +406,13 @@ int32_t pct_score_parents(const pct_build_desc* desc, int32_t n_par, const void*
   PCT_CU(cudaMemsetAsync(dev_status, 0, sizeof(int32_t) * P.batch, s));
   PCT_CU(cudaMemsetAsync(err, 0, sizeof(int32_t), s));
   PCT_CU(launch_gather_rows(rows, parent_tok, P.V, P.r, P.r_pad, P.mdt, E, ws + o_eg, dev_status,
-                            n_par, s));
+                            n_par, SeedArgs{}, s));
   ScoreArgs a;
   a.n_req = P.batch; a.n_par = n_par; a.V = P.V; a.r = P.r; a.r_pad = P.r_pad; a.k = P.k;
   a.logits_dtype = P.ldt; a.markov_dtype = P.mdt; a.L = L_row; a.L_req_stride = P.V;
   a.Eg = ws + o_eg; a.M_pad = P.M_pad; a.W = W; a.part = part; a.S = S; a.err = err;
   a.row_thr = reinterpret_cast<uint32_t*>(ws + o_thr);
+  a.thr_seeded = false;
   PCT_CU(launch_score(a, s));
   PCT_CU(launch_rows_finalize(rows, P.k, S, part, lse, top_tok, top_logpi, err, dev_status, n_par, s));
   return PCT_OK;

@@ -66,17 +66,39 @@ struct ScoreArgs {
   Partials part;
   int S;                  // V-slices (partials per row)
   int32_t* err;           // device word, set on a timed-out wait
-  uint32_t* row_thr;      // [rows] best published k-th value per row (ordered key,
-                          // 0 = none); cleared by launch_score
+  uint32_t* row_thr;      // [rows] best known lower bound of each row's k-th value
+                          // (ordered key, 0 = none)
+  bool thr_seeded;        // row_thr holds seeds; otherwise launch_score clears it
 };
 // Slices the scoring kernel will use for `rows` rows (deterministic per device).
 int score_slices(int rows, int V, int markov_dtype);
 cudaError_t launch_score(const ScoreArgs& a, cudaStream_t s);
 
-// Gather E rows of tokens into Eg (zero padded to r_pad for bf16).
+// Admission seeds of the next scoring launch (seed.cuh). Seed data of the
+// (request b, depth) entry in use: cols/lval/wmax + b * req_stride [ks] and
+// wcol + b * req_stride * r_pad [ks][r_pad]. Null thr: no seeds.
+struct SeedArgs {
+  const int32_t* cols;
+  const float* lval;
+  const float* wmax;
+  const void* wcol;        // bf16
+  long long req_stride;
+  int ks;
+  uint32_t* thr;
+};
+
+// Gather E rows of tokens into Eg (zero padded to r_pad for bf16); with
+// seeds, one row per request (status_div == 1).
 cudaError_t launch_gather_rows(int rows, const int32_t* toks, int V, int r, int r_pad,
                                int markov_dtype, const void* E, void* Eg, int32_t* status,
-                               int status_div, cudaStream_t s);
+                               int status_div, const SeedArgs& seed, cudaStream_t s);
+
+// Seed data for every row of the logits [rows][V] (V % 8 == 0, bf16 W [r][V]):
+// the ks best columns (approximately), L at them, W's columns (bf16, zero
+// padded to r_pad) and their largest magnitude.
+cudaError_t launch_drafter_topk(int rows, int V, int ks, int logits_dtype, const void* L,
+                                const void* W, int r, int r_pad, int32_t* cols, float* lval,
+                                float* wmax, void* wcol, cudaStream_t s);
 
 struct MergeArgs {
   int batch, F_prev, F_new, k, beam, S, V, r, r_pad, markov_dtype, depth;
@@ -91,6 +113,7 @@ struct MergeArgs {
   void* Eg_next;             // null at the last depth
   const int32_t* err;
   int32_t* status;
+  SeedArgs seed;             // next depth's seeds (thr null: none)
 };
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s);
 

@@ -22,9 +22,11 @@
 //             gives every selected node its canonical BFS index; parents are
 //             remapped through the same scan.
 #include <climits>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
+#include "seed.cuh"
 
 namespace pct {
 namespace {
@@ -32,7 +34,7 @@ namespace {
 template <typename TE>
 __global__ void gather_rows_kernel(int rows, const int32_t* __restrict__ toks, int V, int r,
                                    int r_pad, const TE* __restrict__ E, TE* __restrict__ Eg,
-                                   int32_t* __restrict__ status, int status_div) {
+                                   int32_t* __restrict__ status, int status_div, SeedArgs seed) {
   const int row = blockIdx.x;
   if (row >= rows) return;
   int t = toks[row];
@@ -43,6 +45,18 @@ __global__ void gather_rows_kernel(int rows, const int32_t* __restrict__ toks, i
   const TE* src = E + (size_t)t * r;
   TE* dst = Eg + (size_t)row * r_pad;
   for (int j = threadIdx.x; j < r_pad; j += blockDim.x) dst[j] = j < r ? src[j] : TE(0.f);
+  if constexpr (std::is_same<TE, __nv_bfloat16>::value) {
+    if (seed.thr == nullptr) return;
+    // one row per request: its seed from the request's seed data
+    __shared__ __align__(16) SeedSmem sm;
+    const size_t e = (size_t)row * seed.req_stride;
+    const SeedData sd{seed.cols + e, seed.lval + e, seed.wmax + e,
+                      static_cast<const __nv_bfloat16*>(seed.wcol) + e * r_pad};
+    seed_prefetch(sd, seed.ks, r_pad, &sm);
+    seed_prefetch_wait();   // also orders the Eg row written above
+    seed_rows(1, [&](int) { return static_cast<const __nv_bfloat16*>(dst); }, &sm, seed.ks, r_pad,
+              seed.thr + row);
+  }
 }
 
 // Fold the S partials of one row (warp-cooperative). Returns lse and writes
@@ -128,6 +142,16 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
   const int nwarps = kMergeThreads / 32;
   const int F = a.F_prev, k = a.k, C = F * k;
   if (threadIdx.x == 0 && *a.err) atomicOr(&a.status[b], PCT_DEV_TIMEOUT);
+  // the next depth's seed data (W columns) arrive while the merge runs
+  __shared__ __align__(16) SeedSmem seed_sm;
+  const size_t se = (size_t)b * a.seed.req_stride;
+  if constexpr (std::is_same<TE, __nv_bfloat16>::value) {
+    if (a.seed.thr != nullptr) {
+      const SeedData sd{a.seed.cols + se, a.seed.lval + se, a.seed.wmax + se,
+                        static_cast<const __nv_bfloat16*>(a.seed.wcol) + se * a.r_pad};
+      seed_prefetch(sd, a.seed.ks, a.r_pad, &seed_sm);
+    }
+  }
 
   // candidates (score, parent position, token) as ordered keys, a warp per parent row
   for (int i = warp; i < F; i += nwarps) {
@@ -196,6 +220,13 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
       tok = (tok < 0 || tok >= a.V) ? 0 : tok;
       Eg[((size_t)b * Fn + t) * a.r_pad + j] = j < a.r ? E[(size_t)tok * a.r + j] : TE(0.f);
     }
+  }
+  if constexpr (std::is_same<TE, __nv_bfloat16>::value) {
+    if (a.seed.thr == nullptr) return;
+    // next depth's admission seeds for this request's new parents
+    seed_prefetch_wait();   // also orders the Eg rows written above
+    seed_rows(kept, [&](int t) { return static_cast<const __nv_bfloat16*>(Eg) + ((size_t)b * Fn + t) * a.r_pad; },
+              &seed_sm, a.seed.ks, a.r_pad, a.seed.thr + (size_t)b * Fn);
   }
 }
 
@@ -330,20 +361,26 @@ __global__ void rows_finalize_kernel(int rows, int k, int S, Partials part, floa
 
 cudaError_t launch_gather_rows(int rows, const int32_t* toks, int V, int r, int r_pad,
                                int markov_dtype, const void* E, void* Eg, int32_t* status,
-                               int status_div, cudaStream_t s) {
+                               int status_div, const SeedArgs& seed, cudaStream_t s) {
+  if (seed.thr != nullptr && (status_div != 1 || markov_dtype != PCT_BF16 || seed.ks > kSeedMaxK ||
+                              r_pad > kSeedMaxR))
+    return cudaErrorInvalidValue;
   TraceScope t(s, "gather_rows");
   if (markov_dtype == PCT_BF16)
     gather_rows_kernel<__nv_bfloat16><<<rows, 128, 0, s>>>(
         rows, toks, V, r, r_pad, static_cast<const __nv_bfloat16*>(E),
-        static_cast<__nv_bfloat16*>(Eg), status, status_div);
+        static_cast<__nv_bfloat16*>(Eg), status, status_div, seed);
   else
     gather_rows_kernel<float><<<rows, 128, 0, s>>>(rows, toks, V, r, r_pad,
                                                    static_cast<const float*>(E),
-                                                   static_cast<float*>(Eg), status, status_div);
+                                                   static_cast<float*>(Eg), status, status_div, seed);
   return cudaGetLastError();
 }
 
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s) {
+  if (a.seed.thr != nullptr && (a.seed.ks > kSeedMaxK || a.r_pad > kSeedMaxR ||
+                                a.Eg_next == nullptr || a.markov_dtype != PCT_BF16))
+    return cudaErrorInvalidValue;
   TraceScope t(s, "pct_merge_beam");
   const bool bf = a.markov_dtype == PCT_BF16;
 #define PCT_MERGE(KM)                                                                  \

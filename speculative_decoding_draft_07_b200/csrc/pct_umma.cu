@@ -35,10 +35,15 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "umma.cuh"
 
 namespace pct {
 
 cudaError_t launch_score_simt(const ScoreArgs& a, cudaStream_t s);
+// CTA-pair form (pct_umma2.cu), used from pair_rows_min() rows on
+int pair_rows_min();
+int pair_slices(int rows, int V);
+cudaError_t launch_score_pair(const ScoreArgs& a, cudaStream_t s);
 
 namespace {
 
@@ -57,9 +62,18 @@ constexpr int THREADS = 64 + 32 * NUM_EPI_WARPS; // producer + MMA warps + epilo
 constexpr int TMEM_COLS = 512;
 constexpr int LBMAX = 64;                        // request rows of L_d staged per N-tile
 constexpr int L_SLOT_BYTES = 2 * 64 * LBMAX * 2; // two [LB][64] bf16 boxes = 16 KB
+// Folded L_d: a CTA whose rows span at most LFOLD requests adds L_d inside the
+// MMA, as one more K=16 step whose A operand is the rows' one-hot request
+// indicator and whose B operand is the requests' [16][128] L_d tile.
+constexpr int LFOLD = 16;
+constexpr int LF_PART_BYTES = LFOLD * BN * 2;    // [16 K][128 N] bf16 per ring slot = 4 KB
+constexpr int LF_ONEHOT_BYTES = BM * LFOLD * 2;  // [128 rows][16 K] bf16 per row tile = 4 KB
+// L_d modes of the scoring kernel
+constexpr int L_GLOBAL = 0;   // epilogue loads L_d from global memory (L2)
+constexpr int L_STAGE = 1;    // L_d tiles staged in shared memory by TMA, added by the epilogue
+constexpr int L_FOLD = 2;     // L_d added by the tensor cores
 constexpr size_t SMEM_BYTES = 1024 + (size_t)NSUBMAX * KBMAX * A_TILE_BYTES +
                               (size_t)STAGES * B_STAGE_BYTES + 2 * (size_t)L_SLOT_BYTES + 256;
-constexpr long long kTimeoutCycles = 4000000000ll;   // ~2 s at 2 GHz
 
 // Instruction descriptor, kind::f16: D = f32, A = B = bf16, A K-major,
 // B MN-major (W is [r][V], V contiguous), N = 128, M = 128.
@@ -78,205 +92,12 @@ struct UmmaParams {
   uint32_t* row_thr;   // [M] best published k-th value per row (ordered key, 0 = none)
 };
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok) : "r"(addr), "r"(parity) : "memory");
-  return ok != 0;
-}
-// Bounded wait. Gives up when another role has aborted or after the timeout.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                         int32_t* err) {
-  const uint32_t addr = smem_u32(bar);
-  if (mbar_try_wait(addr, parity)) return true;
-  const long long t0 = clock64();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(addr, parity)) return true;
-    if ((it & 255u) == 0u) {
-      if (*abort_flag) return false;
-      if (clock64() - t0 > kTimeoutCycles) {
-        *abort_flag = 1;
-        atomicExch(err, 1);
-        return false;
-      }
-    }
-  }
-}
-// Bounded wait used while draining after an abort (no abort check).
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-  const uint32_t addr = smem_u32(bar);
-  const long long t0 = clock64();
-  while (!mbar_try_wait(addr, parity))
-    if (clock64() - t0 > kTimeoutCycles) return;
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 layout (version 1).
-__device__ __forceinline__ uint64_t make_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
-  return d;
-}
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
-}
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-// 16 consecutive fp32 accumulator columns of this thread's TMEM lane (load
-// and wait in one asm statement).
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[16]) { tmem_ld16(taddr, r); }
-__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[32]);
-
-// 32 consecutive fp32 accumulator columns of this thread's TMEM lane. The
-// load and its wait sit in one asm statement so that no use of the outputs can
-// be scheduled before the data has arrived.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ uint4 ld_shared16(uint32_t addr) {
-  uint4 r;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr));
-  return r;
-}
-
-__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[32]) { tmem_ld32(taddr, r); }
-
-// sum_j 2^(x_j log2 e - m log2 e) over N values, arguments and partial sums
-// in fp32 pairs.
-template <int N>
-__device__ __forceinline__ float chunk_exp_sum(const float (&x)[N], float m) {
-  const float2 l2e = make_float2(kLog2e, kLog2e);
-  const float2 nmb = make_float2(-m * kLog2e, -m * kLog2e);
-  float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
-#pragma unroll
-  for (int j = 0; j < N; j += 4) {
-    const float2 a0 = f2_fma(make_float2(x[j], x[j + 1]), l2e, nmb);
-    const float2 a1 = f2_fma(make_float2(x[j + 2], x[j + 3]), l2e, nmb);
-    sa = f2_add(sa, make_float2(ex2(a0.x), ex2(a0.y)));
-    sb = f2_add(sb, make_float2(ex2(a1.x), ex2(a1.y)));
-  }
-  const float2 t = f2_add(sa, sb);
-  return t.x + t.y;
-}
-
-// max of N values as a tree of three-input maxima
-template <int N>
-__device__ __forceinline__ float chunk_max(const float (&x)[N]) {
-  float t[(N + 2) / 3];
-#pragma unroll
-  for (int j = 0; j < N / 3; ++j) t[j] = fmax3(x[3 * j], x[3 * j + 1], x[3 * j + 2]);
-  if (N % 3 == 1) t[N / 3] = x[N - 1];
-  if (N % 3 == 2) t[N / 3] = fmaxf(x[N - 2], x[N - 1]);
-  constexpr int T = (N + 2) / 3;
-  float u[(T + 2) / 3];
-#pragma unroll
-  for (int j = 0; j < T / 3; ++j) u[j] = fmax3(t[3 * j], t[3 * j + 1], t[3 * j + 2]);
-  if (T % 3 == 1) u[T / 3] = t[T - 1];
-  if (T % 3 == 2) u[T / 3] = fmaxf(t[T - 2], t[T - 1]);
-  constexpr int U = (T + 2) / 3;
-  float r = u[0];
-#pragma unroll
-  for (int j = 1; j < U; ++j) r = fmaxf(r, u[j]);
-  return r;
-}
-
-// N drafter logits of one row starting at column col0 (col0 % N == 0, N a
-// multiple of 8). Columns at or past V read as -inf.
-template <typename TL, int N>
-__device__ __forceinline__ void load_logits(const TL* row, int col0, int V, float (&x)[N]) {
-  if (sizeof(TL) == 4) {
-#pragma unroll
-    for (int j = 0; j < N; ++j) {
-      const int c = col0 + j;
-      x[j] = c < V ? load_f(row + c) : neg_inf();
-    }
-    return;
-  }
-#pragma unroll
-  for (int q = 0; q < N / 8; ++q) {
-    const int c = col0 + q * 8;
-    if (c < V) {   // V % 8 == 0: a 16-byte group is entirely in or out
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(row + c));
-      x[q * 8 + 0] = bf16_lo(w.x); x[q * 8 + 1] = bf16_hi(w.x);
-      x[q * 8 + 2] = bf16_lo(w.y); x[q * 8 + 3] = bf16_hi(w.y);
-      x[q * 8 + 4] = bf16_lo(w.z); x[q * 8 + 5] = bf16_hi(w.z);
-      x[q * 8 + 6] = bf16_lo(w.w); x[q * 8 + 7] = bf16_hi(w.w);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) x[q * 8 + j] = neg_inf();
-    }
-  }
-}
-
-// STAGE: the drafter logits of each N-tile arrive in shared memory by TMA
-// (bf16 logits, every CTA touching at most LBMAX requests); otherwise the
-// epilogue reads them from global memory (L2) itself.
-template <typename TL, int KMAX, bool STAGE>
+// LMODE (L_GLOBAL / L_STAGE / L_FOLD) says how the drafter logits L_d join
+// the Markov product: loaded by the epilogue from global memory (L2); staged
+// per N-tile in shared memory by TMA (bf16 logits, a CTA touching at most LBMAX
+// requests) and added by the epilogue; or folded into the MMA (bf16 logits, at
+// most LFOLD requests per CTA), in which case the accumulator already holds z.
+template <typename TL, int KMAX, int LMODE>
 __global__ void __launch_bounds__(THREADS, 1)
     score_umma_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmL, const UmmaParams p) {
@@ -285,7 +106,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + NSUBMAX * KBMAX * A_TILE_BYTES;
-  uint8_t* sL = sB + STAGES * B_STAGE_BYTES;                     // [2] L_d slots
+  uint8_t* sL = sB + STAGES * B_STAGE_BYTES;   // L_STAGE: [2] L_d slots; L_FOLD: [STAGES] L_d
+                                               // parts, then [2] one-hot tiles
+  uint8_t* sOneHot = sL + STAGES * LF_PART_BYTES;
+  constexpr bool STAGE = LMODE == L_STAGE;
+  constexpr bool FOLD = LMODE == L_FOLD;
   uint64_t* full = reinterpret_cast<uint64_t*>(sL + 2 * L_SLOT_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* afull = empty + STAGES;
@@ -317,6 +142,27 @@ __global__ void __launch_bounds__(THREADS, 1)
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (FOLD && warp >= 2) {
+    // one-hot request indicator of every row (K-major, 32-byte swizzle: the
+    // two 16-byte halves of a row swap in rows 4..7 of each 8-row group)
+    const int e = warp - 2, g = e >> 2, st = g / SPLIT, h = g % SPLIT;
+    const int i = (warp & 3) * 32 + lane;        // row within the tile
+    const int rr = row0 + st * BM + i;
+    if (h == 0 && st < NSUBMAX) {
+      const int kk = (st < p.nsub && rr < p.M) ? rr / p.n_par - row0 / p.n_par : -1;
+      uint8_t* rowp = sOneHot + st * LF_ONEHOT_BYTES + (i >> 3) * 256 + (i & 7) * 32;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int kl = kk - 8 * half;
+        const uint32_t one = 0x3F80u << (16 * (kl & 1));   // bf16 1.0 in its half word
+        const int wi = (kl >= 0 && kl < 8) ? (kl >> 1) : -1;
+        const int phys = half ^ ((i >> 2) & 1);
+        *reinterpret_cast<uint4*>(rowp + 16 * phys) =
+            make_uint4(wi == 0 ? one : 0u, wi == 1 ? one : 0u, wi == 2 ? one : 0u, wi == 3 ? one : 0u);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -355,10 +201,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!wait_bar(&empty[stage], phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
-          mbar_expect_tx(&full[stage], B_STAGE_BYTES);
+          const bool lpart = FOLD && kb == 0;
+          mbar_expect_tx(&full[stage], B_STAGE_BYTES + (lpart ? LF_PART_BYTES : 0));
           uint8_t* dst = sB + stage * B_STAGE_BYTES;
           tma_load_2d(dst, &tmB, n0, kb * BK, &full[stage]);
           tma_load_2d(dst + B_STAGE_BYTES / 2, &tmB, n0 + 64, kb * BK, &full[stage]);
+          if (lpart) {
+            // the CTA's requests' L_d rows as the extra K block: [16 K][2 x 64 N]
+            uint8_t* ldst = sL + stage * LF_PART_BYTES;
+            tma_load_2d(ldst, &tmL, n0, req0, &full[stage]);
+            tma_load_2d(ldst + LF_PART_BYTES / 2, &tmL, n0 + 64, req0, &full[stage]);
+          }
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -388,6 +241,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t phase = 0;
       const uint64_t a_desc0 = make_desc(smem_u32(sA), 16, 1024);      // row tile 0, K block 0
       const uint64_t b_desc0 = make_desc(smem_u32(sB), 8192, 1024);    // ring slot 0
+      // folded L_d: one-hot rows (K-major, 32-byte swizzle, 8-row groups 256
+      // bytes apart) times the L_d part of ring slot `stage` (V-major,
+      // 128-byte swizzle, the two 64-column halves 2048 bytes apart)
+      const uint64_t x_desc0 = make_desc(smem_u32(sOneHot), 16, 256, 6);
+      const uint64_t l_desc0 = make_desc(smem_u32(sL), LF_PART_BYTES / 2, 1024);
       const bool two = p.nsub == 2;
       for (int it = 0; it < ntiles && ok; ++it) {
         const int buf = it & 1;
@@ -411,6 +269,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (two)
               umma_f16(d1, ad + (uint64_t)((KBMAX * A_TILE_BYTES >> 4) + k4 * 2),
                        bd + (uint64_t)(k4 * 128), IDESC, 1u);
+          }
+          if (FOLD && kb == 0) {
+            const uint64_t ld = l_desc0 + (uint64_t)((stage * LF_PART_BYTES) >> 4);
+            umma_f16(d0, x_desc0, ld, IDESC, 1u);
+            if (two) umma_f16(d1, x_desc0 + (uint64_t)(LF_ONEHOT_BYTES >> 4), ld, IDESC, 1u);
           }
           umma_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -441,12 +304,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     float m = neg_inf(), s = 0.f;
     TopK<KMAX> tk;
     tk.init(k);
-    // admission gate: max(own k-th value, best k-th value any slice of this
-    // row has published). Every slice's k-th value is a lower bound of the
-    // row's k-th, so values below the gate cannot be in the row's top-k.
-    float gth = neg_inf();
+    // admission gate: the largest known lower bound of the row's k-th value:
+    // the row's seed (k exact values of the row, stored before the launch),
+    // this slice's own k-th value, and the k-th values other slices of the
+    // row have published. Values below the gate cannot be in the row's top-k.
     uint32_t* thr = p.row_thr + (valid ? row : 0);
-    uint32_t pub_prev = 0;   // loaded at the end of the previous tile, used one tile later
+    uint32_t pub_prev = valid ? *reinterpret_cast<volatile uint32_t*>(thr) : 0u;
+    float gth = pub_prev > f2ord(neg_inf()) ? ord2f(pub_prev) : neg_inf();
     for (int it = 0; it < ntiles; ++it) {
       const int buf = it & 1;
       const uint32_t par = (uint32_t)((it >> 1) & 1);
@@ -456,8 +320,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int n0 = (t_begin + it) * BN;
       const uint32_t tbase =
           tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)((buf * NSUBMAX + st) * BN);
-#pragma unroll 1
-      for (int c = h * (BN / CH / SPLIT); c < (h + 1) * (BN / CH / SPLIT); ++c) {
+      // one chunk of CH accumulator columns (acc already waited for)
+      auto chunk = [&](int c, const uint32_t (&acc)[CH]) {
         const int col0 = n0 + c * CH;
         float x[CH];
         if (STAGE) {
@@ -474,19 +338,23 @@ __global__ void __launch_bounds__(THREADS, 1)
             x[q * 8 + 4] = bf16_lo(w[q].z); x[q * 8 + 5] = bf16_hi(w[q].z);
             x[q * 8 + 6] = bf16_lo(w[q].w); x[q * 8 + 7] = bf16_hi(w[q].w);
           }
-        } else if (valid) {
+        } else if (!FOLD && valid) {
           load_logits<TL, CH>(Lr, col0, V, x);
         }
-        uint32_t acc[CH];
-        tmem_ld(tbase + (uint32_t)(c * CH), acc);
         if (valid) {
-          // z = L + E[p].W in fp32 pairs
+          if (FOLD) {
+            // the accumulator holds z = L + E[p].W
 #pragma unroll
-          for (int j = 0; j < CH; j += 2) {
-            const float2 z2 = f2_add(make_float2(x[j], x[j + 1]),
-                                     make_float2(__uint_as_float(acc[j]), __uint_as_float(acc[j + 1])));
-            x[j] = z2.x;
-            x[j + 1] = z2.y;
+            for (int j = 0; j < CH; ++j) x[j] = __uint_as_float(acc[j]);
+          } else {
+            // z = L + E[p].W in fp32 pairs
+#pragma unroll
+            for (int j = 0; j < CH; j += 2) {
+              const float2 z2 = f2_add(make_float2(x[j], x[j + 1]),
+                                       make_float2(__uint_as_float(acc[j]), __uint_as_float(acc[j + 1])));
+              x[j] = z2.x;
+              x[j + 1] = z2.y;
+            }
           }
           if (col0 + CH > V) {
 #pragma unroll
@@ -524,6 +392,22 @@ __global__ void __launch_bounds__(THREADS, 1)
               }
             }
           }
+        }
+      };
+      // the next chunk's accumulator load is in flight while a chunk is processed
+      constexpr int NCH = BN / CH / SPLIT;
+      const int cb = h * NCH;
+      uint32_t acc_a[CH], acc_b[CH];
+      tmem_issue(tbase + (uint32_t)(cb * CH), acc_a);
+#pragma unroll 1
+      for (int i = 0; i < NCH; i += 2) {
+        tmem_wait(acc_a);
+        if (i + 1 < NCH) tmem_issue(tbase + (uint32_t)((cb + i + 1) * CH), acc_b);
+        chunk(cb + i, acc_a);
+        if (i + 1 < NCH) {
+          tmem_wait(acc_b);
+          if (i + 2 < NCH) tmem_issue(tbase + (uint32_t)((cb + i + 2) * CH), acc_a);
+          chunk(cb + i + 1, acc_b);
         }
       }
       // publish this slice's k-th value for the row and pick up the best one
@@ -587,49 +471,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-// ---------------------------------------------------------------------------
-// Host: tensor maps through the driver entry point (no libcuda link needed).
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
-// 2D bf16 tensor map: `inner` contiguous elements per row, rows `row_bytes`
-// apart (0: dense), 128-byte swizzle or none.
-bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                    uint32_t box_inner, uint32_t box_outer, uint64_t row_bytes = 0,
-                    bool swizzle128 = true) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {row_bytes ? row_bytes : inner * 2};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int umma_nsub(int rows) { return rows > BM ? 2 : 1; }
 
 }  // namespace
 
 int score_slices(int rows, int V, int markov_dtype) {
   const int sms = num_sms();
+  if (markov_dtype == PCT_BF16 && rows >= pair_rows_min()) return pair_slices(rows, V);
   if (markov_dtype == PCT_BF16) {
     const int rpc = BM * umma_nsub(rows);
     const int mtiles = (rows + rpc - 1) / rpc;
@@ -646,6 +494,7 @@ size_t score_smem_bytes() { return SMEM_BYTES; }
 cudaError_t launch_score(const ScoreArgs& a, cudaStream_t s) {
   if (a.markov_dtype != PCT_BF16) return launch_score_simt(a, s);
   const int rows = a.n_req * a.n_par;
+  if (rows >= pair_rows_min()) return launch_score_pair(a, s);
   CUtensorMap tmA, tmB;
   if (!encode_2d_bf16(&tmA, a.Eg, (uint64_t)a.r_pad, (uint64_t)a.M_pad, BK, BM)) return cudaErrorInvalidValue;
   if (!encode_2d_bf16(&tmB, a.W, (uint64_t)a.V, (uint64_t)a.r, 64, BK)) return cudaErrorInvalidValue;
@@ -666,7 +515,8 @@ cudaError_t launch_score(const ScoreArgs& a, cudaStream_t s) {
   p.pidx = a.part.idx;
   p.err = a.err;
   p.row_thr = a.row_thr;
-  if (cudaMemsetAsync(a.row_thr, 0, sizeof(uint32_t) * (size_t)rows, s) != cudaSuccess)
+  if (!a.thr_seeded &&
+      cudaMemsetAsync(a.row_thr, 0, sizeof(uint32_t) * (size_t)rows, s) != cudaSuccess)
     return cudaErrorInvalidValue;
   const int mtiles = (rows + p.rows_per_cta - 1) / p.rows_per_cta;
   // requests any CTA's rows span: stage L_d by TMA when that fits a slot
@@ -675,33 +525,44 @@ cudaError_t launch_score(const ScoreArgs& a, cudaStream_t s) {
     const int r0 = mt * p.rows_per_cta, r1 = std::min(rows, r0 + p.rows_per_cta) - 1;
     span = std::max(span, r1 / a.n_par - r0 / a.n_par + 1);
   }
-  const bool stage = a.logits_dtype == PCT_BF16 && span <= LBMAX;
-  p.LB = stage ? (span + 7) / 8 * 8 : 0;
+  const bool bf16_l = a.logits_dtype == PCT_BF16;
+  const int lmode = !bf16_l ? L_GLOBAL : span <= LFOLD ? L_FOLD : span <= LBMAX ? L_STAGE : L_GLOBAL;
+  p.LB = lmode == L_STAGE ? (span + 7) / 8 * 8 : 0;
   CUtensorMap tmL;
-  if (stage) {
+  if (lmode == L_STAGE) {
     if (!encode_2d_bf16(&tmL, a.L, (uint64_t)a.V, (uint64_t)a.n_req, 64, (uint32_t)p.LB,
                         (uint64_t)a.L_req_stride * 2, false))
+      return cudaErrorInvalidValue;
+  } else if (lmode == L_FOLD) {
+    // [16 requests][64 columns] boxes, 128-byte swizzle (the MMA's B layout);
+    // rows past the last request read as zero
+    if (!encode_2d_bf16(&tmL, a.L, (uint64_t)a.V, (uint64_t)a.n_req, 64, (uint32_t)LFOLD,
+                        (uint64_t)a.L_req_stride * 2, true))
       return cudaErrorInvalidValue;
   } else {
     tmL = tmB;   // unused
   }
   dim3 grid(a.S, mtiles);
   TraceScope t(s, "pct_score_umma");
-#define PCT_UMMA(TL, KM, ST)                                                                    \
+#define PCT_UMMA(TL, KM, LM)                                                                    \
   do {                                                                                          \
-    auto kern = score_umma_kernel<TL, KM, ST>;                                                  \
+    auto kern = score_umma_kernel<TL, KM, LM>;                                                  \
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,     \
                                          (int)SMEM_BYTES);                                      \
     if (e != cudaSuccess) return e;                                                             \
     kern<<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, tmL, p);                                   \
   } while (0)
-  if (stage) {
-    if (a.k <= 4) PCT_UMMA(__nv_bfloat16, 4, true); else if (a.k <= 8) PCT_UMMA(__nv_bfloat16, 8, true); else PCT_UMMA(__nv_bfloat16, 16, true);
-  } else if (a.logits_dtype == PCT_BF16) {
-    if (a.k <= 4) PCT_UMMA(__nv_bfloat16, 4, false); else if (a.k <= 8) PCT_UMMA(__nv_bfloat16, 8, false); else PCT_UMMA(__nv_bfloat16, 16, false);
-  } else {
-    if (a.k <= 4) PCT_UMMA(float, 4, false); else if (a.k <= 8) PCT_UMMA(float, 8, false); else PCT_UMMA(float, 16, false);
-  }
+#define PCT_UMMA_K(TL, LM)                                    \
+  do {                                                        \
+    if (a.k <= 4) PCT_UMMA(TL, 4, LM);                        \
+    else if (a.k <= 8) PCT_UMMA(TL, 8, LM);                   \
+    else PCT_UMMA(TL, 16, LM);                                \
+  } while (0)
+  if (lmode == L_FOLD) PCT_UMMA_K(__nv_bfloat16, L_FOLD);
+  else if (lmode == L_STAGE) PCT_UMMA_K(__nv_bfloat16, L_STAGE);
+  else if (bf16_l) PCT_UMMA_K(__nv_bfloat16, L_GLOBAL);
+  else PCT_UMMA_K(float, L_GLOBAL);
+#undef PCT_UMMA_K
 #undef PCT_UMMA
   return cudaGetLastError();
 }

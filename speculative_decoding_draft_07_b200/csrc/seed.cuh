@@ -1,0 +1,136 @@
+// Admission seeds for the scoring kernel's top-k (PCTree parent scoring).
+//
+// PCTree article (qiita), section on the tree that replaces the chain draft:
+// every frontier parent p keeps the k largest z_d(p) = L_d + Markov(p). The
+// scoring kernel admits a value to its running top-k only at or above a gate,
+// and any k actual values of the row bound the row's k-th largest from below.
+// The seed evaluates z exactly at k columns that are likely to be near the top
+// (the request's best drafter-logit columns of that depth, shared by all of its
+// parents) and stores their minimum, less a rounding allowance that covers the
+// difference between this fp32 dot product and the tensor-core accumulation of
+// the same sum, as the row's starting gate. A loose seed only costs speed; it
+// never excludes a value that belongs to the row's top-k.
+#pragma once
+
+#include "common.cuh"
+
+namespace pct {
+
+// Rounding allowance relative to |L| + sum_j |E_j W_j|: two fp32 sums of the
+// same r <= 256 exact bf16 products (in any order, rounded or truncated) differ
+// by at most about (r + 2) * 2^-23 of that magnitude, below 2^-14; the
+// allowance is 2^-12. sum_j |E_j W_j| is bounded by sum_j |E_j| * max_j |W_j|.
+constexpr float kSeedSlack = 1.0f / 4096.0f;
+constexpr int kSeedMaxK = 16;
+constexpr int kSeedMaxR = 256;
+
+// Per (request, depth) seed data, written by the drafter top-k kernel:
+//   cols [ks]            seed columns (distinct; any entry < 0: no seed)
+//   lval [ks]            L_d at those columns
+//   wmax [ks]            max_j |W[j][col]|
+//   wcol [ks][r_pad]     W[.][col] as bf16, zero padded past r
+struct SeedData {
+  const int32_t* cols;
+  const float* lval;
+  const float* wmax;
+  const __nv_bfloat16* wcol;
+};
+
+// Shared-memory copy of one (request, depth) seed entry.
+struct SeedSmem {
+  __nv_bfloat16 wcol[kSeedMaxK * kSeedMaxR];   // first: 16-byte aligned
+  int32_t cols[kSeedMaxK];
+  float lval[kSeedMaxK];
+  float wmax[kSeedMaxK];
+};
+
+// Copies one seed entry (W columns: ks * r_pad bf16, 16-byte aligned) into
+// shared memory with asynchronous copies, so that their latency overlaps the
+// caller's other work; the caller waits with seed_prefetch_wait() before
+// seed_rows().
+__device__ __forceinline__ void seed_prefetch(const SeedData& sd, int ks, int r_pad,
+                                              SeedSmem* sm) {
+  const int n16 = ks * r_pad / 8;
+  for (int i = threadIdx.x; i < n16; i += blockDim.x) {
+    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(sm->wcol + 8 * i));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(sd.wcol + 8 * i)
+                 : "memory");
+  }
+  for (int i = threadIdx.x; i < 3 * ks; i += blockDim.x) {
+    const int w = i / ks, c = i - w * ks;
+    const void* src = w == 0 ? static_cast<const void*>(sd.cols + c)
+                             : w == 1 ? static_cast<const void*>(sd.lval + c)
+                                      : static_cast<const void*>(sd.wmax + c);
+    void* dstp = w == 0 ? static_cast<void*>(sm->cols + c)
+                        : w == 1 ? static_cast<void*>(sm->lval + c) : static_cast<void*>(sm->wmax + c);
+    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(dstp));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void seed_prefetch_wait() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
+}
+
+// One warp per row: rows t < nrows of one request, parent embedding rows
+// eg_row(t) (bf16, r_pad wide, zero padded, 16-byte aligned) written by this
+// block before a __syncthreads. sm holds the seed entry (seed_prefetch).
+// Writes thr[t] = ordered key of the row's bound, 0 when there is none.
+template <typename EgFn>
+__device__ __forceinline__ void seed_rows(int nrows, EgFn eg_row, const SeedSmem* sm, int ks,
+                                          int r_pad, uint32_t* __restrict__ thr) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const __nv_bfloat16* ws = sm->wcol;
+  bool usable = true;
+#pragma unroll
+  for (int c = 0; c < kSeedMaxK; ++c) usable &= (c >= ks) || sm->cols[c] >= 0;
+  for (int t = warp; t < nrows; t += nw) {
+    const int j0 = 8 * lane;
+    float e[8];
+    if (j0 < r_pad) {
+      const uint4 w = *reinterpret_cast<const uint4*>(eg_row(t) + j0);
+      e[0] = bf16_lo(w.x); e[1] = bf16_hi(w.x); e[2] = bf16_lo(w.y); e[3] = bf16_hi(w.y);
+      e[4] = bf16_lo(w.z); e[5] = bf16_hi(w.z); e[6] = bf16_lo(w.w); e[7] = bf16_hi(w.w);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) e[q] = 0.f;
+    }
+    float e1 = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) e1 += fabsf(e[q]);
+    float d[kSeedMaxK];
+#pragma unroll
+    for (int c = 0; c < kSeedMaxK; ++c) {
+      d[c] = 0.f;
+      if (c < ks && j0 < r_pad) {
+        const uint4 w = *reinterpret_cast<const uint4*>(ws + c * r_pad + j0);
+        d[c] = fmaf(e[0], bf16_lo(w.x), d[c]); d[c] = fmaf(e[1], bf16_hi(w.x), d[c]);
+        d[c] = fmaf(e[2], bf16_lo(w.y), d[c]); d[c] = fmaf(e[3], bf16_hi(w.y), d[c]);
+        d[c] = fmaf(e[4], bf16_lo(w.z), d[c]); d[c] = fmaf(e[5], bf16_hi(w.z), d[c]);
+        d[c] = fmaf(e[6], bf16_lo(w.w), d[c]); d[c] = fmaf(e[7], bf16_hi(w.w), d[c]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      e1 += __shfl_xor_sync(0xffffffffu, e1, o);
+#pragma unroll
+      for (int c = 0; c < kSeedMaxK; ++c)
+        if (c < ks) d[c] += __shfl_xor_sync(0xffffffffu, d[c], o);
+    }
+    float lo_min = __int_as_float(0x7f800000);
+    bool finite = usable;
+#pragma unroll
+    for (int c = 0; c < kSeedMaxK; ++c) {
+      if (c < ks) {
+        const float l = sm->lval[c];
+        const float lo = (l + d[c]) - (fabsf(l) + e1 * sm->wmax[c]) * kSeedSlack;
+        finite = finite && (lo == lo) && lo != __int_as_float(0x7f800000);
+        lo_min = fminf(lo_min, lo);
+      }
+    }
+    if (lane == 0) thr[t] = (finite && lo_min > neg_inf()) ? f2ord(lo_min) : 0u;
+  }
+}
+
+}  // namespace pct

@@ -54,13 +54,11 @@ def _score_ref(L_row, ptok, E, W, k):
     return (np.stack(lse_all), np.stack(tok_all), np.stack(lp_all), near_all)
 
 
-@pytest.mark.parametrize("dtype,V,r,k,batch,n_par", [
-    ("bf16", 1024, 64, 4, 1, 1), ("bf16", 1024, 16, 8, 3, 40), ("bf16", 2048, 100, 8, 2, 200),
-    ("bf16", 4096, 256, 16, 3, 100), ("bf16", 64, 64, 1, 2, 5), ("bf16", 1000, 256, 8, 1, 130),
-    ("f32", 1000, 16, 4, 2, 7), ("f32", 777, 33, 8, 3, 20)])
-def test_score_parents_matches_oracle(dtype, V, r, k, batch, n_par):
+def _score_parents_case(dtype, V, r, k, batch, n_par, logits_dtype=None):
     L, _, E, W = _problem(batch, 1, V, r, seed=V + r + k, dtype=dtype)
     L = L[:, 0, :].contiguous()
+    if logits_dtype is not None:
+        L = L.to(logits_dtype)
     g = torch.Generator().manual_seed(k)
     ptok = torch.randint(0, V, (batch, n_par), generator=g, dtype=torch.int64).to(torch.int32)
     lse, tt, tl, st = pct.pct_score_parents(L.to(DEV), ptok.to(DEV), E.to(DEV), W.to(DEV), k)
@@ -82,6 +80,33 @@ def test_score_parents_matches_oracle(dtype, V, r, k, batch, n_par):
             np.testing.assert_allclose(gl[b, p], rlp[b, p], rtol=0, atol=SCORE_TOL)
     assert skipped <= max(1, batch * n_par // 50)
     assert (host(st) == 0).all()
+
+
+@pytest.mark.parametrize("dtype,V,r,k,batch,n_par", [
+    ("bf16", 1024, 64, 4, 1, 1), ("bf16", 1024, 16, 8, 3, 40), ("bf16", 2048, 100, 8, 2, 200),
+    ("bf16", 4096, 256, 16, 3, 100), ("bf16", 64, 64, 1, 2, 5), ("bf16", 1000, 256, 8, 1, 130),
+    ("f32", 1000, 16, 4, 2, 7), ("f32", 777, 33, 8, 3, 20)])
+def test_score_parents_matches_oracle(dtype, V, r, k, batch, n_par):
+    _score_parents_case(dtype, V, r, k, batch, n_par)
+
+
+@pytest.mark.parametrize("batch,n_par,mode", [
+    (3, 40, "fold, one row tile"), (4, 64, "fold, two row tiles"),
+    (5, 100, "fold, requests straddle CTAs"), (16, 16, "fold, 16 requests per CTA"),
+    (24, 2, "staged tiles, 24 requests per CTA"), (80, 1, "global loads, 80 requests per CTA"),
+    (40, 4, "CTA pairs, global loads, 40 requests per pair"),
+    (2, 65, "CTA pairs, fold, second CTA nearly empty")])
+def test_score_parents_logits_modes(batch, n_par, mode):
+    """The tensor-core path adds L_d in the MMA (at most 16 requests per CTA or
+    CTA pair), in the epilogue from staged shared-memory tiles (at most 64, up to
+    128 rows), or from global memory (more); more than 128 rows run on CTA pairs.
+    Each mode against the oracle."""
+    _score_parents_case("bf16", 3000, 128, 8, batch, n_par)
+
+
+@pytest.mark.parametrize("batch,n_par", [(3, 30), (3, 60)])
+def test_score_parents_fp32_logits_bf16_markov(batch, n_par):
+    _score_parents_case("bf16", 2000, 64, 8, batch, n_par, logits_dtype=torch.float32)
 
 
 def _build_and_compare(L, anchor, E, W, k, beam, N, sample=None, max_excluded=0.2, label=""):
@@ -127,6 +152,32 @@ def test_zero_markov_exact_ties():
     W = torch.zeros_like(W)
     L[0, 1, 10:20] = 6.0          # ten identical peaks
     _build_and_compare(L, anchor, E, W, 8, 16, 64, max_excluded=0.0, label="w0")
+
+
+def test_seeded_gate_with_ties_across_slices():
+    """W = 0 and twelve equal peaks spread over the vocabulary: each row's k-th
+    value is a tie held by columns in different V-slices, and the row's seeded
+    gate sits just below it (the rounding allowance); the lower token ids win."""
+    L, anchor, E, W = _problem(2, 3, 8192, 64, seed=21, sigma=1.0)
+    W = torch.zeros_like(W)
+    for b in range(2):
+        for d in range(3):
+            L[b, d, torch.arange(12) * 677 + 5 + d] = 6.0
+    _build_and_compare(L, anchor, E, W, 8, 16, 40, max_excluded=0.0, label="ties")
+
+
+def test_strong_markov_loose_seed():
+    """Markov term several times larger than the drafter logits: the drafter's
+    best columns are not the parents' best, so every seed is loose."""
+    L, anchor, E, W = _problem(8, 4, 4096, 128, seed=23, sigma=0.5, ew=0.6)
+    _build_and_compare(L, anchor, E, W, 8, 16, 64, max_excluded=0.25, label="strong markov")
+
+
+def test_vocab_too_small_for_seed_columns():
+    """V = 64 has eight 8-column groups, fewer than k = 16 seed columns: the
+    rows are scored without seeds."""
+    L, anchor, E, W = _problem(2, 3, 64, 32, seed=25)
+    _build_and_compare(L, anchor, E, W, 16, 32, 60, label="v64")
 
 
 def test_repeated_builds_are_bit_identical():

@@ -549,7 +549,10 @@ cudaError_t launch_score(const ScoreArgs& a, cudaStream_t s) {
     auto kern = score_umma_kernel<TL, KM, LM>;                                                  \
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,     \
                                          (int)SMEM_BYTES);                                      \
-    if (e != cudaSuccess) return e;                                                             \
+    if (e != cudaSuccess) {                                                                     \
+      (void)cudaGetLastError();                                                                 \
+      return e;                                                                                 \
+    }                                                                                           \
     kern<<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, tmL, p);                                   \
   } while (0)
 #define PCT_UMMA_K(TL, LM)                                    \

@@ -50,8 +50,11 @@ constexpr int P_A_BLOCK = P_BM * P_BK * 2;           // 16 KB per K block
 constexpr int P_B_STAGE = P_BK * P_HALF * 2;         // 16 KB per ring slot
 constexpr int P_EPI_WARPS = 16;                      // 4 per TMEM lane quarter
 constexpr int P_THREADS = 64 + 32 * P_EPI_WARPS;
-constexpr int P_CH = 16;                             // accumulator columns per TMEM load
+constexpr int P_CH = 32;                             // accumulator columns per chunk
+constexpr bool P_PREFETCH = false;                   // next chunk's TMEM load in flight
+static_assert(P_CH == 16 || P_CH == 32, "a chunk's candidate mask is one 32-bit word");
 constexpr int P_COLS_PER_WARP = P_BN / 4;            // 64
+constexpr int P_SOFT = 0;   // of every 16 exponentials on the FMA pipe (0, 2, 4, 6 measured: 0 fastest)
 constexpr int P_LFOLD = 16;
 constexpr int P_LPART = P_LFOLD * P_HALF * 2;        // [16 K][128 N] = 4 KB per slot
 constexpr int P_ONEHOT = P_BM * P_LFOLD * 2;         // [128 rows][16 K] = 4 KB
@@ -340,11 +343,11 @@ __global__ void __launch_bounds__(P_THREADS, 1)
         // sum of exp against the running reference m, which moves only when a
         // value exceeds it by more than 64 (the chunk is then summed again)
         float csum = 0.f;
-        if (m != neg_inf()) csum = chunk_exp_sum<P_CH>(x, m);
+        if (m != neg_inf()) csum = chunk_exp_sum<P_CH, P_SOFT>(x, m);
         if (cm > m + 64.f) {
           s = (m == neg_inf()) ? 0.f : s * ex2((m - cm) * kLog2e);
           m = cm;
-          csum = chunk_exp_sum<P_CH>(x, m);
+          csum = chunk_exp_sum<P_CH, P_SOFT>(x, m);
         }
         s += csum;
         if (cm >= gth) {
@@ -364,18 +367,28 @@ __global__ void __launch_bounds__(P_THREADS, 1)
           }
         }
       };
-      // the next chunk's accumulator load is in flight while a chunk is processed
-      constexpr int NCH = P_COLS_PER_WARP / P_CH;   // 4
-      uint32_t acc_a[P_CH], acc_b[P_CH];
-      tmem_issue(tbase, acc_a);
+      constexpr int NCH = P_COLS_PER_WARP / P_CH;
+      if (P_PREFETCH) {
+        // the next chunk's accumulator load is in flight while a chunk is processed
+        uint32_t acc_a[P_CH], acc_b[P_CH];
+        tmem_issue(tbase, acc_a);
 #pragma unroll 1
-      for (int i = 0; i < NCH; i += 2) {
-        tmem_wait(acc_a);
-        tmem_issue(tbase + (uint32_t)((i + 1) * P_CH), acc_b);
-        chunk(i, acc_a);
-        tmem_wait(acc_b);
-        if (i + 2 < NCH) tmem_issue(tbase + (uint32_t)((i + 2) * P_CH), acc_a);
-        chunk(i + 1, acc_b);
+        for (int i = 0; i < NCH; i += 2) {
+          tmem_wait(acc_a);
+          tmem_issue(tbase + (uint32_t)((i + 1) * P_CH), acc_b);
+          chunk(i, acc_a);
+          tmem_wait(acc_b);
+          if (i + 2 < NCH) tmem_issue(tbase + (uint32_t)((i + 2) * P_CH), acc_a);
+          chunk(i + 1, acc_b);
+        }
+      } else {
+#pragma unroll 1
+        for (int i = 0; i < NCH; ++i) {
+          uint32_t acc[P_CH];
+          tmem_issue(tbase + (uint32_t)(i * P_CH), acc);
+          tmem_wait(acc);
+          chunk(i, acc);
+        }
       }
       if (valid) {
         if (pub_prev > f2ord(neg_inf())) gth = fmaxf(gth, ord2f(pub_prev));
@@ -501,9 +514,15 @@ cudaError_t launch_score_pair(const ScoreArgs& a, cudaStream_t s) {
     auto kern = score_pair_kernel<TL, KM, FD>;                                                \
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
                                          (int)P_SMEM);                                        \
-    if (e != cudaSuccess) return e;                                                           \
+    if (e != cudaSuccess) {                                                                   \
+      (void)cudaGetLastError();                                                               \
+      return e;                                                                               \
+    }                                                                                         \
     e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmL, p);                                     \
-    if (e != cudaSuccess) return e;                                                           \
+    if (e != cudaSuccess) {                                                                   \
+      (void)cudaGetLastError(); /* leave no launch error behind for later calls */            \
+      return e;                                                                               \
+    }                                                                                         \
   } while (0)
 #define PCT_PAIR_K(TL, FD)                        \
   do {                                            \

@@ -122,6 +122,32 @@ __device__ __forceinline__ void tmem_wait(uint32_t (&r)[16]) {
                :
                : "memory");
 }
+__device__ __forceinline__ void tmem_issue(uint32_t taddr, uint32_t (&r)[32]) {
+  tmem_issue(taddr, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+  tmem_issue(taddr + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+}
+__device__ __forceinline__ void tmem_wait(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_issue(uint32_t taddr, uint32_t (&r)[64]) {
+  tmem_issue(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  tmem_issue(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+}
+// (the second wait finds no load outstanding; it only fences the upper half)
+__device__ __forceinline__ void tmem_wait(uint32_t (&r)[64]) {
+  tmem_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  tmem_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+}
+
 __device__ __forceinline__ uint4 ld_shared16(uint32_t addr) {
   uint4 r;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -130,21 +156,52 @@ __device__ __forceinline__ uint4 ld_shared16(uint32_t addr) {
 }
 
 
+// 2^t of a pair on the FMA pipe (no SFU). t is clamped below at -125 (the
+// smaller terms of a softmax sum underflow anyway); t <= 92 holds for every
+// caller (values exceed the running reference by at most 64 nats). Cody-Waite
+// style split t = n + f with n = round(t), taken from the low mantissa bits of
+// t + 1.5 * 2^23, and f in [-1/2, 1/2]; 2^f by the degree-5 polynomial that
+// interpolates 2^f at the six Chebyshev nodes of [-1/2, 1/2] (coefficients
+// rounded to fp32; relative error below 1.1e-7, about 2.2e-7 with the fp32
+// Horner evaluation); n is added to the exponent field.
+constexpr float kExp2C0 = 1.00000012f, kExp2C1 = 0.693147182f, kExp2C2 = 0.240221068f,
+                kExp2C3 = 0.0555035695f, kExp2C4 = 0.00967603177f, kExp2C5 = 0.00133908633f;
+__device__ __forceinline__ float2 soft_exp2x2(float2 t) {
+  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+  t.x = fmaxf(t.x, -125.0f);
+  t.y = fmaxf(t.y, -125.0f);
+  const float2 r = f2_add(t, make_float2(kRound, kRound));
+  const float2 n = f2_add(r, make_float2(-kRound, -kRound));
+  const float2 f = f2_fma(n, make_float2(-1.0f, -1.0f), t);
+  float2 q = f2_fma(make_float2(kExp2C5, kExp2C5), f, make_float2(kExp2C4, kExp2C4));
+  q = f2_fma(q, f, make_float2(kExp2C3, kExp2C3));
+  q = f2_fma(q, f, make_float2(kExp2C2, kExp2C2));
+  q = f2_fma(q, f, make_float2(kExp2C1, kExp2C1));
+  q = f2_fma(q, f, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(r.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(r.y) << 23)));
+}
+
 // sum_j 2^(x_j log2 e - m log2 e) over N values, arguments and partial sums
-// in fp32 pairs.
-template <int N>
+// in fp32 pairs. The last SOFT values of the chunk take soft_exp2x2 (FMA
+// pipe), the rest the SFU, so that the two units share the work.
+template <int N, int SOFT = 0>
 __device__ __forceinline__ float chunk_exp_sum(const float (&x)[N], float m) {
+  static_assert(SOFT % 2 == 0 && SOFT <= N, "soft share in pairs");
   const float2 l2e = make_float2(kLog2e, kLog2e);
   const float2 nmb = make_float2(-m * kLog2e, -m * kLog2e);
-  float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
+  // four independent partial sums (pairs) keep several SFU results in flight
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
 #pragma unroll
-  for (int j = 0; j < N; j += 4) {
-    const float2 a0 = f2_fma(make_float2(x[j], x[j + 1]), l2e, nmb);
-    const float2 a1 = f2_fma(make_float2(x[j + 2], x[j + 3]), l2e, nmb);
-    sa = f2_add(sa, make_float2(ex2(a0.x), ex2(a0.y)));
-    sb = f2_add(sb, make_float2(ex2(a1.x), ex2(a1.y)));
+  for (int j = 0; j < N; j += 2) {
+    const float2 a = f2_fma(make_float2(x[j], x[j + 1]), l2e, nmb);
+    float2 e;
+    if (j >= N - SOFT) e = soft_exp2x2(a);
+    else e = make_float2(ex2(a.x), ex2(a.y));
+    acc[(j >> 1) & 3] = f2_add(acc[(j >> 1) & 3], e);
   }
-  const float2 t = f2_add(sa, sb);
+  const float2 t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
   return t.x + t.y;
 }
 

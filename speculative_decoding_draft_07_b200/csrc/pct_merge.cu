@@ -59,18 +59,21 @@ __global__ void gather_rows_kernel(int rows, const int32_t* __restrict__ toks, i
   }
 }
 
-// Fold the S partials of one row (warp-cooperative). Returns lse and writes
-// the row's k best (value desc, token asc) to out_v / out_i: each lane folds
-// its slices' lists into a register top-k, then k rounds of "take the best
-// head across the warp, the owner pops".
-template <int KMAX>
+// Fold the S partials of one row with a group of G lanes (G = 16 or 32, the
+// group aligned within the warp; every lane of the warp calls it). Returns lse
+// and writes the row's k best (value desc, token asc) to out_v / out_i. Each
+// lane takes its slices' lists (sorted by the scoring kernel: a lane with a
+// single slice copies it, more are merged into it), then k rounds of "take the
+// best head across the group, the owner pops".
+template <int KMAX, int G>
 __device__ __forceinline__ float merge_row(const Partials& part, size_t row, int S, int k,
                                            float* out_v, int* out_i) {
-  const int lane = threadIdx.x & 31;
+  const int gl = threadIdx.x & (G - 1);
   float m = neg_inf(), s = 0.f;
   TopK<KMAX> tk;
   tk.init(k);
-  for (int sl = lane; sl < S; sl += 32) {
+  bool first = true;
+  for (int sl = gl; sl < S; sl += G) {
     const size_t ps = row * S + sl;
     const float2 ms = part.ms[ps];
     lse_combine(m, s, ms.x, ms.y);
@@ -81,13 +84,19 @@ __device__ __forceinline__ float merge_row(const Partials& part, size_t row, int
       v[j] = j < k ? part.val[ps * k + j] : neg_inf();
       id[j] = j < k ? part.idx[ps * k + j] : 0x7fffffff;
     }
+    if (first && k == KMAX) {
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j)
-      if (j < k && tk.admits(v[j], id[j])) tk.insert(v[j], id[j]);
+      for (int j = 0; j < KMAX; ++j) { tk.v[j] = v[j]; tk.i[j] = id[j]; }
+    } else {
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (j < k && tk.admits(v[j], id[j])) tk.insert(v[j], id[j]);
+    }
+    first = false;
   }
   tk.finish(k);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
+  for (int o = G / 2; o > 0; o >>= 1) {
     const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
     lse_combine(m, s, m2, s2);
   }
@@ -97,11 +106,43 @@ __device__ __forceinline__ float merge_row(const Partials& part, size_t row, int
     if (j >= k) break;
     float v = tk.v[0];
     int i = tk.i[0];
-    warp_best(v, i);
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) {
+      const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+      const int i2 = __shfl_xor_sync(0xffffffffu, i, o);
+      if (better(v2, i2, v, i)) { v = v2; i = i2; }
+    }
     if (tk.v[0] == v && tk.i[0] == i) tk.pop();
-    if (lane == 0) { out_v[j] = v; out_i[j] = i; }
+    if (gl == 0) { out_v[j] = v; out_i[j] = i; }
   }
   return lse;
+}
+
+// 64-bit keys, one per lane: bitonic sort of the warp's 32 keys, descending.
+__device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long x, int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, stride);
+      const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0 || size == 32);
+      x = keep_max ? (x > y ? x : y) : (x < y ? x : y);
+    }
+  }
+  return x;
+}
+// a, b sorted descending across the warp (one key per lane): the 32 largest of
+// their union, sorted descending (elementwise max against b reversed is a
+// bitonic sequence holding them; one bitonic merge sorts it).
+__device__ __forceinline__ unsigned long long warp_merge_top(unsigned long long a,
+                                                             unsigned long long b_rev, int lane) {
+  unsigned long long x = a > b_rev ? a : b_rev;
+#pragma unroll
+  for (int stride = 16; stride > 0; stride >>= 1) {
+    const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, stride);
+    x = ((lane & stride) == 0) ? (x > y ? x : y) : (x < y ? x : y);
+  }
+  return x;
 }
 
 constexpr int kMergeThreads = 512;
@@ -135,8 +176,10 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
   __shared__ unsigned long long keys[kMaxCand];
   __shared__ unsigned long long ck[256];
   __shared__ float kept_s[256];
-  __shared__ float wv[kMergeThreads / 32][16];
-  __shared__ int wi[kMergeThreads / 32][16];
+  __shared__ float wv[kMergeThreads / 32][32];
+  __shared__ int wi[kMergeThreads / 32][32];
+  // the next depth's parent embeddings (bf16), kept for the seeds (up to 32 rows)
+  __shared__ __align__(16) uint16_t egs[32 * kSeedMaxR];
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = kMergeThreads / 32;
@@ -153,22 +196,56 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
     }
   }
 
-  // candidates (score, parent position, token) as ordered keys, a warp per parent row
-  for (int i = warp; i < F; i += nwarps) {
-    const size_t row = (size_t)b * F + i;
-    const float lse = merge_row<KMAX>(a.part, row, a.S, k, wv[warp], wi[warp]);
-    __syncwarp();
-    const float sp = a.prev_s ? a.prev_s[(size_t)b * a.prev_stride + i] : 0.f;
-    for (int j = lane; j < k; j += 32) keys[i * k + j] = cand_key(sp + (wv[warp][j] - lse), i, wi[warp][j]);
-    __syncwarp();
+  // candidates (score, parent position, token) as ordered keys: a half warp
+  // per parent row when a row has at most 16 V-slices, else a warp
+  if (a.S <= 16) {
+    const int h = lane >> 4, gl = lane & 15;
+    for (int i0 = 2 * warp; i0 < F; i0 += 2 * nwarps) {
+      const int i = i0 + h;
+      const size_t row = (size_t)b * F + min(i, F - 1);   // both halves take part in the shuffles
+      const float lse = merge_row<KMAX, 16>(a.part, row, a.S, k, wv[warp] + 16 * h, wi[warp] + 16 * h);
+      __syncwarp();
+      if (i < F) {
+        const float sp = a.prev_s ? a.prev_s[(size_t)b * a.prev_stride + i] : 0.f;
+        for (int j = gl; j < k; j += 16)
+          keys[i * k + j] = cand_key(sp + (wv[warp][16 * h + j] - lse), i, wi[warp][16 * h + j]);
+      }
+      __syncwarp();
+    }
+  } else {
+    for (int i = warp; i < F; i += nwarps) {
+      const size_t row = (size_t)b * F + i;
+      const float lse = merge_row<KMAX, 32>(a.part, row, a.S, k, wv[warp], wi[warp]);
+      __syncwarp();
+      const float sp = a.prev_s ? a.prev_s[(size_t)b * a.prev_stride + i] : 0.f;
+      for (int j = lane; j < k; j += 32) keys[i * k + j] = cand_key(sp + (wv[warp][j] - lse), i, wi[warp][j]);
+      __syncwarp();
+    }
   }
-  int P = 1;
+  int P = 32;
   while (P < C) P <<= 1;
   for (int t = C + threadIdx.x; t < P; t += blockDim.x) keys[t] = 0ull;
   __syncthreads();
   // beam: the best `beam` candidates under (score desc, parent position asc, token asc)
-  bitonic_desc_block(keys, P);
   const int kept = min(a.beam, C);
+  if (kept <= 32) {
+    // every 32-key chunk sorted by a warp, then pairs of chunks merged to their
+    // top 32 until one chunk is left (keys are distinct: parent, token)
+    for (int c = warp; c < P / 32; c += nwarps)
+      keys[32 * c + lane] = warp_sort_desc(keys[32 * c + lane], lane);
+    __syncthreads();
+    for (int width = 1; width < P / 32; width <<= 1) {
+      for (int c = warp * 2 * width; c < P / 32; c += nwarps * 2 * width) {
+        if (c + width < P / 32) {
+          const unsigned long long x = keys[32 * c + lane], y = keys[32 * (c + width) + 31 - lane];
+          keys[32 * c + lane] = warp_merge_top(x, y, lane);
+        }
+      }
+      __syncthreads();
+    }
+  } else {
+    bitonic_desc_block(keys, P);
+  }
   // canonical order of the kept: ascending (parent position, token); the beam
   // rank rides along in the low bits to find the score again
   int Q = 1;
@@ -185,7 +262,16 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
     }
   }
   __syncthreads();
-  bitonic_desc_block(ck, Q);
+  if (Q <= 32) {
+    if (warp == 0) {
+      const unsigned long long x = lane < Q ? ck[lane] : 0ull;
+      const unsigned long long y = warp_sort_desc(x, lane);
+      if (lane < Q) ck[lane] = y;
+    }
+    __syncthreads();
+  } else {
+    bitonic_desc_block(ck, Q);
+  }
   for (int t = threadIdx.x; t < kept; t += blockDim.x) {
     const unsigned long long x = ~ck[t];
     const size_t o = (size_t)b * a.beam + t;
@@ -201,6 +287,8 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
   constexpr int per16 = 16 / (int)sizeof(TE);
   const bool vec = (a.r % per16 == 0) && (a.r_pad % per16 == 0) &&
                    ((reinterpret_cast<uintptr_t>(E) & 15u) == 0);
+  const bool stash = std::is_same<TE, __nv_bfloat16>::value && a.seed.thr != nullptr &&
+                     kept <= 32 && a.r_pad <= kSeedMaxR;
   if (vec) {
     const int rv = a.r / per16, rpv = a.r_pad / per16;
     for (int idx = threadIdx.x; idx < kept * rpv; idx += blockDim.x) {
@@ -211,6 +299,7 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
       const uint4 val = j < rv ? reinterpret_cast<const uint4*>(E + (size_t)tok * a.r)[j]
                                : make_uint4(0u, 0u, 0u, 0u);
       reinterpret_cast<uint4*>(Eg + ((size_t)b * Fn + t) * a.r_pad)[j] = val;
+      if (stash) reinterpret_cast<uint4*>(egs + t * a.r_pad)[j] = val;
     }
   } else {
     for (int idx = threadIdx.x; idx < kept * a.r_pad; idx += blockDim.x) {
@@ -225,8 +314,12 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
     if (a.seed.thr == nullptr) return;
     // next depth's admission seeds for this request's new parents
     seed_prefetch_wait();   // also orders the Eg rows written above
-    seed_rows(kept, [&](int t) { return static_cast<const __nv_bfloat16*>(Eg) + ((size_t)b * Fn + t) * a.r_pad; },
-              &seed_sm, a.seed.ks, a.r_pad, a.seed.thr + (size_t)b * Fn);
+    if (stash && vec)
+      seed_rows(kept, [&](int t) { return reinterpret_cast<const __nv_bfloat16*>(egs + t * a.r_pad); },
+                &seed_sm, a.seed.ks, a.r_pad, a.seed.thr + (size_t)b * Fn);
+    else
+      seed_rows(kept, [&](int t) { return static_cast<const __nv_bfloat16*>(Eg) + ((size_t)b * Fn + t) * a.r_pad; },
+                &seed_sm, a.seed.ks, a.r_pad, a.seed.thr + (size_t)b * Fn);
   }
 }
 
@@ -345,7 +438,7 @@ __global__ void rows_finalize_kernel(int rows, int k, int S, Partials part, floa
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + warp;
   if (row >= rows) return;
-  const float lse = merge_row<KMAX>(part, row, S, k, wv[warp], wi[warp]);
+  const float lse = merge_row<KMAX, 32>(part, row, S, k, wv[warp], wi[warp]);
   __syncwarp();
   for (int j = lane; j < k; j += 32) {
     top_tok[(size_t)row * k + j] = wi[warp][j];

@@ -389,6 +389,81 @@ def run_reference(args, rank, world, budget_s: float = 120.0):
     return 0
 
 
+def run_configs(args):
+    """One line per configuration of the hot path (not the default bench line):
+    GPU rounds/s over --steps timed runs after --warmup, the dominant kernel's
+    rate against the measured peak, and the oracle timed on one request of the
+    same inputs (host cores), scaled to the configuration's batch."""
+    import oracle
+    import speculative_decoding_draft_07_b200 as pct
+    dev = torch.device("cuda", 0)
+    pk, pk_src = peaks()
+    f64 = lambda t: t.detach().cpu().double().numpy() if t.dtype != torch.bfloat16 else \
+        t.detach().cpu().float().double().numpy()
+    lines = []
+
+    def gpu_rate(fn):
+        for _ in range(args.warmup):
+            fn()
+        return args.steps / (timed(fn, args.steps, dev) / 1e3)
+
+    def oracle_requests_per_s(fn):   # the oracle on one request
+        t0 = time.perf_counter()
+        fn()
+        return 1.0 / (time.perf_counter() - t0)
+
+    for name in ("tiny", "qwen3_4b_scale", "long_block"):
+        w = workloads.WORKLOADS[name]
+        d = workloads.drafter_inputs(w, device=dev)
+        L, a, E, Wm = d["L"], d["anchor"], d["E"], d["W"]
+        r = gpu_rate(lambda: pct.pct_tree_build(L, a, E, Wm, w.k, w.beam, w.n_nodes))
+        F = [1]
+        for _ in range(w.depth):
+            F.append(min(w.beam, F[-1] * w.k))
+        rows = sum(w.batch * F[d_ - 1] for d_ in range(1, w.depth + 1))
+        flop = 2.0 * w.rank * w.vocab * rows
+        wbytes = float(w.rank * w.vocab * (2 if w.dtype == "bf16" else 4) * w.depth)
+        o_rate = oracle_requests_per_s(lambda: oracle.pct_tree_build(
+            f64(L[:1]), a[:1].cpu().numpy(), f64(E), f64(Wm), w.k, w.beam, w.n_nodes))
+        lines.append({"config": name, "rounds_per_s": r, "requests": w.batch,
+                      "tflops": flop * r / 1e12, "frac_bf16_sustained": flop * r / 1e12 /
+                      float(pk["bf16_tflops_sustained"]),
+                      "w_stream_gbs": wbytes * r / 1e9,
+                      "frac_hbm": wbytes * r / 1e9 / float(pk["hbm_gbs"]),
+                      "oracle_rounds_per_s": o_rate / w.batch, "oracle_sample": "1 request"})
+    for ell in C.ells:
+        d = workloads.cadd_inputs(C, ell, device=dev)
+        L, a, ctx = d["L"], d["anchor"], d["ctx_len"]
+        r = gpu_rate(lambda: pct.cadd_tree_grow(L, a, ctx, C.n_max, **COST))
+        nbytes = float(L.numel() * L.element_size())
+        o_rate = oracle_requests_per_s(lambda: oracle.cadd_tree_grow(
+            f64(L[:1]), a[:1].cpu().numpy(), ctx[:1].cpu().numpy(), C.n_max, **COST))
+        lines.append({"config": f"caddtree_l{ell}", "rounds_per_s": r, "requests": C.batch,
+                      "gbs": nbytes * r / 1e9, "frac_hbm": nbytes * r / 1e9 / float(pk["hbm_gbs"]),
+                      "oracle_rounds_per_s": o_rate / C.batch, "oracle_sample": "1 request"})
+    for ln in lines:
+        print(json.dumps({k: (round(v, 6) if isinstance(v, float) else v) for k, v in ln.items()}))
+    return 0
+
+
+def run_stage(args):
+    """One stage of the round, repeated, with only its own inputs on the device
+    (the drafter logits and Markov parameters: about 0.45 GB), so that ncu
+    captures of its kernels stay small."""
+    import speculative_decoding_draft_07_b200 as pct
+    dev = torch.device("cuda", 0)
+    rnd = RoundInputs(dev)
+    for _ in range(args.warmup + args.steps):
+        if args.profile_stage == "pctree":
+            out = pct.pct_tree_build(rnd.L, rnd.anchor, rnd.E, rnd.W, W.k, W.beam, W.n_nodes)
+        else:
+            out = pct.cadd_tree_grow(rnd.L, rnd.anchor, rnd.ctx, C.n_max, **COST)
+    torch.cuda.synchronize(dev)
+    print(f"{args.profile_stage}: {args.warmup + args.steps} runs, status "
+          f"{int(out.status.abs().sum().item())}, nodes {int(out.count.sum().item())}")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -399,9 +474,19 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--requests", type=int, default=W.batch,
                     help="requests per round (smaller only for profiling captures)")
+    ap.add_argument("--profile-stage", default=None, choices=["pctree", "cadd"],
+                    help="for profiler captures: run only this stage of the round on its "
+                         "inputs, --warmup + --steps times, and print no bench line")
+    ap.add_argument("--configs", action="store_true",
+                    help="time every configuration of the hot path (one line each) instead of "
+                         "the full round")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     set_requests(args.requests)
+    if args.profile_stage is not None:
+        return run_stage(args)
+    if args.configs:
+        return run_configs(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -183,7 +183,7 @@ int check_cadd(const cadd_desc* d) {
   return PCT_OK;
 }
 struct CaddPlan {
-  size_t o_lse, o_cnt, o_q, o_tok, total;
+  size_t o_lse, o_cnt, o_q, o_tok, o_seg, seg_bytes, total;
 };
 void cadd_plan(const cadd_desc* d, CaddPlan* P) {
   const size_t rows = (size_t)d->batch * d->depth;
@@ -193,6 +193,8 @@ void cadd_plan(const cadd_desc* d, CaddPlan* P) {
   P->o_cnt = o; o += align_up(rows * sizeof(int32_t));
   P->o_q = o;   o += align_up(rows * K1 * sizeof(float));
   P->o_tok = o; o += align_up(rows * K1 * sizeof(int32_t));
+  P->seg_bytes = cadd_seg_workspace(d->batch, d->depth, d->vocab, d->logits_dtype);
+  P->o_seg = o; o += align_up(P->seg_bytes);
   P->total = o;
 }
 
@@ -446,7 +448,8 @@ int32_t cadd_tree_grow(const cadd_desc* desc, const void* L, const int32_t* anch
                desc->C_d, desc->a, desc->b, desc->c, desc->e};
   PCT_CU(launch_cadd(p, L, anchor, ctx_len, tok, parent, depth, score, count, phi, dev_status,
                      reinterpret_cast<float*>(ws + P.o_lse), reinterpret_cast<int32_t*>(ws + P.o_cnt),
-                     reinterpret_cast<float*>(ws + P.o_q), reinterpret_cast<int32_t*>(ws + P.o_tok), s));
+                     reinterpret_cast<float*>(ws + P.o_q), reinterpret_cast<int32_t*>(ws + P.o_tok),
+                     P.seg_bytes ? ws + P.o_seg : nullptr, s));
   return PCT_OK;
 }
 

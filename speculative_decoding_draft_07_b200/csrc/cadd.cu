@@ -123,15 +123,15 @@ __device__ __forceinline__ void for_row(const T* x, int V, bool vec, F&& f) {
   if (sizeof(T) == 2 && vec) {
     const uint4* p = reinterpret_cast<const uint4*>(x);
     const int nvec = V >> 3;
-    for (int c = threadIdx.x; c < nvec; c += kRowThreads) {
+    for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
       const uint4 q = p[c];
       const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
       for (int j = 0; j < 8; ++j) f((j & 1) ? bf16_hi(w[j >> 1]) : bf16_lo(w[j >> 1]), c * 8 + j);
     }
-    for (int v = (nvec << 3) + threadIdx.x; v < V; v += kRowThreads) f(elem(x, v), v);
+    for (int v = (nvec << 3) + threadIdx.x; v < V; v += blockDim.x) f(elem(x, v), v);
   } else {
-    for (int v = threadIdx.x; v < V; v += kRowThreads) f(elem(x, v), v);
+    for (int v = threadIdx.x; v < V; v += blockDim.x) f(elem(x, v), v);
   }
 }
 
@@ -159,28 +159,6 @@ __device__ float cadd_ln_theta(const CaddParams& p, double ell, int lane, bool r
   }
   if (report && lane == 0 && bad) atomicOr(status_b, PCT_DEV_BAD_COST);
   return (nonpos || th >= 1e299) ? neg_inf() : (float)log(th);
-}
-
-// ln(theta) in fp32 by one warp: its rounding error (about 1e-6 relative) is
-// far inside the kThetaSlack subtracted before use, so the filter stays a
-// superset of the double-precision one. dC(n) = c + e (2n + 1) >= 0 since
-// c, e >= 0 (checked on the host).
-__device__ float cadd_ln_theta_f(const CaddParams& p, float ell, int lane) {
-  const float cb = p.C_d + p.a + p.b * ell;
-  float th = __int_as_float(0x7f800000);
-  int nonpos = 0;
-  for (int n = 1 + lane; n < p.n_max; n += 32) {
-    const float fn = (float)n;
-    const float Cn = cb + p.c * fn + p.e * fn * fn;
-    const float dC = p.c + p.e * (2.0f * fn + 1.0f);
-    if (dC <= 0.0f) nonpos = 1; else if (Cn > 0.0f) th = fminf(th, dC / Cn);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    th = fminf(th, __shfl_xor_sync(0xffffffffu, th, o));
-    nonpos |= __shfl_xor_sync(0xffffffffu, nonpos, o);
-  }
-  return (nonpos || th == __int_as_float(0x7f800000)) ? neg_inf() : logf(th);
 }
 
 // Keep (value, token) in the candidate buffer; the counter keeps counting past
@@ -440,23 +418,35 @@ __global__ __launch_bounds__(kRowThreads, 3) void cadd_rowpass_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Row pass on CTA clusters (bf16 rows, 16-byte aligned, V <= kClSegs * 40960):
-// a cluster of kClSegs CTAs per (request, depth) row. Each CTA copies its
-// segment of the row into shared memory with bulk asynchronous copies (in
-// pieces, so the first is reduced while the others land), folds it into a
-// partial log-sum-exp, and writes the partial into the leader CTA's shared
-// memory. After a cluster barrier every CTA combines the kClSegs partials in
-// segment order into the row's log-sum-exp and the exact threshold
-// lse + ln(theta), filters its staged segment against it, and appends the
-// survivors to the leader's buffer (distributed shared memory). After a second
-// barrier the leader sorts them (value desc, token asc) and writes the first
-// n_max - 1; if the buffer overflowed (theta tiny) it selects them exactly over
-// the row instead. HBM sees the row once.
+// Segmented row pass (bf16 rows, 16-byte aligned, V % 8 == 0), two kernels.
+//  * cadd_seg_rowpass_kernel: every row is cut into S segments of at most
+//    kSegG * kSegThreads 16-byte groups, one kSegThreads-thread block per
+//    (row, segment), with no dependence between blocks. The segment is loaded
+//    straight into registers (kSegG 16-byte loads per thread in flight), folded
+//    into a partial log-sum-exp against each thread's own maximum, and filtered
+//    against the segment's own threshold lse_seg + ln(theta): since lse_seg <=
+//    lse of the row, that keeps a superset of the row's survivors. They go to
+//    the segment's slot of a buffer in global memory, with the partial and the
+//    count beside them.
+//  * cadd_seg_finish_kernel, one block per row: combines the S partials into
+//    the row's lse, keeps the buffered values above the exact threshold
+//    lse + ln(theta), sorts them (value desc, token asc) and writes the first
+//    n_max - 1; if a segment's slot overflowed (theta tiny) it selects them
+//    exactly over the row instead.
+// HBM sees every row once; the survivors add a few KB per row.
 
-constexpr int kClSegs = 8;
-constexpr int kClPiece = 16384;                 // bytes per bulk copy
-constexpr int kClSegMax = 5 * kClPiece;         // segment bytes staged (80 KB)
-constexpr int kClCap = 1024;                    // survivors buffered in the leader
+constexpr int kSegThreads = 128;
+constexpr int kSegG = 10;                 // 16-byte groups per thread (80 values)
+constexpr int kSegCap = 256;              // survivors buffered per segment
+constexpr int kSegFinCap = 1024;          // exact survivors sorted per row (>= n_max - 1)
+constexpr float kSegMargin = 1e-3f;       // covers the rounding of lse_seg against lse
+
+// Segments of a row of V values (V % 8 == 0).
+__host__ __device__ __forceinline__ int seg_count(int V) {
+  const int ngroups = V / 8;
+  const int per = kSegG * kSegThreads;
+  return ngroups < per ? 1 : (ngroups + per - 1) / per;
+}
 
 // Elementwise max of two packed bf16 pairs.
 __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
@@ -464,237 +454,293 @@ __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
   asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
-
-__device__ __forceinline__ uint32_t cl_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cl_map0(const void* p) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, 0;"
-               : "=r"(r) : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
-  return r;
-}
-__device__ __forceinline__ void cl_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
-__device__ __forceinline__ uint32_t cl_smem(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+__device__ __forceinline__ float group_max(const uint4& q) {
+  const uint32_t mx = bf16x2_max(bf16x2_max(q.x, q.y), bf16x2_max(q.z, q.w));
+  return fmaxf(bf16_lo(mx), bf16_hi(mx));
 }
 
-__global__ __launch_bounds__(kRowThreads, 2) void cadd_cluster_rowpass_kernel(
-    CaddParams p, const __nv_bfloat16* __restrict__ L, const int64_t* __restrict__ ctx,
-    float* __restrict__ row_lse, int32_t* __restrict__ cand_cnt, float* __restrict__ cand_q,
-    int32_t* __restrict__ cand_tok, int32_t* __restrict__ status) {
-  extern __shared__ __align__(128) uint8_t cl_smem_raw[];
-  uint8_t* segbuf = cl_smem_raw;                         // this CTA's segment (seg_cap bytes)
-  __shared__ __align__(8) uint64_t bars[kClSegMax / kClPiece];
-  __shared__ float2 part[kClSegs];       // leader: the segments' partial (max, sum)
-  __shared__ int s_cnt;                  // leader: survivors appended
-  __shared__ float sm[32], ss[32];
-  __shared__ int sbuf[32];
-  __shared__ int hist[256];
-  __shared__ int s_n;
-  __shared__ float s_lnth;
-  __shared__ int s_timeout;
+// Sum of s_i 2^((m_i - M) log2 e) with M the block-wide max of m_i, in a fixed
+// order (thread, then lane tree, then warps in order), so every block that
+// reduces the same values gets the same bits. Returns (M, sum) in every thread.
+__device__ float2 block_lse_fixed(float m, float s, float2* wred) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float M = m;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float sc = (m == neg_inf()) ? 0.f : s * ex2((m - M) * kLog2e);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+  if (lane == 0) wred[warp] = make_float2(M, sc);
+  __syncthreads();
+  constexpr int nw = kSegThreads / 32;
+  float BM = neg_inf();
+#pragma unroll
+  for (int w = 0; w < nw; ++w) BM = fmaxf(BM, wred[w].x);
+  float BS = 0.f;
+#pragma unroll
+  for (int w = 0; w < nw; ++w) {
+    const float2 e = wred[w];
+    if (e.x != neg_inf()) BS += e.y * ex2((e.x - BM) * kLog2e);
+  }
+  __syncthreads();   // wred is reused by the caller's next reduction
+  return make_float2(BM, BS);
+}
 
-  const uint32_t rank = cl_rank();
-  const int d = blockIdx.x / kClSegs, b = blockIdx.y;
+// Descending bitonic sort of one key per lane across a warp.
+__device__ __forceinline__ unsigned long long warp_sort_desc_u64(unsigned long long v, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, j);
+      const bool keep_max = ((lane & k) == 0) == ((lane & j) == 0);
+      v = keep_max ? (o > v ? o : v) : (o < v ? o : v);
+    }
+  }
+  return v;
+}
+
+// ln(theta) for context length ell, theta = min over n in [1, n_max - 1] of
+// dC(n) / C(n), in closed form: with c, e >= 0, C is nondecreasing, and
+// f(n) = dC(n) / C(n) has f' of the sign of -2e^2 n^2 - 2e(c + e) n + (2eA -
+// c^2 - ce) (A = C_d + a + b l), a parabola opening downwards: f only falls,
+// or rises and then falls, for n > 0, so its minimum over an interval is at an
+// end, and theta = min(f(1), f(n_max - 1)) when C(1) > 0. -inf (no token can be
+// excluded) when c = e = 0 or C(1) <= 0 (a cost the growth reports as bad);
+// fp32 rounding (about 1e-6 relative) stays far inside the slack the filter
+// subtracts.
+__device__ __forceinline__ float cadd_ln_theta_closed(const CaddParams& p, float ell) {
+  if (p.n_max < 2) return neg_inf();
+  const float A = p.C_d + p.a + p.b * ell;
+  const float C1 = A + p.c + p.e;
+  if (!(p.c > 0.f || p.e > 0.f) || !(C1 > 0.f)) return neg_inf();
+  const float n1 = (float)(p.n_max - 1);
+  const float f1 = (p.c + 3.f * p.e) / C1;
+  const float fN = (p.c + p.e * (2.f * n1 + 1.f)) / (A + p.c * n1 + p.e * n1 * n1);
+  return logf(fminf(f1, fN));
+}
+
+struct SegWs {
+  float* lnth;                 // [rows] filter offset ln(theta) - slack
+  float2* part;                // [rows][S] partial (max, sum)
+  int* cnt;                    // [rows][S] survivors of the segment (may exceed kSegCap)
+  unsigned long long* surv;    // [rows][S][kSegCap] survivor keys
+};
+
+__global__ __launch_bounds__(kSegThreads, 6) void cadd_seg_rowpass_kernel(
+    CaddParams p, const __nv_bfloat16* __restrict__ L, const int64_t* __restrict__ ctx, SegWs w) {
+  __shared__ float2 wred[kSegThreads / 32];
+  __shared__ uint4 stg_v[kSegThreads / 32][kSegG * 32];   // candidate groups, per warp
+  __shared__ int stg_g[kSegThreads / 32][kSegG * 32];
+  __shared__ int s_cnt;
+
   const int V = p.V;
-  const size_t row = (size_t)b * p.D + d;
-  const __nv_bfloat16* x = L + row * (size_t)V;
+  const int S = seg_count(V);
+  const int row = blockIdx.x / S, seg = blockIdx.x - row * S;
+  const int b = row / p.D;
   const int K = p.n_max - 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ngroups = V / 8;                             // V % 8 == 0 on this path
-  const int g_per = (ngroups + kClSegs - 1) / kClSegs;
-  const int g_begin = min(ngroups, (int)rank * g_per), g_end = min(ngroups, g_begin + g_per);
-  const int seg_bytes = (g_end - g_begin) * 16;
-  const int npieces = (seg_bytes + kClPiece - 1) / kClPiece;
-  // survivors buffer after the largest segment (same offset in every CTA)
-  unsigned long long* keys =
-      reinterpret_cast<unsigned long long*>(segbuf + (g_per * 16 + 127) / 128 * 128);   // [kClCap]
+  const int ngroups = V >> 3;
+  const int g_per = (ngroups + S - 1) / S;
+  const int g0 = min(ngroups, seg * g_per);
+  const int ng = min(ngroups, g0 + g_per) - g0;
+  const uint4* src = reinterpret_cast<const uint4*>(L + (size_t)row * V) + g0;
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < npieces; ++i) {
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(cl_smem(&bars[i])));
+  // the whole segment in flight: kSegG independent 16-byte loads per thread
+  // (groups past the segment read as -inf)
+  uint4 q[kSegG];
+#pragma unroll
+  for (int j = 0; j < kSegG; ++j) {
+    const int g = j * kSegThreads + threadIdx.x;
+    q[j] = g < ng ? ld_stream16(src + g) : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+  }
+  if (threadIdx.x == 0) s_cnt = 0;
+  const float lnth = cadd_ln_theta_closed(p, (float)ctx[b]) - kThetaSlack;
+
+  // partial log-sum-exp against the thread's own maximum (no rescaling)
+  float m = neg_inf();
+#pragma unroll
+  for (int j = 0; j < kSegG; ++j) m = fmaxf(m, group_max(q[j]));
+  float s = 0.f;
+  if (m != neg_inf()) {
+    const float2 nmb = make_float2(-m * kLog2e, -m * kLog2e);
+    const float2 l2e = make_float2(kLog2e, kLog2e);
+    float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < kSegG; ++j) {
+      const uint4 v = q[j];
+      const float2 a0 = f2_fma(make_float2(bf16_lo(v.x), bf16_hi(v.x)), l2e, nmb);
+      const float2 a1 = f2_fma(make_float2(bf16_lo(v.y), bf16_hi(v.y)), l2e, nmb);
+      const float2 a2 = f2_fma(make_float2(bf16_lo(v.z), bf16_hi(v.z)), l2e, nmb);
+      const float2 a3 = f2_fma(make_float2(bf16_lo(v.w), bf16_hi(v.w)), l2e, nmb);
+      acc0 = f2_add(acc0, f2_add(make_float2(ex2(a0.x), ex2(a0.y)), make_float2(ex2(a1.x), ex2(a1.y))));
+      acc1 = f2_add(acc1, f2_add(make_float2(ex2(a2.x), ex2(a2.y)), make_float2(ex2(a3.x), ex2(a3.y))));
     }
-    s_cnt = 0;
-    s_timeout = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    const float2 acc = f2_add(acc0, acc1);
+    s = acc.x + acc.y;
+  }
+  const float2 ps = block_lse_fixed(m, s, wred);
+  const float lse_seg = (ps.x == neg_inf()) ? neg_inf() : ps.x + logf(ps.y);
+  const float t_loc = (K <= 0) ? __int_as_float(0x7f800000) : lse_seg + lnth - kSegMargin;
+
+  // the segment's values above its own threshold, into its slot. Groups whose
+  // max reaches it are first packed per warp into shared memory (ballot
+  // compaction), then tested value by value one group per lane, so the rare
+  // candidates cost no divergent passes over the registers.
+  int nst = 0;   // staged groups of this warp
+#pragma unroll
+  for (int j = 0; j < kSegG; ++j) {
+    const bool c = group_max(q[j]) > t_loc;
+    const unsigned ball = __ballot_sync(0xffffffffu, c);
+    if (c) {
+      const int at = nst + __popc(ball & ((1u << lane) - 1u));
+      stg_v[warp][at] = q[j];
+      stg_g[warp][at] = g0 + j * kSegThreads + threadIdx.x;
+    }
+    nst += __popc(ball);
+  }
+  __syncwarp();
+  const size_t slot = (size_t)row * S + seg;
+  unsigned long long* out = w.surv + slot * kSegCap;
+  for (int r0 = 0; r0 < nst; r0 += 32) {
+    const int i = r0 + lane;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    int g = 0;
+    uint32_t vm = 0;
+    if (i < nst) {
+      v = stg_v[warp][i];
+      g = stg_g[warp][i];
+      vm = (uint32_t)(bf16_lo(v.x) > t_loc) | (uint32_t)(bf16_hi(v.x) > t_loc) << 1 |
+           (uint32_t)(bf16_lo(v.y) > t_loc) << 2 | (uint32_t)(bf16_hi(v.y) > t_loc) << 3 |
+           (uint32_t)(bf16_lo(v.z) > t_loc) << 4 | (uint32_t)(bf16_hi(v.z) > t_loc) << 5 |
+           (uint32_t)(bf16_lo(v.w) > t_loc) << 6 | (uint32_t)(bf16_hi(v.w) > t_loc) << 7;
+    }
+    const int cnt = __popc(vm);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int base = 0;
+    if (lane == 31 && incl > 0) base = atomicAdd(&s_cnt, incl);
+    int pos = __shfl_sync(0xffffffffu, base, 31) + (incl - cnt);
+    while (vm) {
+      const int e = __ffs(vm) - 1;
+      vm &= vm - 1;
+      const uint32_t wd = (e >> 1) == 0 ? v.x : (e >> 1) == 1 ? v.y : (e >> 1) == 2 ? v.z : v.w;
+      const float z = (e & 1) ? bf16_hi(wd) : bf16_lo(wd);
+      if (pos < kSegCap) out[pos] = cand_key(z, g * 8 + e);
+      ++pos;
+    }
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    // the whole segment in flight at once: one bulk copy per piece
-    const char* src = reinterpret_cast<const char*>(x) + (size_t)g_begin * 16;
-    for (int i = 0; i < npieces; ++i) {
-      const int bytes = min(kClPiece, seg_bytes - i * kClPiece);
-      const uint32_t bar = cl_smem(&bars[i]);
-      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                   : "memory");
-      asm volatile(
-          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-              cl_smem(segbuf + i * kClPiece)),
-          "l"(src + (size_t)i * kClPiece), "r"(bytes), "r"(bar)
-          : "memory");
-    }
+    w.part[slot] = ps;
+    w.cnt[slot] = s_cnt;
+    if (seg == 0) w.lnth[row] = lnth;
   }
-  if (warp == 1 && rank == 0) {   // the leader's copy is read by the whole cluster
-    const float lt = cadd_ln_theta_f(p, (float)ctx[b], lane);
-    if (lane == 0) s_lnth = lt - kThetaSlack;
-  }
-  if (warp == 2 && rank == 0 && d == 0) (void)cadd_ln_theta(p, (double)ctx[b], lane, true, &status[b]);
+}
 
-  // pass 1: partial log-sum-exp of the segment, piece by piece as they land.
-  // Each thread sums 2^((z - m) log2 e) against its own reference m, which
-  // moves only when a group exceeds it by more than 64 (so no term overflows);
-  // m starts finite so that leading -inf values add 0 instead of NaN.
-  float m = -1e30f, s = 0.f;
-  float2 acc = make_float2(0.f, 0.f);
-  float2 nmb = make_float2(1e30f * kLog2e, 1e30f * kLog2e);
-  const float2 l2e = make_float2(kLog2e, kLog2e);
-  const uint4* sv = reinterpret_cast<const uint4*>(segbuf);
-  for (int i = 0; i < npieces; ++i) {
-    // bounded wait for piece i by one warp; the others sleep in the block barrier
-    if (warp == 0) {
-      const uint32_t bar = cl_smem(&bars[i]);
-      const long long t0 = clock64();
-      uint32_t ok = 0;
-      while (!ok) {
-        asm volatile(
-            "{\n\t.reg .pred q;\n\tmbarrier.try_wait.parity.shared::cta.b64 q, [%1], 0, 20000;\n\t"
-            "selp.u32 %0, 1, 0, q;\n\t}"
-            : "=r"(ok) : "r"(bar) : "memory");
-        if (!ok && clock64() - t0 > 4000000000ll) { s_timeout = 1; break; }
-      }
-    }
-    __syncthreads();
-    const int gi0 = i * (kClPiece / 16);
-    const int gi1 = min(g_end - g_begin, gi0 + kClPiece / 16);
-    for (int g = gi0 + threadIdx.x; g < gi1; g += kRowThreads) {
-      const uint4 q = sv[g];
-      float f[8];
-      f[0] = bf16_lo(q.x); f[1] = bf16_hi(q.x); f[2] = bf16_lo(q.y); f[3] = bf16_hi(q.y);
-      f[4] = bf16_lo(q.z); f[5] = bf16_hi(q.z); f[6] = bf16_lo(q.w); f[7] = bf16_hi(q.w);
-      const float cm = fmaxf(fmax3(f[0], f[1], f[2]), fmax3(f[3], fmax3(f[4], f[5], f[6]), f[7]));
-      if (cm > m + 64.f) {
-        s = (s + acc.x + acc.y) * ex2((m - cm) * kLog2e);
-        acc = make_float2(0.f, 0.f);
-        m = cm;
-        nmb = make_float2(-m * kLog2e, -m * kLog2e);
-      }
-      const float2 a0 = f2_fma(make_float2(f[0], f[1]), l2e, nmb);
-      const float2 a1 = f2_fma(make_float2(f[2], f[3]), l2e, nmb);
-      const float2 a2 = f2_fma(make_float2(f[4], f[5]), l2e, nmb);
-      const float2 a3 = f2_fma(make_float2(f[6], f[7]), l2e, nmb);
-      const float2 e01 = f2_add(make_float2(ex2(a0.x), ex2(a0.y)), make_float2(ex2(a1.x), ex2(a1.y)));
-      const float2 e23 = f2_add(make_float2(ex2(a2.x), ex2(a2.y)), make_float2(ex2(a3.x), ex2(a3.y)));
-      acc = f2_add(acc, f2_add(e01, e23));
-    }
+__global__ __launch_bounds__(kSegThreads) void cadd_seg_finish_kernel(
+    CaddParams p, const __nv_bfloat16* __restrict__ L, const int64_t* __restrict__ ctx, SegWs w,
+    float* __restrict__ row_lse, int32_t* __restrict__ cand_cnt, float* __restrict__ cand_q,
+    int32_t* __restrict__ cand_tok, int32_t* __restrict__ status) {
+  __shared__ float2 wred[kSegThreads / 32];
+  __shared__ unsigned long long keys[kSegFinCap];
+  __shared__ int cnt_sm[kSegThreads];
+  __shared__ int hist[256];
+  __shared__ int sbuf[32];
+  __shared__ int s_n;
+
+  const int V = p.V;
+  const int S = seg_count(V);
+  const int row = blockIdx.x;
+  const int b = row / p.D, d = row - b * p.D;
+  const int K = p.n_max - 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const __nv_bfloat16* x = L + (size_t)row * V;
+
+  // C(n) <= 0 for some n: reported once per request
+  if (d == 0 && warp == 1) (void)cadd_ln_theta(p, (double)ctx[b], lane, true, &status[b]);
+
+  // one round trip for the partials, the counts and the threshold offset;
+  // the row's lse from the partials in a fixed order
+  if (threadIdx.x == 0) s_n = 0;
+  const float lnth = w.lnth[row];
+  float pm = neg_inf(), pss = 0.f;
+  int over = 0;   // some segment's slot overflowed
+  for (int g = threadIdx.x; g < S; g += kSegThreads) {
+    const float2 e = w.part[(size_t)row * S + g];
+    const int c = w.cnt[(size_t)row * S + g];
+    if (g < kSegThreads) cnt_sm[g] = c;
+    over |= c > kSegCap;
+    lse_combine(pm, pss, e.x, e.y);
   }
-  s += acc.x + acc.y;
-  if (!(s > 0.f)) { m = neg_inf(); s = 0.f; }   // nothing finite seen
-  block_lse(m, s, sm, ss);
-  // the segment's partial into the leader, then every CTA sees all of them
-  if (threadIdx.x == 0) {
-    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(cl_map0(&part[rank])), "f"(m), "f"(s)
-                 : "memory");
-  }
-  cl_sync();
-  float lm = neg_inf(), ls = 0.f;
-  for (int g = 0; g < kClSegs; ++g) {   // segment order: independent of arrival
-    float pm, ps;
-    asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(pm), "=f"(ps) : "r"(cl_map0(&part[g])));
-    lse_combine(lm, ls, pm, ps);
-  }
-  const float lse = (lm == neg_inf()) ? neg_inf() : lm + logf(ls);
-  float lnth;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(lnth) : "r"(cl_map0(&s_lnth)));
+  const float2 rl = block_lse_fixed(pm, pss, wred);   // its barriers publish cnt_sm
+  const float lse = (rl.x == neg_inf()) ? neg_inf() : rl.x + logf(rl.y);
   const float t = (K <= 0) ? __int_as_float(0x7f800000) : lse + lnth;
 
-  // pass 2: the segment's values above the exact threshold, into the leader
-  const uint32_t cnt_addr = cl_map0(&s_cnt);
-  const uint32_t keys_addr = cl_map0(keys);
-  const int ng = g_end - g_begin;
-  for (int g0 = 0; g0 < ng; g0 += kRowThreads) {   // uniform trip count for the warp scans
-    const int g = g0 + threadIdx.x;
-    float f[8];
-    int cnt = 0;
-    if (g < ng) {
-      const uint4 q = sv[g];
-      // the group's max by packed bf16 maxima (exact: every bf16 value is an
-      // fp32 value), the exact per-value test only for groups that reach t
-      const uint32_t mx = bf16x2_max(bf16x2_max(q.x, q.y), bf16x2_max(q.z, q.w));
-      if (fmaxf(bf16_lo(mx), bf16_hi(mx)) > t) {
-        f[0] = bf16_lo(q.x); f[1] = bf16_hi(q.x); f[2] = bf16_lo(q.y); f[3] = bf16_hi(q.y);
-        f[4] = bf16_lo(q.z); f[5] = bf16_hi(q.z); f[6] = bf16_lo(q.w); f[7] = bf16_hi(q.w);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) cnt += f[j] > t;
+  // buffered survivors above the exact threshold, kFinSegs segments per batch
+  // of loads (a window of kSegThreads segments' counts at a time)
+  int n = 0;
+  if (K > 0) {
+    constexpr int kFinSegs = 16;
+    constexpr int kSlots = kSegCap / kSegThreads;   // keys per thread per segment
+    for (int w0 = 0; w0 < S; w0 += kSegThreads) {
+      const int nwin = min(kSegThreads, S - w0);
+      if (w0 > 0) {
+        __syncthreads();
+        if (threadIdx.x < nwin) cnt_sm[threadIdx.x] = w.cnt[(size_t)row * S + w0 + threadIdx.x];
+        __syncthreads();
       }
-    }
-    if (__ballot_sync(0xffffffffu, cnt > 0)) {
-      int incl = cnt;
+      for (int s0 = 0; s0 < nwin; s0 += kFinSegs) {
+        unsigned long long kk[kFinSegs * kSlots];
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      uint32_t pos = 0;
-      if (lane == 31)
-        asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(pos) : "r"(cnt_addr), "r"(incl)
-                     : "memory");
-      pos = __shfl_sync(0xffffffffu, pos, 31) + (uint32_t)(incl - cnt);
-      if (cnt > 0) {
-        const int v0 = (g_begin + g) * 8;
+        for (int u = 0; u < kFinSegs; ++u) {
+          const int sg = s0 + u;
+          const int c = sg < nwin ? min(cnt_sm[sg], kSegCap) : 0;
+          const unsigned long long* in = w.surv + ((size_t)row * S + w0 + sg) * kSegCap;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (f[j] > t) {
-            if (pos < (uint32_t)kClCap) {
-              const unsigned long long kk = cand_key(f[j], v0 + j);
-              asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(keys_addr + 8u * pos), "l"(kk)
-                           : "memory");
-            }
-            ++pos;
+          for (int h = 0; h < kSlots; ++h) {
+            const int j = h * kSegThreads + threadIdx.x;
+            kk[u * kSlots + h] = j < c ? in[j] : 0ull;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kFinSegs * kSlots; ++u) {
+          if (kk[u] != 0ull && ord2f((unsigned)(kk[u] >> 32)) > t) {
+            const int at = atomicAdd(&s_n, 1);
+            if (at < kSegFinCap) keys[at] = kk[u];
           }
         }
       }
     }
-  }
-  cl_sync();   // every survivor is in the leader; no CTA touches another's memory after this
-  if (s_timeout) {
-    // a copy that never completed: report it and give it (bounded) time to land
-    // before this CTA's shared memory is released
-    if (threadIdx.x == 0) {
-      atomicOr(&status[b], PCT_DEV_TIMEOUT);
-      for (int i = 0; i < npieces; ++i) {
-        const uint32_t bar = cl_smem(&bars[i]);
-        const long long t0 = clock64();
-        uint32_t ok = 0;
-        while (!ok && clock64() - t0 < 4000000000ll)
-          asm volatile(
-              "{\n\t.reg .pred q;\n\tmbarrier.try_wait.parity.shared::cta.b64 q, [%1], 0;\n\t"
-              "selp.u32 %0, 1, 0, q;\n\t}"
-              : "=r"(ok) : "r"(bar) : "memory");
-      }
-    }
     __syncthreads();
+    n = s_n;
   }
-  if (rank != 0) return;
-  int n = s_cnt;
-  if (K > 0 && n > kClCap) {
+  over = __syncthreads_or(over);
+  if (K > 0 && (over || n > kSegFinCap)) {
     select_topk_exact(x, V, true, K, keys, hist, sbuf, &s_n);
     n = K;
   }
-  int P = 1;
-  while (P < n) P <<= 1;
-  for (int j = n + threadIdx.x; j < P; j += kRowThreads) keys[j] = 0ull;
-  __syncthreads();
-  if (P > 1) bitonic_desc(keys, P);
+  if (n <= 32) {
+    if (warp == 0) {
+      unsigned long long v = lane < n ? keys[lane] : 0ull;
+      v = warp_sort_desc_u64(v, lane);
+      keys[lane] = v;
+    }
+    __syncthreads();
+  } else {
+    int P = 1;
+    while (P < n) P <<= 1;
+    for (int j = n + threadIdx.x; j < P; j += kSegThreads) keys[j] = 0ull;
+    __syncthreads();
+    bitonic_desc(keys, P);
+  }
   const int keep = min(n, max(K, 0));
-  const size_t cbase = row * (size_t)max(K, 1);
-  for (int j = threadIdx.x; j < keep; j += kRowThreads) {
+  const size_t cbase = (size_t)row * (size_t)max(K, 1);
+  for (int j = threadIdx.x; j < keep; j += kSegThreads) {
     const unsigned long long kk = keys[j];
     cand_q[cbase + j] = ord2f((unsigned)(kk >> 32)) - lse;
     cand_tok[cbase + j] = (int)(~(unsigned)(kk & 0xffffffffu));
@@ -838,36 +884,43 @@ size_t cadd_rowpass_bytes_per_row(int n_max) {
   return K1 * (sizeof(float) + sizeof(int32_t)) + sizeof(float) + sizeof(int32_t);
 }
 
+static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+size_t cadd_seg_workspace(int batch, int D, int V, int dtype) {
+  if (dtype != PCT_BF16 || V % 8 != 0) return 0;
+  const size_t rows = (size_t)batch * D, slots = rows * seg_count(V);
+  return align256(rows * sizeof(float)) + align256(slots * sizeof(float2)) +
+         align256(slots * sizeof(int)) + slots * kSegCap * sizeof(unsigned long long);
+}
+
 cudaError_t launch_cadd(const CaddParams& p, const void* L, const int32_t* anchor,
                         const int64_t* ctx, int32_t* tok, int32_t* parent, int32_t* depth,
                         float* score, int32_t* count, float* phi, int32_t* status,
                         float* row_lse, int32_t* cand_cnt, float* cand_q, int32_t* cand_tok,
-                        cudaStream_t s) {
-  const int cl_seg = (p.V / 8 + kClSegs - 1) / kClSegs * 16;   // bytes of the largest segment
-  const bool cluster = p.dtype == PCT_BF16 && p.V % 8 == 0 &&
-                       (reinterpret_cast<uintptr_t>(L) & 15u) == 0 && cl_seg <= kClSegMax;
-  if (cluster) {
-    const size_t smem = (size_t)(cl_seg + 127) / 128 * 128 + (size_t)kClCap * sizeof(unsigned long long);
-    cudaError_t e = cudaFuncSetAttribute(cadd_cluster_rowpass_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) { (void)cudaGetLastError(); return e; }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kClSegs * p.D, p.batch);
-    cfg.blockDim = dim3(kRowThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kClSegs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    TraceScope t(s, "cadd_rowpass");
-    e = cudaLaunchKernelEx(&cfg, cadd_cluster_rowpass_kernel, p,
-                           static_cast<const __nv_bfloat16*>(L), ctx, row_lse, cand_cnt, cand_q,
-                           cand_tok, status);
-    if (e != cudaSuccess) { (void)cudaGetLastError(); return e; }
+                        void* seg_ws, cudaStream_t s) {
+  const bool segmented = seg_ws != nullptr && p.dtype == PCT_BF16 && p.V % 8 == 0 &&
+                         (reinterpret_cast<uintptr_t>(L) & 15u) == 0;
+  if (segmented) {
+    const size_t rows = (size_t)p.batch * p.D, slots = rows * seg_count(p.V);
+    char* c = static_cast<char*>(seg_ws);
+    SegWs w;
+    w.lnth = reinterpret_cast<float*>(c);              c += align256(rows * sizeof(float));
+    w.part = reinterpret_cast<float2*>(c);             c += align256(slots * sizeof(float2));
+    w.cnt = reinterpret_cast<int*>(c);                 c += align256(slots * sizeof(int));
+    w.surv = reinterpret_cast<unsigned long long*>(c);
+    if (slots > 0x7fffffffu) return cudaErrorInvalidConfiguration;
+    const __nv_bfloat16* Lb = static_cast<const __nv_bfloat16*>(L);
+    {
+      TraceScope t(s, "cadd_rowpass");
+      cadd_seg_rowpass_kernel<<<(unsigned)slots, kSegThreads, 0, s>>>(p, Lb, ctx, w);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    TraceScope t(s, "cadd_finish");
+    cadd_seg_finish_kernel<<<(unsigned)rows, kSegThreads, 0, s>>>(p, Lb, ctx, w, row_lse, cand_cnt,
+                                                                 cand_q, cand_tok, status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
   } else {
     dim3 grid(p.D, p.batch);
     TraceScope t(s, "cadd_rowpass");

@@ -38,11 +38,13 @@ struct CaddParams {
   float C_d, a, b, c, e;
 };
 size_t cadd_rowpass_bytes_per_row(int n_max);
+// Workspace of the segmented row pass (bf16 rows with V % 8 == 0; else 0).
+size_t cadd_seg_workspace(int batch, int D, int V, int dtype);
 cudaError_t launch_cadd(const CaddParams& p, const void* L, const int32_t* anchor,
                         const int64_t* ctx, int32_t* tok, int32_t* parent, int32_t* depth,
                         float* score, int32_t* count, float* phi, int32_t* status,
                         float* row_lse, int32_t* cand_cnt, float* cand_q, int32_t* cand_tok,
-                        cudaStream_t s);
+                        void* seg_ws, cudaStream_t s);
 
 // ---- PCTree (pct_*.cu) ------------------------------------------------------
 // Partial results of one (row, V-slice): online log-sum-exp state and the

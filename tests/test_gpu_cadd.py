@@ -72,6 +72,27 @@ def test_stop_disabled_uses_exact_selection_fallback():
     assert (ref.count == 40).all()
 
 
+def test_many_rows_mixed_overflow():
+    """240 rows, so each cluster of the row pass walks several rows through its two
+    segment buffers; flat rows (std 0.05) overflow the survivor buffer and take the
+    exact selection, sharply peaked rows (std 2, peak +40) keep one survivor, the two
+    interleaved at random in row order."""
+    batch, D, V = 16, 15, 4096
+    L = _sharp_logits(batch, D, V, seed=21, sigma=0.05, peak=(0.0, 0.5)).float()
+    g = torch.Generator().manual_seed(22)
+    sharp = torch.rand((batch, D), generator=g) < 0.5
+    tok = torch.randint(0, V, (batch, D), generator=g)
+    for b in range(batch):
+        for d in range(D):
+            if sharp[b, d]:
+                L[b, d] *= 40.0
+                L[b, d, tok[b, d]] += 40.0
+    L = L.to(torch.bfloat16)
+    cost = dict(C_d=1.0, a=1.0, b=0.0, c=1e-6, e=0.0)
+    out, ref = _run(L, np.arange(batch), np.arange(batch) * 1000, 32, cost, label="mixed overflow")
+    assert (ref.count == 32).all()
+
+
 def test_exhausted_small_vocab():
     L = _sharp_logits(3, 2, 3, seed=3, sigma=0.5, peak=(0.0, 0.1))
     cost = dict(C_d=1.0, a=0.0, b=0.0, c=0.0, e=0.0)

@@ -93,6 +93,37 @@ def test_many_rows_mixed_overflow():
     assert (ref.count == 32).all()
 
 
+@pytest.mark.parametrize("seed", [51, 52])
+def test_multi_segment_rows(seed):
+    """V = 20488: each row splits into three segments of the row pass (854, 854 and 853
+    16-byte groups), so the survivors of every segment's own threshold are merged and
+    filtered again against the row's."""
+    batch, D, V = 8, 6, 20488
+    L = _sharp_logits(batch, D, V, seed=seed, sigma=2.0, peak=(0.0, 6.0))
+    ctx = np.array([512, 4096, 32768, 0, 100, 2000, 50000, 7])
+    out, ref = _run(L, np.arange(batch), ctx, 128, COST, label=f"segments {seed}")
+    assert ref.count.max() > 30
+
+
+def test_multi_segment_overflow():
+    """Three segments per row with flat rows whose segments overflow their slots (exact
+    selection over the row) interleaved with sharply peaked rows."""
+    batch, D, V = 6, 5, 20488
+    L = _sharp_logits(batch, D, V, seed=41, sigma=0.05, peak=(0.0, 0.5)).float()
+    g = torch.Generator().manual_seed(42)
+    sharp = torch.rand((batch, D), generator=g) < 0.5
+    tok = torch.randint(0, V, (batch, D), generator=g)
+    for b in range(batch):
+        for d in range(D):
+            if sharp[b, d]:
+                L[b, d] *= 40.0
+                L[b, d, tok[b, d]] += 40.0
+    L = L.to(torch.bfloat16)
+    cost = dict(C_d=1.0, a=1.0, b=0.0, c=1e-6, e=0.0)
+    out, ref = _run(L, np.arange(batch), np.arange(batch) * 1000, 32, cost, label="segment overflow")
+    assert (ref.count == 32).all()
+
+
 def test_exhausted_small_vocab():
     L = _sharp_logits(3, 2, 3, seed=3, sigma=0.5, peak=(0.0, 0.1))
     cost = dict(C_d=1.0, a=0.0, b=0.0, c=0.0, e=0.0)

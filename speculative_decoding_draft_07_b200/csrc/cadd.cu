@@ -7,20 +7,24 @@
 // objective is unimodal, so nodes are added until the marginal gain is
 // non-positive.
 //
-// Two kernels:
-//  * row pass, one 256-thread block per (request, depth) row of marginal
-//    logits, streamed once from HBM in 32 KB register chunks: a running
-//    log-sum-exp of the block (a lower bound of the row's) gives after every
-//    chunk a threshold with which the chunk's survivors are taken straight from
-//    registers; a final exact filter keeps only the tokens that can ever enter
-//    the tree. A node is added at size n only if its prefix
-//    probability p satisfies p > (1 + Phi) dC(n) / C(n) >= theta, where
-//    theta = min_n dC(n) / C(n) and dC(n) = C(n + 1) - C(n); since p never
-//    exceeds the marginal q_d of its last token, tokens with q_d <= theta can
-//    be dropped without changing the result. At most n_max - 1 tokens of a row
-//    can ever be used, so the survivors are sorted (value desc, token asc) and
-//    cut to n_max - 1. If more than the buffer survive (theta tiny), an exact
-//    radix select finds the n_max - 1 best instead.
+// The row pass gives every (request, depth) row of marginal logits its
+// log-sum-exp and the tokens that can ever enter the tree. A node is added at
+// size n only if its prefix probability p satisfies
+// p > (1 + Phi) dC(n) / C(n) >= theta, where theta = min_n dC(n) / C(n) and
+// dC(n) = C(n + 1) - C(n). Since p never exceeds the marginal q_d of its last
+// token, tokens with q_d <= theta can be dropped without changing the result.
+// At most n_max - 1 tokens of a row can ever be used, so the survivors are
+// sorted (value desc, token asc) and cut to n_max - 1; if too many survive
+// (theta tiny), an exact radix select finds the n_max - 1 best instead.
+//
+// Kernels:
+//  * bf16 rows (V % 8 == 0, 16-byte aligned): cadd_seg_rowpass_kernel, one
+//    block per (row, segment) with the segment in registers, filtering against
+//    the segment's own threshold, then cadd_seg_finish_kernel, one block per
+//    row, applying the row's exact threshold (details at the kernels);
+//  * other rows: cadd_rowpass_kernel, one 256-thread block per row streamed in
+//    32 KB register chunks, a running log-sum-exp of the block (a lower bound
+//    of the row's) giving after every chunk a threshold for its survivors;
 //  * best-first growth, one warp per request: a pool of candidate (next
 //    sibling, first child) entries packed into 64-bit keys (score, depth,
 //    parent insertion index, rank) so that one warp max-reduction pops the

@@ -350,6 +350,21 @@ def roofline_entry(name, kinfo, launches, total_ms, steps, pk, pk_src):
 
 
 # ---------------------------------------------------------------------------
+def rank_seed_offset(rank: int) -> int:
+    """Seed offset of a rank's inputs: every rank draws its own batch of requests
+    (weak scaling, no data-path collective)."""
+    return 100 * rank
+
+
+def max_over_ranks(x: float, dist=None, dev=None) -> float:
+    """The slowest rank's value (device times are reported as the max over ranks)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_reference(args, rank, world, budget_s: float = 120.0):
     """--impl reference: the CPU oracle on the same workload (rank 0 only).
 
@@ -507,7 +522,7 @@ def main():
     import speculative_decoding_draft_07_b200 as pct
     pct.lib()
 
-    rnd = Round(dev, seed_offset=100 * rank)
+    rnd = Round(dev, seed_offset=rank_seed_offset(rank))
     for _ in range(args.warmup):
         rnd.step()
     torch.cuda.synchronize(dev)
@@ -524,19 +539,13 @@ def main():
     clocks = sampler.stop()
     kernels = pct.trace_read()
     pct.trace_enable(False)
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, dev)
     ms_step = ms / args.steps
     value = world * 1e3 / ms_step
 
     # end-to-end through the public API with host buffers
     e2e_ms, h2d, d2h = e2e_measure(rnd, args.e2e_steps, dev)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
 
     if rank == 0:
         pk, pk_src = peaks()

@@ -28,11 +28,11 @@ Parity status of each function (what pins it, other than itself, is in
 ``tests/test_oracle_*.py``):
 
 * ``pct_tree_build``: pinned by brute-force enumeration of every path (k = V,
-  unbounded beam), by the DSpark greedy chain (k = 1, N = B), by agreement with
-  the best-first tree when the Markov term is zero, and by a hand-derived finite
-  beam example. For larger finite k and beam, where the beam boundary itself is
-  only defined by the algorithm, the result is "parity unpinned" beyond that
-  hand example and the structural invariants the tests check.
+  unbounded beam), by the pruned tree defined by predicates over every path
+  for finite k and beam (eligible = child of a kept path among its parent's k
+  best; kept = the beam best eligible paths of a depth; V <= 5, D <= 4), by the
+  DSpark greedy chain (k = 1, N = B), by agreement with the best-first tree
+  when the Markov term is zero, and by a hand-derived finite beam example.
 * ``cadd_tree_grow``: pinned by brute force (the top prefix-probability nodes
   for every n), by an exhaustive scan of the throughput objective over n, by a
   closed form on uniform marginals, and by Monte Carlo acceptance.

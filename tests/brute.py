@@ -74,3 +74,48 @@ def canonical_table(anchor, paths, scores):
     depth = [len(p) for p in order]
     score = [0.0] + [scores[p] for p in order[1:]]
     return tok, parent, depth, score
+
+
+def pruned_selection(scores, z_of, V, D, k, beam, N):
+    """PCTree with finite k and beam, from predicates over every path.
+
+    A path p of depth d is eligible when its parent p[:-1] is kept and its last
+    token is among the k best children of that parent by z (ties: lower token
+    id); kept at depth d are the `beam` best eligible paths of that depth in
+    the total order (score desc, then the smaller token path). The tree is the
+    root plus the N-1 best kept paths of all depths in the total order (score
+    desc, lower depth, smaller token path). z_of(parent_path, token) gives z.
+    Returns (selected paths, per-depth kept counts).
+    """
+    kept = {(): True}
+    all_kept, sizes = [], []
+    for d in range(1, D + 1):
+        eligible = []
+        for p in itertools.product(range(V), repeat=d):
+            par = p[:-1]
+            if par not in kept:
+                continue
+            zs = [(z_of(par, v), -v) for v in range(V)]
+            mine = zs[p[-1]]
+            better = sum(1 for t in zs if t > mine)
+            if better < k:
+                eligible.append(p)
+        eligible.sort(key=lambda p: (-scores[p], p))
+        layer = eligible[:beam]
+        for p in layer:
+            kept[p] = True
+        all_kept.extend(layer)
+        sizes.append(len(layer))
+    sel = sorted(all_kept, key=lambda p: (-scores[p], len(p), p))[: max(N - 1, 0)]
+    return sel, sizes
+
+
+def conditioned_z(L, anchor, E, W):
+    """z_of(parent_path, v) for the conditioned head: L[d-1][v] + Markov(last token)[v]."""
+    r = len(W)
+
+    def z_of(par, v):
+        d = len(par) + 1
+        u = par[-1] if par else anchor
+        return L[d - 1][v] + sum(E[u][i] * W[i][v] for i in range(r))
+    return z_of

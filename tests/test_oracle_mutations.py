@@ -25,6 +25,11 @@ MUTATIONS = [
      "test_oracle_pctree.py"),                                     # global top-N reversed
     ("pctree.py", "score_parents(L[d - 1],", "score_parents(L[d % D],",
      "test_oracle_pctree.py"),                                     # depth off by one
+    ("pctree.py", "cands.sort(key=lambda c: (-c.s, c.path))", "cands.sort(key=lambda c: (c.path,))",
+     "test_oracle_pctree.py"),                                     # beam by path, not score
+    ("pctree.py", "kept = sorted(cands[:beam], key=lambda c: c.path)",
+     "kept = sorted(cands[max(len(cands) - beam, 0):], key=lambda c: c.path)",
+     "test_oracle_pctree.py"),                                     # beam keeps the worst
     ("numerics.py", "lse = m_safe + np.log(", "lse = np.log(",
      "test_oracle_numerics.py"),                                   # dropped max shift
     ("caddtree.py", "(1.0 + phi + p) / C(n + 1) <= (1.0 + phi) / C(n)",

@@ -106,6 +106,33 @@ def test_hand_derived_finite_beam():
     assert list(r.tok[0]) == [2, 0, 1, 0] and list(r.parent[0]) == [-1, 0, 0, 1]
 
 
+@pytest.mark.parametrize("seed", range(40))
+def test_bruteforce_with_finite_k_and_beam(seed):
+    """Finite k and beam: the oracle equals the pruned tree defined by predicates over
+    every path (eligible = child of a kept path and among its parent's k best by z;
+    kept = the beam best eligible paths of the depth; tree = the N-1 best kept)."""
+    rng = np.random.default_rng(500 + seed)
+    V = int(rng.integers(2, 6))
+    D = int(rng.integers(2, 5 if V <= 3 else 4))
+    r = int(rng.integers(1, 4))
+    k = int(rng.integers(1, V + 1))
+    beam = int(rng.integers(1, min(V ** D, 3 * V) + 1))
+    N = int(rng.integers(2, 2 + D * beam + 2))
+    L, anchor, E, W = _random_problem(rng, V, D, r)
+    res = oracle.pct_tree_build(L[None], [anchor], E, W, k=k, beam=beam, n_nodes=N)
+    scores = brute.conditioned_path_scores(L.tolist(), anchor, E.tolist(), W.tolist())
+    z_of = brute.conditioned_z(L.tolist(), anchor, E.tolist(), W.tolist())
+    sel, sizes = brute.pruned_selection(scores, z_of, V, D, k, beam, N)
+    assert res.frontier_sizes[0] == sizes
+    tok, par, dep, sc = brute.canonical_table(anchor, sel, scores)
+    n = len(tok)
+    assert res.count[0] == n
+    np.testing.assert_array_equal(res.tok[0, :n], tok)
+    np.testing.assert_array_equal(res.parent[0, :n], par)
+    np.testing.assert_array_equal(res.depth[0, :n], dep)
+    np.testing.assert_allclose(res.score[0, :n], sc, atol=1e-12)
+
+
 def test_zero_markov_matches_best_first_tree():
     """W = 0 and k, beam >= N-1: PCTree's tree is the best-first prefix-probability tree."""
     rng = np.random.default_rng(7)

@@ -163,7 +163,11 @@ size_t cadd_tree_grow_workspace(const cadd_desc* desc);
  *   anchor  [batch] int32;  ctx_len [batch] int64 (context length l)
  *   tok, parent, depth [batch][n_max] int32; score [batch][n_max] float (log prefix prob)
  *   count   [batch] int32  n*;  phi [batch] float  Phi(T)
- *   dev_status [batch] int32 */
+ *   dev_status [batch] int32
+ * Fixed-budget (DDTree) trees: c = e = 0 with C_d + a + b l > 0 makes
+ * dC(n) = 0, so the stop never fires and every request grows to n_max nodes,
+ * or until its candidates run out. Since growth is best-first, Phi_n for every
+ * n is then the sum of the n - 1 largest exp(score). */
 int32_t cadd_tree_grow(const cadd_desc* desc, const void* L, const int32_t* anchor,
                        const int64_t* ctx_len, int32_t* tok, int32_t* parent, int32_t* depth,
                        float* score, int32_t* count, float* phi, int32_t* dev_status,

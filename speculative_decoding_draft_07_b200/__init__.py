@@ -9,6 +9,9 @@
 * ``tree_verify_accept`` -- greedy verification: argmax per node, accept walk,
   correction token.
 * ``pct_score_parents``  -- one depth of PCTree's batched parent scoring.
+* ``ddtree_grow`` and ``budget`` -- the fixed-budget best-first tree (CaDDTree's
+  growth with the stop disabled) and the host-side sweep of fixed budgets
+  against CaDDTree's adaptive size.
 
 All compute runs in ``libpctree.so`` (CUDA C++ behind a C ABI, declared in
 ``include/pctree.h``); this package only marshals torch tensors to it.
@@ -22,3 +25,5 @@ from ._lib import (  # noqa: F401
     cadd_tree_grow, tree_ancestor_mask, tree_verify_accept, trace_enable, trace_reset,
     trace_read, version,
 )
+from . import budget  # noqa: F401,E402
+from .budget import ddtree_grow  # noqa: F401,E402

@@ -12,6 +12,8 @@
 * ``ddtree_grow`` and ``budget`` -- the fixed-budget best-first tree (CaDDTree's
   growth with the stop disabled) and the host-side sweep of fixed budgets
   against CaDDTree's adaptive size.
+* ``tau`` -- Monte Carlo acceptance length of a round's trees against a synthetic
+  target (marginal or parent-conditioned), host side.
 
 All compute runs in ``libpctree.so`` (CUDA C++ behind a C ABI, declared in
 ``include/pctree.h``); this package only marshals torch tensors to it.
@@ -27,3 +29,4 @@ from ._lib import (  # noqa: F401
 )
 from . import budget  # noqa: F401,E402
 from .budget import ddtree_grow  # noqa: F401,E402
+from . import tau  # noqa: F401,E402

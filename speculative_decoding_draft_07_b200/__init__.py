@@ -14,6 +14,8 @@
   against CaDDTree's adaptive size.
 * ``tau`` -- Monte Carlo acceptance length of a round's trees against a synthetic
   target (marginal or parent-conditioned), host side.
+* ``costfit`` -- non-negative (convex, non-decreasing) fit of the verification
+  cost C_v(n; l) = a + b l + c n + e n^2 to latency samples, host side.
 
 All compute runs in ``libpctree.so`` (CUDA C++ behind a C ABI, declared in
 ``include/pctree.h``); this package only marshals torch tensors to it.
@@ -30,3 +32,4 @@ from ._lib import (  # noqa: F401
 from . import budget  # noqa: F401,E402
 from .budget import ddtree_grow  # noqa: F401,E402
 from . import tau  # noqa: F401,E402
+from . import costfit  # noqa: F401,E402

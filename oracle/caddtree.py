@@ -34,6 +34,14 @@ Near ties. A request is excluded when the last node added and the first
 candidate not added differ by less than ``tol`` in s (unless their per-depth
 logits are identical), or when the stop test at any step was within ``2 tol``
 of flipping (|s - log((1 + Phi) dC(n) / C(n))| < 2 tol).
+
+Near ties resolved toward a given tree. With ``prefer`` (per request, a set of
+token paths and a node count, e.g. a tree built elsewhere) growth takes, at
+each step, the best candidate in the set instead of the best candidate overall
+when their scores differ by less than ``tol``, and a stop test within ``2 tol``
+of flipping stops exactly when the tree has the given count. The result is the
+tree this algorithm grows when its near ties fall the preferred way. Without
+``prefer`` nothing changes.
 """
 from __future__ import annotations
 
@@ -64,7 +72,7 @@ class CaddResult:
     f_values: list = field(default_factory=list)      # f(1..n*) per request
 
 
-def _grow_one(L, anchor, ell, n_max, C_d, a, b, c, e, tol):
+def _grow_one(L, anchor, ell, n_max, C_d, a, b, c, e, tol, prefer=None):
     D, V = L.shape
     q, _ = row_log_softmax(L)                           # log q_d(v), [D][V]
     order = [np.argsort(-q[d], kind="stable") for d in range(D)]   # (q desc, v asc)
@@ -96,18 +104,32 @@ def _grow_one(L, anchor, ell, n_max, C_d, a, b, c, e, tol):
         if not heap:
             reason = "exhausted"
             break
-        negs, d, path, pidx, rank, vals = heap[0]
+        pick = 0
+        if prefer is not None and heap[0][2] not in prefer[0]:
+            # a preferred candidate within tol of the best takes its place
+            best = -heap[0][0]
+            near = [j for j, h in enumerate(heap) if h[2] in prefer[0] and -h[0] > best - tol]
+            if near:
+                pick = min(near, key=lambda j: heap[j][:3])
+        negs, d, path, pidx, rank, vals = heap[pick]
         s = -negs
         p = math.exp(s)
         dC = C(n + 1) - C(n)
+        flip = False
         if dC > 0:
             margin = s - math.log((1.0 + phi) * dC / C(n))
             if abs(margin) < 2 * tol:
                 excluded = True
-        if (1.0 + phi + p) / C(n + 1) <= (1.0 + phi) / C(n):
+                flip = prefer is not None
+        stop = (1.0 + phi + p) / C(n + 1) <= (1.0 + phi) / C(n)
+        if flip:
+            stop = n >= prefer[1]
+        if stop:
             reason = "gain"
             break
-        heapq.heappop(heap)
+        heap[pick] = heap[-1]
+        heap.pop()
+        heapq.heapify(heap)
         nodes.append((path[-1], d, s, path, vals))
         phi += p
         n += 1
@@ -126,11 +148,13 @@ def _grow_one(L, anchor, ell, n_max, C_d, a, b, c, e, tol):
 
 
 def cadd_tree_grow(L, anchor, ctx_len, n_max: int, C_d: float, a: float, b: float,
-                   c: float, e: float, tol: float = 1e-4) -> CaddResult:
+                   c: float, e: float, tol: float = 1e-4, prefer=None) -> CaddResult:
     """CaDDTree over a batch of independent requests.
 
     L: float64 [batch][D][V] marginal logits; anchor: int [batch]; ctx_len: the
     context length l per request. Output arrays are [batch][n_max].
+    ``prefer``: None, or per request a pair (set of token paths below the root,
+    node count) toward which near ties are resolved (module docstring).
     """
     L = np.asarray(L, dtype=np.float64)
     batch = L.shape[0]
@@ -144,7 +168,8 @@ def cadd_tree_grow(L, anchor, ctx_len, n_max: int, C_d: float, a: float, b: floa
     reasons, fv = [], []
     for r in range(batch):
         out, index, ph, ex, why, f = _grow_one(L[r], anchor[r], float(ctx_len[r]), n_max,
-                                               C_d, a, b, c, e, tol)
+                                               C_d, a, b, c, e, tol,
+                                               None if prefer is None else prefer[r])
         for i, (t, d, s, path, _) in enumerate(out):
             tok[r, i], dep[r, i], score[r, i] = t, d, s
             par[r, i] = -1 if d == 0 else index[path[:-1]]

@@ -40,6 +40,15 @@ A local top-k or beam boundary whose better score lies more than ``2 tol``
 below the global cut cannot change the output (every node it could add or drop
 scores below every selected node, and so do all its descendants) and is not
 counted.
+
+Near ties resolved toward a given tree. When two candidates differ by less
+than ``tol``, either may be kept: both orders are correct to the tolerance. With
+``prefer`` (a set of token paths, e.g. the nodes of a tree built elsewhere)
+every cut keeps its usual members except that a rejected candidate in
+``prefer`` replaces a kept one that is not in ``prefer`` when their scores
+differ by less than ``tol``. The result is the tree this algorithm builds when
+its near ties fall the preferred way; a tree equal to it is therefore a valid
+output of the algorithm. Without ``prefer`` nothing changes.
 """
 from __future__ import annotations
 
@@ -69,39 +78,61 @@ class _Node:
         self.tok, self.depth, self.s, self.path, self.vals = tok, depth, s, path, vals
 
 
-def score_parents(L_d, parent_tok, E, W, k):
+def score_parents(L_d, parent_tok, E, W, k, extra=1):
     """One depth of batched parent scoring for one request.
 
     For every parent token p: z = L_d + E[p] . W (all parents in one matrix
-    product), log pi = z - lse(z), and the k + 1 best children in the order
-    (z desc, token asc). Returns (z, markov, log_pi, lse, order) with order
-    holding the first min(k + 1, V) token ids of each row.
+    product), log pi = z - lse(z), and the k + extra best children in the
+    order (z desc, token asc). Returns (z, markov, log_pi, lse, order) with
+    order holding the first min(k + extra, V) token ids of each row.
     """
     toks = np.asarray(parent_tok, dtype=np.int64)
     markov = E[toks] @ W                                       # [|F|][V]
     Z = L_d[None, :] + markov                                  # z_d(p)
     logpi, lse = row_log_softmax(Z)
     # stable sort of -z keeps the lower token first among equal z
-    order = np.argsort(-Z, axis=1, kind="stable")[:, : min(k + 1, Z.shape[1])]
+    order = np.argsort(-Z, axis=1, kind="stable")[:, : min(k + extra, Z.shape[1])]
     return Z, markov, logpi, lse, order
 
 
-def _build_one(L, anchor, E, W, k, beam, n_nodes, tol):
+def _near_tie_keep(ranked, keep, score, preferred, tol):
+    """The first ``keep`` of ``ranked`` (best first), except that each rejected
+    item in ``preferred`` takes the place of the lowest-ranked kept item not in
+    ``preferred`` whose score is within ``tol`` of its own."""
+    kept, rest = list(ranked[:keep]), ranked[keep:]
+    if not kept or preferred is None:
+        return kept
+    floor = score(kept[-1]) - tol
+    for y in rest:
+        if score(y) <= floor:
+            break
+        if not preferred(y):
+            continue
+        for j in range(len(kept) - 1, -1, -1):
+            x = kept[j]
+            if not preferred(x) and abs(score(x) - score(y)) < tol:
+                kept[j] = y
+                break
+    return kept
+
+
+def _build_one(L, anchor, E, W, k, beam, n_nodes, tol, prefer=None):
     D, V = L.shape
     root = _Node(int(anchor), 0, 0.0, (), ())
     frontier = [root]
     levels = []
     boundaries = []            # (better score, worse score, identical inputs?)
     kk = min(k, V)
+    pref = None if prefer is None else (lambda c: c.path in prefer)
     for d in range(1, D + 1):
         # one batched Markov call for every frontier parent: E[tok(p)] . W
-        Z, markov, logpi, lse, order = score_parents(L[d - 1], [p.tok for p in frontier], E, W, k)
+        Z, markov, logpi, lse, order = score_parents(L[d - 1], [p.tok for p in frontier], E, W, k,
+                                                     extra=1 if prefer is None else 8)
         cands = []
         for i, p in enumerate(frontier):
-            for j in range(kk):
-                v = int(order[i, j])
-                cands.append(_Node(v, d, p.s + logpi[i, v], p.path + (v,),
-                                   p.vals + ((L[d - 1][v], markov[i, v], lse[i]),)))
+            row = [_Node(int(v), d, p.s + logpi[i, v], p.path + (int(v),),
+                         p.vals + ((L[d - 1][v], markov[i, v], lse[i]),)) for v in order[i]]
+            cands.extend(_near_tie_keep(row, kk, lambda c: c.s, pref, tol))
             if kk < V:
                 vi, vo = int(order[i, kk - 1]), int(order[i, kk])
                 same = (L[d - 1][vi] == L[d - 1][vo]) and (markov[i, vi] == markov[i, vo])
@@ -110,13 +141,15 @@ def _build_one(L, anchor, E, W, k, beam, n_nodes, tol):
         if len(cands) > beam:
             a, b = cands[beam - 1], cands[beam]
             boundaries.append((a.s, b.s, a.vals == b.vals))
-        kept = sorted(cands[:beam], key=lambda c: c.path)     # canonical order
+        kept = sorted(_near_tie_keep(cands, beam, lambda c: c.s, pref, tol),
+                      key=lambda c: c.path)                   # canonical order
         levels.append(kept)
         frontier = kept
 
     union = [n for lvl in levels for n in lvl]
     ranked = sorted(union, key=lambda c: (-c.s, c.depth, c.path))
-    sel = ranked[: n_nodes - 1]
+    chosen = {id(c) for c in _near_tie_keep(ranked, n_nodes - 1, lambda c: c.s, pref, tol)}
+    sel = [c for c in ranked if id(c) in chosen]
     excluded = False
     if len(ranked) > n_nodes - 1:
         s_cut = sel[-1].s if sel else np.inf
@@ -136,12 +169,14 @@ def _build_one(L, anchor, E, W, k, beam, n_nodes, tol):
 
 
 def pct_tree_build(L, anchor, E, W, k: int, beam: int, n_nodes: int,
-                   tol: float = 1e-4) -> PCTreeResult:
+                   tol: float = 1e-4, prefer=None) -> PCTreeResult:
     """PCTree over a batch of independent requests.
 
     L: float64 [batch][D][V] drafter logits (decoded); anchor: int [batch];
     E: float64 [V][r]; W: float64 [r][V]. Returns the node tables in canonical
-    BFS order with float64 scores.
+    BFS order with float64 scores. ``prefer``: None, or one set of token paths
+    per request (tuples of tokens below the root) toward which near ties are
+    resolved (module docstring).
     """
     L = np.asarray(L, dtype=np.float64)
     E = np.asarray(E, dtype=np.float64)
@@ -155,7 +190,8 @@ def pct_tree_build(L, anchor, E, W, k: int, beam: int, n_nodes: int,
     excl = np.zeros(batch, bool)
     sizes, kept = [], []
     for b in range(batch):
-        out, index, ex, fs, union = _build_one(L[b], anchor[b], E, W, k, beam, n_nodes, tol)
+        out, index, ex, fs, union = _build_one(L[b], anchor[b], E, W, k, beam, n_nodes, tol,
+                                               None if prefer is None else prefer[b])
         for i, n in enumerate(out):
             tok[b, i] = n.tok
             dep[b, i] = n.depth

@@ -19,7 +19,7 @@ MUTATIONS = [
      "test_oracle_pctree.py"),                                     # wrong parent index
     ("pctree.py", "p.s + logpi[i, v], p.path", "logpi[i, v], p.path",
      "test_oracle_pctree.py"),                                     # dropped prefix term
-    ("pctree.py", "v = int(order[i, j])", "v = int(order[i, -1 - j])",
+    ("pctree.py", "for v in order[i]]", "for v in order[i][::-1]]",
      "test_oracle_pctree.py"),                                     # top-k from the wrong end
     ("pctree.py", "key=lambda c: (-c.s, c.depth, c.path)", "key=lambda c: (c.s, c.depth, c.path)",
      "test_oracle_pctree.py"),                                     # global top-N reversed
@@ -27,8 +27,8 @@ MUTATIONS = [
      "test_oracle_pctree.py"),                                     # depth off by one
     ("pctree.py", "cands.sort(key=lambda c: (-c.s, c.path))", "cands.sort(key=lambda c: (c.path,))",
      "test_oracle_pctree.py"),                                     # beam by path, not score
-    ("pctree.py", "kept = sorted(cands[:beam], key=lambda c: c.path)",
-     "kept = sorted(cands[max(len(cands) - beam, 0):], key=lambda c: c.path)",
+    ("pctree.py", "kept = sorted(_near_tie_keep(cands, beam,",
+     "kept = sorted(_near_tie_keep(cands[::-1], beam,",
      "test_oracle_pctree.py"),                                     # beam keeps the worst
     ("numerics.py", "lse = m_safe + np.log(", "lse = np.log(",
      "test_oracle_numerics.py"),                                   # dropped max shift

@@ -28,3 +28,18 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Parity counts per configuration: requests compared bit-exactly with the
+    oracle, compared after resolving near ties toward the GPU's nodes, and
+    excluded (not matched either way)."""
+    try:
+        from gpu_util import REPORT
+    except Exception:  # pragma: no cover
+        return
+    if not REPORT:
+        return
+    terminalreporter.write_line("parity (requests: exact / near-tie resolved / excluded):")
+    for label, (n, ex, res, exc) in REPORT.items():
+        terminalreporter.write_line(f"  {label}: {n}: {ex} / {res} / {exc}")

@@ -10,7 +10,7 @@ import torch
 import oracle
 import speculative_decoding_draft_07_b200 as pct
 import workloads
-from gpu_util import PHI_RTOL, compare_trees, f64, host
+from gpu_util import compare_all, f64, host, oracle_map
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda")
@@ -26,17 +26,34 @@ def _sharp_logits(batch, D, V, seed, dtype="bf16", sigma=1.0, peak=(8.0, 16.0)):
     return L.to(torch.bfloat16 if dtype == "bf16" else torch.float32)
 
 
-def _run(L, anchor, ctx, n_max, cost, max_excluded=0.1, label=""):
+def _cadd_oracle(L, anchor, ctx, n_max, cost):
+    """Per-request oracle runs (in parallel) and the near-tie rebuild."""
+    anchor, ctx = np.asarray(anchor), np.asarray(ctx)
+
+    def grow(b, prefer=None):
+        return oracle.cadd_tree_grow(f64(L[b:b + 1]), anchor[b:b + 1], ctx[b:b + 1], n_max, **cost,
+                                     prefer=None if prefer is None else [prefer])
+    return grow
+
+
+def _run(L, anchor, ctx, n_max, cost, label="", max_unresolved=0):
+    """GPU growth of every request, each compared with the oracle (node tables
+    bit-exact, scores within 1e-4, Phi within 1e-4 relative; near ties resolved
+    toward the GPU's tree)."""
     out = pct.cadd_tree_grow(L.to(DEV), torch.as_tensor(anchor, dtype=torch.int32, device=DEV),
                              torch.as_tensor(ctx, dtype=torch.int64, device=DEV), n_max, **cost)
     torch.cuda.synchronize()
-    ref = oracle.cadd_tree_grow(f64(L), np.asarray(anchor), np.asarray(ctx), n_max, **cost)
-    n = compare_trees(out, ref, label=label)
-    assert n >= (1 - max_excluded) * len(anchor), f"{label}: {len(anchor) - n} excluded"
-    keep = ~ref.excluded
-    np.testing.assert_allclose(host(out.phi)[keep], ref.phi[keep], rtol=PHI_RTOL, atol=1e-7)
+    grow = _cadd_oracle(L, anchor, ctx, n_max, cost)
+    rows = list(range(len(anchor)))
+    refs = oracle_map(grow, rows)
+    cnt = host(out.count)
+    compare_all(out, refs, lambda j, paths: grow(j, (paths, int(cnt[j]))), rows, label,
+                max_unresolved=max_unresolved, phi=True)
     assert (host(out.status) == 0).all()
-    return out, ref
+
+    class Ref:   # the batch's oracle results, stacked (for the callers' extra checks)
+        count = np.array([r.count[0] for r in refs])
+    return out, Ref
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -143,19 +160,11 @@ def test_bad_cost_flagged():
 @pytest.mark.slow
 @pytest.mark.parametrize("ell", workloads.CADDTREE.ells)
 def test_caddtree_workload_full_size(ell):
-    """64 requests, V = 151936, D = 15, n_max = 512; the oracle checks 16 of them."""
+    """64 requests, V = 151936, D = 15, n_max = 512: every request against the oracle."""
     w = workloads.CADDTREE
     d = workloads.cadd_inputs(w, ell, device=DEV)
     cost = dict(C_d=w.C_d, a=w.a, b=w.b, c=w.c, e=w.e)
-    out = pct.cadd_tree_grow(d["L"], d["anchor"], d["ctx_len"], w.n_max, **cost)
-    torch.cuda.synchronize()
-    sample = list(range(0, w.batch, 4))
-    Ls = d["L"][sample]
-    ref = oracle.cadd_tree_grow(f64(Ls), host(d["anchor"])[sample], host(d["ctx_len"])[sample],
-                                w.n_max, **cost)
-    n = compare_trees(out, ref, rows=sample, label=f"caddtree l={ell}")
-    assert n >= len(sample) - 1
-    keep = ~ref.excluded
-    np.testing.assert_allclose(host(out.phi)[sample][keep], ref.phi[keep], rtol=PHI_RTOL)
+    out, ref = _run(d["L"].cpu(), host(d["anchor"]), host(d["ctx_len"]), w.n_max, cost,
+                    label=f"caddtree l={ell} (cfg 3)", max_unresolved=1)
     counts = host(out.count)
     assert (counts >= 2).all() and (counts <= w.n_max).all()

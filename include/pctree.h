@@ -212,6 +212,52 @@ int32_t tree_verify_accept(int32_t batch, int32_t n_stride, int32_t vocab, int32
                            void* cuda_stream);
 
 /* ------------------------------------------------------------------------ *
+ * Lazy greedy verification: the same acceptance as tree_verify_accept, with
+ * the argmax taken only where the walk goes.
+ * Source: DSpark explainer (xiaohu-jiedu), section on one round from drafting
+ * to confirmation: the drafts are compared from the head and the comparison
+ * stops at the first miss, so only the rows of the nodes the walk reaches (the
+ * root and each accepted node: at most max_depth + 1 rows per request) decide
+ * the round; no other row is read.
+ * Arguments, layouts, errors, accept_len, accept_path and correction are those
+ * of tree_verify_accept (identical results). argmax [batch][n_stride] holds the
+ * argmax of every row the walk reached and -1 in every other slot. No
+ * workspace; one launch. The rows of one request are read one after another,
+ * so the call is bound by latency rather than bandwidth.
+ * ------------------------------------------------------------------------ */
+int32_t tree_verify_walk(int32_t batch, int32_t n_stride, int32_t vocab, int32_t max_depth,
+                         const int32_t* tok, const int32_t* parent, const int32_t* count,
+                         const void* target, int32_t target_dtype, int32_t* argmax,
+                         int32_t* accept_len, int32_t* accept_path, int32_t* correction,
+                         int32_t* dev_status, void* cuda_stream);
+
+/* ------------------------------------------------------------------------ *
+ * Monte Carlo acceptance length of a batch of trees (tau = accepted + 1).
+ * Source: DSpark explainer (xiaohu-jiedu), section on one round from drafting
+ * to confirmation (checked from the head, the first miss ends the round, the
+ * target adds its own token); PCTree article (qiita), numbers table (tau,
+ * tokens accepted per round).
+ * A walk starts at the root; at node u it draws one uniform x and moves to the
+ * first child c of u, in index order, whose running sum of p_child exceeds x;
+ * it stops when none does or after max_depth moves. p_child[b][c] is the
+ * probability that the target's token at c's position equals c's token, given
+ * that the target agreed with the path to c's parent (for a target equal to
+ * the drafter: exp(score[c] - score[parent[c]])); the p_child of one node's
+ * children must sum to at most 1.
+ * Random numbers: Philox4x32-10 with counter (trial, request, step, 0) and key
+ * (seed low 32 bits, seed high 32 bits); x = (first word >> 8) * 2^-24. Sums
+ * and comparisons are fp32 in child index order (reproducible on a host).
+ *   parent, p_child [batch][n_stride]; count [batch]
+ *   hist [batch][max_depth + 1] int64: walks per accepted length (written)
+ *   dev_status [batch]: PCT_DEV_BAD_PARENT / PCT_DEV_BAD_COUNT (that request's
+ *   histogram stays zero)
+ * n_stride in 1..4096, max_depth in 1..4096, trials in 1..2^31 - 1.
+ * ------------------------------------------------------------------------ */
+int32_t tree_accept_sim(int32_t batch, int32_t n_stride, int32_t max_depth, const int32_t* parent,
+                        const int32_t* count, const float* p_child, int64_t trials, uint64_t seed,
+                        int64_t* hist, int32_t* dev_status, void* cuda_stream);
+
+/* ------------------------------------------------------------------------ *
  * Allocation-free variant of tree_verify_accept. The pages have no
  * counterpart to this call: it exists for users of the library whose code
  * cannot allocate device memory -- for example a component inside a serving
@@ -226,8 +272,10 @@ int32_t tree_verify_accept(int32_t batch, int32_t n_stride, int32_t vocab, int32
  * exits. batch > PCT_NOALLOC_MAX_BATCH returns PCT_EUNSUPPORTED before
  * anything is launched. The call allocates nothing; it clears the counters it
  * uses on its stream before the kernel runs.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - The first call in each CUDA context (per device, and again after
+ *     cudaDeviceReset or when another context is made current) looks up the
+ *     array's device address (cudaGetSymbolAddress); make that first call
+ *     before any stream capture.
  *   - All calls share the one array: two calls that can run at the same time on
  *     the GPU (for example on different streams) race on it and give undefined
  *     results. Order them on one stream or with events.

@@ -40,15 +40,21 @@ Parity status of each function (what pins it, other than itself, is in
   plus 1 correction) and by planted paths.
 * ``tree_ancestor_mask``: pinned by an independent transitive closure of the
   parent relation.
+* ``accept_sim``: Monte Carlo walks of greedy verification on a tree (the
+  acceptance length tau); pinned by the generator's published known answers,
+  by walks worked out by hand, and by the identity E[accepted] = Phi(T) when the
+  target is the drafter itself.
 """
 from .numerics import decode_bf16, to_f64, row_log_softmax
 from .pctree import pct_tree_build, PCTreeResult, score_parents
 from .caddtree import cadd_tree_grow, CaddResult, cadd_cost
 from .verify import tree_verify_accept, tree_ancestor_mask, VerifyResult
+from .accept_sim import accept_sim, philox4x32_10, uniform24
 
 __all__ = [
     "decode_bf16", "to_f64", "row_log_softmax",
     "pct_tree_build", "PCTreeResult", "score_parents",
     "cadd_tree_grow", "CaddResult", "cadd_cost",
     "tree_verify_accept", "tree_ancestor_mask", "VerifyResult",
+    "accept_sim", "philox4x32_10", "uniform24",
 ]

@@ -1,5 +1,10 @@
 """B200-native (sm_100a) per-round hot path of tree-based speculative decoding.
 
+The hot path, all of it in ``libpctree.so`` (CUDA C++ for sm_100a behind the
+C ABI declared in ``include/pctree.h``); the functions here only check shapes,
+allocate outputs and pass pointers (``_lib.py``), and raise if the library is
+missing:
+
 * ``pct_tree_build``     -- PCTree: parent-conditioned drafting tree (batched
   Markov scoring on tcgen05 tensor cores, log-softmax, local top-k, beam,
   global top-N).
@@ -8,17 +13,20 @@
 * ``tree_ancestor_mask`` -- self-plus-ancestor bitmask for tree attention.
 * ``tree_verify_accept`` -- greedy verification: argmax per node, accept walk,
   correction token.
+* ``tree_verify_walk``   -- the same acceptance reading only the rows the walk
+  reaches.
+* ``tree_accept_sim``    -- Monte Carlo acceptance length (tau) of a batch of
+  trees against a synthetic target given per node.
 * ``pct_score_parents``  -- one depth of PCTree's batched parent scoring.
-* ``ddtree_grow`` and ``budget`` -- the fixed-budget best-first tree (CaDDTree's
-  growth with the stop disabled) and the host-side sweep of fixed budgets
-  against CaDDTree's adaptive size.
-* ``tau`` -- Monte Carlo acceptance length of a round's trees against a synthetic
-  target (marginal or parent-conditioned), host side.
-* ``costfit`` -- non-negative (convex, non-decreasing) fit of the verification
-  cost C_v(n; l) = a + b l + c n + e n^2 to latency samples, host side.
+* ``budget.ddtree_grow`` -- the fixed-budget best-first tree (CaDDTree's growth
+  with the stop disabled), a call of ``cadd_tree_grow``.
 
-All compute runs in ``libpctree.so`` (CUDA C++ behind a C ABI, declared in
-``include/pctree.h``); this package only marshals torch tensors to it.
+Host-side tools around the hot path (numpy on the host, not part of it and not
+marshalling): ``budget`` (Phi curves, the greedy size and the sweep of fixed
+budgets against the adaptive size, evaluated from the library's trees),
+``tau`` (Monte Carlo acceptance length of a round's trees against a synthetic
+target) and ``costfit`` (non-negative fit of C_v(n; l) = a + b l + c n + e n^2
+to latency samples).
 """
 from ._lib import (  # noqa: F401
     BuildDesc, CaddDesc, PctError, TreeOut, VerifyOut, LIB_PATH, EXPORTED,
@@ -26,7 +34,8 @@ from ._lib import (  # noqa: F401
     PCT_F32, PCT_BF16, DEV_BAD_PARENT, DEV_BAD_TOKEN, DEV_BAD_COUNT, DEV_DEPTH_OVERFLOW,
     DEV_BAD_COST, DEV_TIMEOUT,
     lib, build_desc, cadd_desc, pct_tree_build_workspace, pct_tree_build, pct_score_parents,
-    cadd_tree_grow, tree_ancestor_mask, tree_verify_accept, trace_enable, trace_reset,
+    cadd_tree_grow, tree_ancestor_mask, tree_verify_accept, tree_verify_walk, tree_accept_sim,
+    trace_enable, trace_reset,
     trace_read, version,
 )
 from . import budget  # noqa: F401,E402

@@ -28,7 +28,8 @@ EXPORTED = [
     "pct_tree_build_workspace", "pct_tree_build", "pct_score_parents_workspace",
     "pct_score_parents", "cadd_tree_grow_workspace", "cadd_tree_grow", "tree_ancestor_mask",
     "tree_verify_accept_workspace", "tree_verify_accept", "pct_trace_enable", "pct_trace_reset",
-    "pct_trace_read", "pct_version", "tree_verify_accept_noalloc",
+    "pct_trace_read", "pct_version", "tree_verify_accept_noalloc", "tree_verify_walk",
+    "tree_accept_sim",
 ]
 
 
@@ -83,6 +84,9 @@ def lib() -> ctypes.CDLL:
         "pct_version": (ctypes.c_char_p, []),
         "tree_verify_accept_noalloc": (i32, [i32, i32, i32, i32, vp, vp, vp, vp, i32, vp, vp, vp,
                                              vp, vp, vp]),
+        "tree_verify_walk": (i32, [i32, i32, i32, i32, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]),
+        "tree_accept_sim": (i32, [i32, i32, i32, vp, vp, vp, ctypes.c_int64, ctypes.c_uint64, vp,
+                                  vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -297,6 +301,51 @@ def tree_verify_accept(tok: torch.Tensor, parent: torch.Tensor, count: torch.Ten
                                     _p(ws), wsb, _stream(stream))
     _raise(code, "tree_verify_accept")
     return out
+
+
+def tree_verify_walk(tok: torch.Tensor, parent: torch.Tensor, count: torch.Tensor,
+                     target: torch.Tensor, max_depth: int, out: Optional[VerifyOut] = None,
+                     stream=None) -> VerifyOut:
+    """Greedy verification reading only the rows the walk reaches: the same
+    accept_len, accept_path and correction as tree_verify_accept; argmax holds
+    the walked rows' argmax and -1 elsewhere."""
+    dev = tok.device
+    batch, n_stride = tok.shape
+    V = target.shape[2]
+    _check(tok, "tok", dev, dtype=torch.int32)
+    _check(parent, "parent", dev, (batch, n_stride), torch.int32)
+    _check(count, "count", dev, (batch,), torch.int32)
+    _check(target, "target", dev, (batch, n_stride, V))
+    if out is None:
+        out = VerifyOut(torch.empty((batch, n_stride), dtype=torch.int32, device=dev),
+                        torch.empty(batch, dtype=torch.int32, device=dev),
+                        torch.empty((batch, max_depth), dtype=torch.int32, device=dev),
+                        torch.empty(batch, dtype=torch.int32, device=dev),
+                        torch.empty(batch, dtype=torch.int32, device=dev))
+    code = lib().tree_verify_walk(batch, n_stride, V, max_depth, _p(tok), _p(parent), _p(count),
+                                  _p(target), _code(target), _p(out.argmax), _p(out.accept_len),
+                                  _p(out.accept_path), _p(out.correction), _p(out.status),
+                                  _stream(stream))
+    _raise(code, "tree_verify_walk")
+    return out
+
+
+def tree_accept_sim(parent: torch.Tensor, count: torch.Tensor, p_child: torch.Tensor,
+                    trials: int, seed: int, max_depth: int, stream=None):
+    """Monte Carlo walks of greedy verification: (hist [batch][max_depth + 1]
+    int64 walks per accepted length, status [batch])."""
+    dev = parent.device
+    batch, n_stride = parent.shape
+    _check(parent, "parent", dev, dtype=torch.int32)
+    _check(count, "count", dev, (batch,), torch.int32)
+    _check(p_child, "p_child", dev, (batch, n_stride), torch.float32)
+    hist = torch.empty((batch, max_depth + 1), dtype=torch.int64, device=dev)
+    status = torch.empty(batch, dtype=torch.int32, device=dev)
+    code = lib().tree_accept_sim(batch, n_stride, max_depth, _p(parent), _p(count), _p(p_child),
+                                 int(trials), int(seed) & ((1 << 64) - 1), _p(hist), _p(status),
+                                 _stream(stream))
+    _raise(code, "tree_accept_sim")
+    return hist, status
 
 
 def trace_enable(on: bool = True) -> bool:

@@ -104,7 +104,13 @@ struct PctPlan {
   int Mmax, M_pad;
   size_t max_ps;
   size_t o_eg, o_ms, o_val, o_idx, o_ltok, o_lppos, o_ls, o_err, o_thr, o_scol, o_slval, o_swmax, o_swcol, total;
+  bool chain;             // small frontiers: one persistent launch (pct_chain.cu)
+  size_t o_chain;
 };
+
+ChainShape chain_shape(const PctPlan& P) {
+  return ChainShape{P.batch, P.D, P.V, P.r, P.r_pad, P.k, P.beam, P.ldt, P.mdt};
+}
 
 int check_build_desc(const pct_build_desc* d) {
   if (!d) return PCT_EINVAL;
@@ -153,6 +159,8 @@ int make_plan(const pct_build_desc* d, PctPlan* P) {
   P->o_slval = o; o += align_up(seeds * sizeof(float));
   P->o_swmax = o; o += align_up(seeds * sizeof(float));
   P->o_swcol = o; o += P->mdt == PCT_BF16 ? align_up(seeds * P->r_pad * 2) : 0;
+  P->chain = chain_eligible(chain_shape(*P));
+  P->o_chain = o; o += P->chain ? align_up(chain_workspace(chain_shape(*P))) : 0;
   P->total = o;
   return PCT_OK;
 }
@@ -283,6 +291,21 @@ int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t*
   const size_t lvl = (size_t)P.batch * P.beam;
 
   PCT_CU(cudaMemsetAsync(dev_status, 0, sizeof(int32_t) * P.batch, s));
+  if (P.chain && aligned(E, 16) && aligned(W, 16) && aligned(L, 16)) {
+    // every depth in one persistent launch, then the global top-N
+    int32_t* cerr = nullptr;
+    PCT_CU(launch_chain(chain_shape(P), L, anchor, E, W, ws + P.o_chain, ltok, lppos, ls, &cerr,
+                        dev_status, s));
+    FinalArgs f;
+    f.batch = P.batch; f.D = P.D; f.beam = P.beam; f.N = P.N;
+    for (int d = 0; d <= P.D; ++d) f.F[d] = P.F[d];
+    f.anchor = anchor; f.lvl_tok = ltok; f.lvl_ppos = lppos; f.lvl_s = ls;
+    f.tok = tok; f.parent = parent; f.depth = depth; f.count = count; f.score = score;
+    f.status = dev_status;
+    f.err = cerr;
+    PCT_CU(launch_final(f, s));
+    return PCT_OK;
+  }
   PCT_CU(cudaMemsetAsync(err, 0, sizeof(int32_t), s));
   // tensor-core scoring: every row's top-k gate starts from a seed (k exact
   // values of the row at the request's best drafter columns of that depth)
@@ -343,6 +366,7 @@ int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t*
   f.anchor = anchor; f.lvl_tok = ltok; f.lvl_ppos = lppos; f.lvl_s = ls;
   f.tok = tok; f.parent = parent; f.depth = depth; f.count = count; f.score = score;
   f.status = dev_status;
+  f.err = err;
   PCT_CU(launch_final(f, s));
   return PCT_OK;
 }
@@ -492,6 +516,41 @@ int32_t tree_verify_accept(int32_t batch, int32_t n_stride, int32_t vocab, int32
   PCT_CU(cudaMemsetAsync(arrive, 0, sizeof(unsigned) * batch, s));
   PCT_CU(launch_verify(batch, n_stride, vocab, max_depth, tok, parent, count, target, target_dtype,
                        argmax, accept_len, accept_path, correction, dev_status, arrive, s));
+  return PCT_OK;
+}
+
+int32_t tree_verify_walk(int32_t batch, int32_t n_stride, int32_t vocab, int32_t max_depth,
+                         const int32_t* tok, const int32_t* parent, const int32_t* count,
+                         const void* target, int32_t target_dtype, int32_t* argmax,
+                         int32_t* accept_len, int32_t* accept_path, int32_t* correction,
+                         int32_t* dev_status, void* cuda_stream) {
+  if (batch < 1 || batch > 65535 || n_stride < 1 || n_stride > 4096) return PCT_EINVAL;
+  if (vocab < 1 || max_depth < 1 || max_depth > 4096 || !dtype_ok(target_dtype)) return PCT_EINVAL;
+  if (!tok || !parent || !count || !target || !argmax || !accept_len || !accept_path ||
+      !correction || !dev_status)
+    return PCT_EINVAL;
+  if (!device_ok()) return PCT_EDEVICE;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  PCT_CU(cudaMemsetAsync(dev_status, 0, sizeof(int32_t) * batch, s));
+  PCT_CU(launch_verify_walk(batch, n_stride, vocab, max_depth, tok, parent, count, target,
+                            target_dtype, argmax, accept_len, accept_path, correction, dev_status,
+                            s));
+  return PCT_OK;
+}
+
+int32_t tree_accept_sim(int32_t batch, int32_t n_stride, int32_t max_depth, const int32_t* parent,
+                        const int32_t* count, const float* p_child, int64_t trials, uint64_t seed,
+                        int64_t* hist, int32_t* dev_status, void* cuda_stream) {
+  if (batch < 1 || batch > 65535 || n_stride < 1 || n_stride > 4096) return PCT_EINVAL;
+  if (max_depth < 1 || max_depth > 4096 || trials < 1 || trials > 2147483647LL) return PCT_EINVAL;
+  if (!parent || !count || !p_child || !hist || !dev_status) return PCT_EINVAL;
+  if (!device_ok()) return PCT_EDEVICE;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  PCT_CU(cudaMemsetAsync(dev_status, 0, sizeof(int32_t) * batch, s));
+  PCT_CU(cudaMemsetAsync(hist, 0, sizeof(int64_t) * (size_t)batch * (max_depth + 1), s));
+  PCT_CU(launch_accept_sim(batch, n_stride, max_depth, parent, count, p_child, (long long)trials,
+                           (unsigned long long)seed, reinterpret_cast<unsigned long long*>(hist),
+                           dev_status, s));
   return PCT_OK;
 }
 

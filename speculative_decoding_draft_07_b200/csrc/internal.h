@@ -32,6 +32,19 @@ cudaError_t launch_verify(int batch, int n_stride, int vocab, int max_depth, con
                           int dtype, int32_t* argmax, int32_t* alen, int32_t* apath,
                           int32_t* corr, int32_t* status, unsigned* arrive, cudaStream_t s);
 
+// Lazy walk: argmax only of the rows the walk reaches (no workspace).
+cudaError_t launch_verify_walk(int batch, int n_stride, int vocab, int max_depth,
+                               const int32_t* tok, const int32_t* parent, const int32_t* count,
+                               const void* target, int dtype, int32_t* argmax, int32_t* alen,
+                               int32_t* apath, int32_t* corr, int32_t* status, cudaStream_t s);
+
+// ---- accept_sim.cu ----------------------------------------------------------
+size_t accept_sim_smem(int n_stride, int max_depth);
+cudaError_t launch_accept_sim(int batch, int n_stride, int max_depth, const int32_t* parent,
+                              const int32_t* count, const float* p_child, long long trials,
+                              unsigned long long seed, unsigned long long* hist, int32_t* status,
+                              cudaStream_t s);
+
 // ---- cadd.cu ----------------------------------------------------------------
 struct CaddParams {
   int batch, D, V, n_max, dtype;
@@ -119,6 +132,18 @@ struct MergeArgs {
 };
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s);
 
+// PCTree in one persistent launch for small frontiers (pct_chain.cu): bf16
+// logits and Markov parameters, at most 16 requests and 128 parent rows per
+// depth, beam <= 32. The level arrays are those launch_final reads.
+struct ChainShape {
+  int batch, D, V, r, r_pad, k, beam, logits_dtype, markov_dtype;
+};
+bool chain_eligible(const ChainShape& c);           // shape and current device
+size_t chain_workspace(const ChainShape& c);
+cudaError_t launch_chain(const ChainShape& c, const void* L, const int32_t* anchor, const void* E,
+                         const void* W, void* ws, int32_t* lvl_tok, int32_t* lvl_ppos, float* lvl_s,
+                         int32_t** err_out, int32_t* status, cudaStream_t s);
+
 struct FinalArgs {
   int batch, D, beam, N;
   int F[65];                 // F[d] for d = 1..D
@@ -129,6 +154,7 @@ struct FinalArgs {
   int32_t *tok, *parent, *depth, *count;
   float* score;
   int32_t* status;
+  const int32_t* err;        // optional: nonzero -> PCT_DEV_TIMEOUT for every request
 };
 cudaError_t launch_final(const FinalArgs& a, cudaStream_t s);
 

@@ -27,6 +27,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "seed.cuh"
+#include "select.cuh"
 
 namespace pct {
 namespace {
@@ -118,33 +119,6 @@ __device__ __forceinline__ float merge_row(const Partials& part, size_t row, int
   return lse;
 }
 
-// 64-bit keys, one per lane: bitonic sort of the warp's 32 keys, descending.
-__device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long x, int lane) {
-#pragma unroll
-  for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, stride);
-      const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0 || size == 32);
-      x = keep_max ? (x > y ? x : y) : (x < y ? x : y);
-    }
-  }
-  return x;
-}
-// a, b sorted descending across the warp (one key per lane): the 32 largest of
-// their union, sorted descending (elementwise max against b reversed is a
-// bitonic sequence holding them; one bitonic merge sorts it).
-__device__ __forceinline__ unsigned long long warp_merge_top(unsigned long long a,
-                                                             unsigned long long b_rev, int lane) {
-  unsigned long long x = a > b_rev ? a : b_rev;
-#pragma unroll
-  for (int stride = 16; stride > 0; stride >>= 1) {
-    const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, stride);
-    x = ((lane & stride) == 0) ? (x > y ? x : y) : (x < y ? x : y);
-  }
-  return x;
-}
-
 constexpr int kMergeThreads = 512;
 constexpr int kMaxCand = 1024;
 
@@ -162,13 +136,6 @@ __device__ void bitonic_desc_block(unsigned long long* keys, int P) {
       __syncthreads();
     }
   }
-}
-
-// Candidate key: larger = better under (score desc, parent position asc,
-// token asc); tokens < 2^22, parent positions < 1024.
-__device__ __forceinline__ unsigned long long cand_key(float s, int ppos, int tok) {
-  return ((unsigned long long)f2ord(s) << 32) | ((unsigned long long)(1023 - ppos) << 22) |
-         (unsigned long long)(0x3fffff - tok);
 }
 
 template <int KMAX, typename TE>
@@ -208,7 +175,7 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
       if (i < F) {
         const float sp = a.prev_s ? a.prev_s[(size_t)b * a.prev_stride + i] : 0.f;
         for (int j = gl; j < k; j += 16)
-          keys[i * k + j] = cand_key(sp + (wv[warp][16 * h + j] - lse), i, wi[warp][16 * h + j]);
+          keys[i * k + j] = beam_key(sp + (wv[warp][16 * h + j] - lse), i, wi[warp][16 * h + j]);
       }
       __syncwarp();
     }
@@ -218,7 +185,7 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
       const float lse = merge_row<KMAX, 32>(a.part, row, a.S, k, wv[warp], wi[warp]);
       __syncwarp();
       const float sp = a.prev_s ? a.prev_s[(size_t)b * a.prev_stride + i] : 0.f;
-      for (int j = lane; j < k; j += 32) keys[i * k + j] = cand_key(sp + (wv[warp][j] - lse), i, wi[warp][j]);
+      for (int j = lane; j < k; j += 32) keys[i * k + j] = beam_key(sp + (wv[warp][j] - lse), i, wi[warp][j]);
       __syncwarp();
     }
   }
@@ -427,6 +394,7 @@ __global__ __launch_bounds__(kFinalThreads) void final_kernel(FinalArgs a) {
     a.count[b] = cnt;
   }
   if (bad) atomicOr(&a.status[b], PCT_DEV_BAD_PARENT);
+  if (threadIdx.x == 0 && a.err && *a.err) atomicOr(&a.status[b], PCT_DEV_TIMEOUT);
 }
 
 template <int KMAX>

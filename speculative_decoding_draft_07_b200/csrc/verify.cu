@@ -15,6 +15,8 @@
 // instructions per 16 bytes. The block that finishes last for a request
 // (arrival counter) performs that request's accept walk, so no second launch
 // and no grid-wide wait is needed.
+#include <cuda.h>
+
 #include <climits>
 #include <mutex>
 
@@ -306,6 +308,233 @@ cudaError_t launch_verify(int batch, int n_stride, int vocab, int max_depth, con
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Lazy verification walk (the same acceptance, argmax only along the walk).
+//
+// DSpark explainer, one round from drafting to confirmation: the drafts are
+// checked from the head and checking stops at the first miss, so the only
+// target rows whose argmax decides the round are the rows of the nodes the walk
+// reaches: the root and each accepted node, at most max_depth + 1 rows.
+//
+// One cluster of kWalkCluster CTAs per request. Each CTA owns a fixed eighth of
+// the vocabulary; per step it scans its part of the current node's row, the
+// eight partial (max, first index) pairs are merged through distributed shared
+// memory after one cluster barrier, and every CTA finds the same next node in
+// its shared-memory copy of the tree. The partial slots alternate between two
+// buffers, so one barrier per step keeps a slot from being rewritten before
+// every CTA has read it. Cluster barriers are hardware barriers: no CTA waits on
+// a flag.
+namespace {
+
+constexpr int kWalkCluster = 8;
+constexpr int kWalkThreads = 256;
+
+__device__ __forceinline__ uint32_t walk_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void walk_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// A value and an index from the same shared-memory object of CTA `rank` of the cluster.
+__device__ __forceinline__ void walk_remote_pair(const float* v, const int* i, uint32_t rank,
+                                                 float& rv, int& ri) {
+  uint32_t av, ai;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(av) : "r"((uint32_t)__cvta_generic_to_shared(v)), "r"(rank));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(ai) : "r"((uint32_t)__cvta_generic_to_shared(i)), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(rv) : "r"(av) : "memory");
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(ri) : "r"(ai) : "memory");
+}
+
+// Argmax (value desc, index asc) of row[lo, hi) by this thread: MODE 0 bf16 in
+// 8-value groups (lo, hi multiples of 8, row 16-byte aligned), 2 fp32 in
+// 4-value groups (same for 4), 1 / 3 element by element.
+template <int MODE>
+__device__ __forceinline__ void walk_scan(const void* rowp, int lo, int hi, float& best, int& bidx) {
+  const int tid = threadIdx.x;
+  if (MODE == 0) {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(rowp));
+    const int g0 = lo >> 3, g1 = hi >> 3;
+    for (int base = g0 + tid; base < g1; base += kWalkThreads * kUnroll) {
+      uint4 q[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int c = base + u * kWalkThreads;
+        q[u] = c < g1 ? ld_stream16(p + c) : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const float cm = max8_bf16(q[u]);
+        if (cm > best) {
+          best = cm;
+          bidx = (base + u * kWalkThreads) * 8 + first_eq8(q[u], cm);
+        }
+      }
+    }
+  } else if (MODE == 2) {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(rowp));
+    const int g0 = lo >> 2, g1 = hi >> 2;
+    for (int base = g0 + tid; base < g1; base += kWalkThreads * kUnroll) {
+      float4 q[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int c = base + u * kWalkThreads;
+        if (c < g1) {
+          const uint4 t = ld_stream16(p + c);
+          q[u] = make_float4(__uint_as_float(t.x), __uint_as_float(t.y), __uint_as_float(t.z),
+                             __uint_as_float(t.w));
+        } else {
+          q[u] = make_float4(neg_inf(), neg_inf(), neg_inf(), neg_inf());
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int v0 = (base + u * kWalkThreads) * 4;
+        if (q[u].x > best) { best = q[u].x; bidx = v0; }
+        if (q[u].y > best) { best = q[u].y; bidx = v0 + 1; }
+        if (q[u].z > best) { best = q[u].z; bidx = v0 + 2; }
+        if (q[u].w > best) { best = q[u].w; bidx = v0 + 3; }
+      }
+    }
+  } else {
+    for (int v = lo + tid; v < hi; v += kWalkThreads) {
+      const float x = MODE == 1 ? load_f(static_cast<const __nv_bfloat16*>(rowp) + v)
+                                : load_f(static_cast<const float*>(rowp) + v);
+      if (x > best) { best = x; bidx = v; }
+    }
+  }
+}
+
+template <int MODE>
+__global__ __launch_bounds__(kWalkThreads) void verify_walk_kernel(
+    int n_stride, int V, int max_depth, const int32_t* __restrict__ tok,
+    const int32_t* __restrict__ parent, const int32_t* __restrict__ count,
+    const void* __restrict__ target, int32_t* __restrict__ argmax, int32_t* __restrict__ alen,
+    int32_t* __restrict__ apath, int32_t* __restrict__ corr, int32_t* __restrict__ status) {
+  extern __shared__ int32_t walk_tree[];          // [n_stride] tokens, then [n_stride] parents
+  __shared__ float part_v[2];
+  __shared__ int part_i[2];
+  __shared__ float sv[32];
+  __shared__ int si[32];
+  __shared__ int s_am;
+  const uint32_t rank = walk_ctarank();
+  const int b = blockIdx.x / kWalkCluster;
+  const int raw_cnt = count[b];
+  const int cnt = min(max(raw_cnt, 0), n_stride);
+  int32_t* stok = walk_tree;
+  int32_t* spar = walk_tree + n_stride;
+  const int32_t* tk = tok + (size_t)b * n_stride;
+  const int32_t* pr = parent + (size_t)b * n_stride;
+  int bad = 0;
+  for (int c = threadIdx.x; c < cnt; c += blockDim.x) {
+    const int t = tk[c], p = pr[c];
+    stok[c] = t;
+    spar[c] = p;
+    if (c == 0 ? (p != -1) : (p < 0 || p >= c)) bad |= PCT_DEV_BAD_PARENT;
+    if (t < 0 || t >= V) bad |= PCT_DEV_BAD_TOKEN;
+  }
+  if (rank == 0) {
+    if (threadIdx.x == 0 && (raw_cnt < 1 || raw_cnt > n_stride)) bad |= PCT_DEV_BAD_COUNT;
+    if (bad) atomicOr(&status[b], bad);
+    for (int c = threadIdx.x; c < n_stride; c += blockDim.x) argmax[(size_t)b * n_stride + c] = -1;
+  }
+  // this CTA's part of every row, in whole 16-byte groups where the mode uses them
+  const int unit = MODE == 0 ? 8 : (MODE == 2 ? 4 : 1);
+  const int units = V / unit;
+  const int lo = (int)((long long)units * rank / kWalkCluster) * unit;
+  const int hi = (int)((long long)units * (rank + 1) / kWalkCluster) * unit;
+  const size_t esz = (MODE == 0 || MODE == 1) ? 2 : 4;
+  const char* tb = static_cast<const char*>(target) + (size_t)b * n_stride * V * esz;
+  __syncthreads();
+
+  int u = 0, len = 0;
+  bool go = cnt > 0;
+  for (int step = 0; go; ++step) {
+    const int par = step & 1;
+    float best = neg_inf();
+    int bidx = INT_MAX;
+    walk_scan<MODE>(tb + (size_t)u * V * esz, lo, hi, best, bidx);
+    block_best(best, bidx, sv, si);
+    if (threadIdx.x == 0) { part_v[par] = best; part_i[par] = bidx; }
+    walk_cluster_sync();
+    if (threadIdx.x < 32) {
+      float v = neg_inf();
+      int i = INT_MAX;
+      if (threadIdx.x < kWalkCluster) walk_remote_pair(&part_v[par], &part_i[par], threadIdx.x, v, i);
+      warp_best(v, i);
+      // a row that is entirely -inf: every position is a maximum, the first wins
+      if (threadIdx.x == 0) s_am = (v == neg_inf()) ? 0 : i;
+    }
+    __syncthreads();
+    const int am = s_am;
+    if (rank == 0 && threadIdx.x == 0) argmax[(size_t)b * n_stride + u] = am;
+    int nxt = INT_MAX;
+    for (int c = 1 + threadIdx.x; c < cnt; c += blockDim.x)
+      if (spar[c] == u && stok[c] == am) nxt = min(nxt, c);
+    nxt = block_min(nxt, si);
+    if (nxt == INT_MAX) {
+      go = false;
+      if (rank == 0 && threadIdx.x == 0) corr[b] = am;
+    } else if (len == max_depth) {
+      go = false;
+      if (rank == 0 && threadIdx.x == 0) {
+        atomicOr(&status[b], PCT_DEV_DEPTH_OVERFLOW);
+        corr[b] = am;
+      }
+    } else {
+      if (rank == 0 && threadIdx.x == 0) apath[(size_t)b * max_depth + len] = nxt;
+      ++len;
+      u = nxt;
+    }
+  }
+  if (rank == 0) {
+    for (int j = len + threadIdx.x; j < max_depth; j += blockDim.x) apath[(size_t)b * max_depth + j] = -1;
+    if (threadIdx.x == 0) {
+      alen[b] = len;
+      if (cnt == 0) corr[b] = -1;
+    }
+  }
+  walk_cluster_sync();   // no CTA leaves while another may still read its partial slots
+}
+
+}  // namespace
+
+cudaError_t launch_verify_walk(int batch, int n_stride, int vocab, int max_depth,
+                               const int32_t* tok, const int32_t* parent, const int32_t* count,
+                               const void* target, int dtype, int32_t* argmax, int32_t* alen,
+                               int32_t* apath, int32_t* corr, int32_t* status, cudaStream_t s) {
+  const bool aligned16 = (reinterpret_cast<uintptr_t>(target) & 15u) == 0;
+  int mode;
+  if (dtype == PCT_BF16) mode = (aligned16 && vocab % 8 == 0) ? 0 : 1;
+  else mode = (aligned16 && vocab % 4 == 0) ? 2 : 3;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(batch * kWalkCluster);
+  cfg.blockDim = dim3(kWalkThreads);
+  cfg.dynamicSmemBytes = 2 * sizeof(int32_t) * (size_t)n_stride;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kWalkCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  TraceScope t(s, "verify_walk");
+  cudaError_t e;
+  switch (mode) {
+    case 0: e = cudaLaunchKernelEx(&cfg, verify_walk_kernel<0>, n_stride, vocab, max_depth, tok, parent, count, target, argmax, alen, apath, corr, status); break;
+    case 1: e = cudaLaunchKernelEx(&cfg, verify_walk_kernel<1>, n_stride, vocab, max_depth, tok, parent, count, target, argmax, alen, apath, corr, status); break;
+    case 2: e = cudaLaunchKernelEx(&cfg, verify_walk_kernel<2>, n_stride, vocab, max_depth, tok, parent, count, target, argmax, alen, apath, corr, status); break;
+    default: e = cudaLaunchKernelEx(&cfg, verify_walk_kernel<3>, n_stride, vocab, max_depth, tok, parent, count, target, argmax, alen, apath, corr, status); break;
+  }
+  if (e != cudaSuccess) (void)cudaGetLastError();
+  return e;
+}
+
 }  // namespace pct
 
 // ---------------------------------------------------------------------------
@@ -322,21 +551,48 @@ namespace {
 __device__ __align__(256) unsigned g_noalloc_arrive[PCT_NOALLOC_MAX_BATCH];
 
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[64] = {};
+struct NoallocSlot {
+  CUcontext ctx;   // context the address belongs to
+  void* ptr;
+};
+NoallocSlot g_noalloc_slot[64] = {};
 
-// Device address of the counters on the current device, looked up once per
-// device (host code may not use the array's name as a device pointer).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  }
+  return fn;
+}
+
+// Device address of the counters in the current context. Host code may not use
+// the array's name as a device pointer, so the address is looked up with
+// cudaGetSymbolAddress the first time a context calls in, and kept per device
+// together with that context: a different context on the same device (after
+// cudaDeviceReset, or one the caller made current) is looked up again.
 int noalloc_counters(unsigned** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PCT_ECUDA;
   if (dev < 0 || dev >= 64) return PCT_EUNSUPPORTED;
+  CtxGetCurrentFn cur = ctx_get_current();
+  if (!cur) return PCT_ECUDA;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
+  CUcontext ctx = nullptr;
+  if (cur(&ctx) != CUDA_SUCCESS) return PCT_ECUDA;
+  NoallocSlot& slot = g_noalloc_slot[dev];
+  if (ctx == nullptr || slot.ptr == nullptr || slot.ctx != ctx) {
+    void* p = nullptr;   // the lookup makes the device's context current if none was
     if (cudaGetSymbolAddress(&p, g_noalloc_arrive) != cudaSuccess || p == nullptr) return PCT_ECUDA;
-    g_noalloc_ptr[dev] = p;
+    if (cur(&ctx) != CUDA_SUCCESS || ctx == nullptr) return PCT_ECUDA;
+    slot.ctx = ctx;
+    slot.ptr = p;
   }
-  *out = static_cast<unsigned*>(g_noalloc_ptr[dev]);
+  *out = static_cast<unsigned*>(slot.ptr);
   return PCT_OK;
 }
 

@@ -129,3 +129,27 @@ def mean_tau(tree, V: int, draws: int, rng: np.random.Generator,
                                   conditioned_logits=lambda d, u, b=b: conditioned_logits(b, d, u))
         out[b] = acc.mean() + 1.0
     return out
+
+
+def drafter_child_probs(tree):
+    """p(child) for a target equal to the drafter: exp(s(child) - s(parent)),
+    0 at the root and past count (torch tensors on the tree's device). This is
+    the input of the library's device simulation (``tree_accept_sim``)."""
+    import torch
+    par = tree.parent.to(torch.int64).clamp(min=0)
+    p = torch.exp(tree.score - tree.score.gather(1, par))
+    return torch.where(tree.parent >= 0, p, torch.zeros_like(p)).contiguous()
+
+
+def mean_tau_device(tree, trials: int, seed: int, max_depth: int, p_child=None):
+    """Mean tau (accepted drafts + 1) per request, walked on the GPU by
+    ``tree_accept_sim`` (the drafter as the target unless p_child is given).
+    Returns (mean tau [batch], histogram [batch][max_depth + 1]) as numpy."""
+    from ._lib import tree_accept_sim
+    p = drafter_child_probs(tree) if p_child is None else p_child
+    hist, status = tree_accept_sim(tree.parent, tree.count, p, trials, seed, max_depth)
+    h = hist.cpu().numpy().astype(np.float64)
+    if (status.cpu().numpy() != 0).any():
+        raise ValueError("tree_accept_sim flagged a malformed tree")
+    lens = np.arange(h.shape[1])
+    return (h * lens).sum(1) / np.maximum(h.sum(1), 1) + 1.0, h

@@ -218,3 +218,71 @@ def test_long_block_workload_every_request():
     L, a, E, W = (d[x].cpu() for x in ("L", "anchor", "E", "W"))
     _build_and_compare(L, a, E, W, w.k, w.beam, w.n_nodes, label="long block (cfg 2)",
                        max_unresolved=1)
+
+
+# ---------------------------------------------------------------------------
+# The persistent small-frontier path (one launch for all depths: at most 16
+# requests, 128 parent rows per depth, beam <= 32, bf16 logits and Markov
+# parameters) and the multi-launch path on the same small problems.
+def _kernels_of(fn):
+    pct.trace_enable(True)
+    pct.trace_reset()
+    out = fn()
+    torch.cuda.synchronize()
+    names = set(pct.trace_read())
+    pct.trace_enable(False)
+    return out, names
+
+
+@pytest.mark.parametrize("V,D,r,k,beam,N,batch", [
+    (3000, 4, 64, 4, 8, 32, 4),      # 4 -> 32 rows: four copies per lane quarter; 24 CTAs
+    (8192, 5, 96, 8, 24, 60, 2),     # up to 48 rows: two copies; r = 96 (zero K past r)
+    (4096, 4, 256, 8, 32, 80, 4),    # 128 rows: one copy; full K
+    (2048, 6, 128, 16, 32, 100, 1),  # k = 16
+    (1024, 6, 64, 1, 4, 7, 5),       # k = 1: chains
+    (20488, 3, 256, 8, 8, 20, 16),   # 16 requests: every request row of the folded L_d
+])
+def test_persistent_path_matches_oracle(V, D, r, k, beam, N, batch):
+    L, anchor, E, W = _problem(batch, D, V, r, seed=V + 3 * D + k)
+    out, names = _kernels_of(lambda: pct.pct_tree_build(L.to(DEV), anchor.to(DEV), E.to(DEV),
+                                                        W.to(DEV), k, beam, N))
+    assert "pct_chain" in names and "pct_score_umma" not in names, names
+    _build_and_compare(L, anchor, E, W, k, beam, N, label=f"persistent V={V} k={k} b={batch}")
+
+
+def test_persistent_path_qwen3_scale_is_used():
+    w = workloads.WORKLOADS["qwen3_4b_scale"]
+    d = workloads.drafter_inputs(w, device=DEV)
+    _, names = _kernels_of(lambda: pct.pct_tree_build(d["L"], d["anchor"], d["E"], d["W"], w.k,
+                                                      w.beam, w.n_nodes))
+    assert "pct_chain" in names, names
+
+
+@pytest.mark.parametrize("V,D,r,k,beam,N", [(3000, 4, 64, 4, 8, 32), (4096, 5, 128, 8, 16, 64)])
+def test_multi_launch_path_on_small_problems(V, D, r, k, beam, N):
+    """17 requests are past the persistent path's 16: the per-depth launches run."""
+    L, anchor, E, W = _problem(17, D, V, r, seed=V + D + 77)
+    out, names = _kernels_of(lambda: pct.pct_tree_build(L.to(DEV), anchor.to(DEV), E.to(DEV),
+                                                        W.to(DEV), k, beam, N))
+    assert "pct_chain" not in names and "pct_merge_beam" in names, names
+    _build_and_compare(L, anchor, E, W, k, beam, N, label=f"multi-launch V={V}")
+
+
+def test_persistent_path_flags_bad_anchor():
+    L, anchor, E, W = _problem(3, 3, 2048, 64, seed=5)
+    anchor[1] = 2048                  # outside the vocabulary
+    out = pct.pct_tree_build(L.to(DEV), anchor.to(DEV), E.to(DEV), W.to(DEV), 4, 8, 20)
+    torch.cuda.synchronize()
+    st = host(out.status)
+    assert st[1] & pct.DEV_BAD_TOKEN and st[0] == 0 and st[2] == 0
+
+
+def test_persistent_path_repeated_builds_are_bit_identical():
+    L, anchor, E, W = _problem(2, 6, 4096, 128, seed=31)
+    Ld, ad, Ed, Wd = L.to(DEV), anchor.to(DEV), E.to(DEV), W.to(DEV)
+    first = pct.pct_tree_build(Ld, ad, Ed, Wd, 8, 16, 64)
+    ref = [host(x).copy() for x in (first.tok, first.parent, first.score, first.count)]
+    for _ in range(20):
+        o = pct.pct_tree_build(Ld, ad, Ed, Wd, 8, 16, 64)
+        for x, y in zip(ref, (o.tok, o.parent, o.score, o.count)):
+            np.testing.assert_array_equal(x, host(y))

@@ -88,6 +88,20 @@ def frontier_sizes():
 PAIR_ROWS_MIN = 129
 
 
+def merge_bytes_per_step():
+    """Algorithmic bytes of the per-depth beam merge over the round: per request
+    and depth, the |F|k candidates (token, score: 8 B) read, the beam's
+    (token, parent, score: 12 B) written, and the next depth's Markov operand
+    rows (beam x r bf16) gathered and written."""
+    F = frontier_sizes()
+    tot = 0.0
+    for d in range(1, W.depth + 1):
+        c = F[d - 1] * W.k
+        kept = F[d]
+        tot += W.batch * (8.0 * c + 12.0 * kept + (4.0 * kept * W.rank if d < W.depth else 0.0))
+    return tot
+
+
 def algorithmic_work():
     F = frontier_sizes()
     rows = [W.batch * F[d - 1] for d in range(1, W.depth + 1)]
@@ -100,6 +114,10 @@ def algorithmic_work():
         "verify_argmax_walk": {"bound": "hbm", "bytes": float(W.batch * W.n_nodes * W.vocab * 2)},
         # every marginal row read once (bf16)
         "cadd_rowpass": {"bound": "hbm", "bytes": float(W.batch * W.depth * W.vocab * 2)},
+        # admission seeds: every drafter logit row read once (bf16)
+        "drafter_topk": {"bound": "hbm", "bytes": float(W.batch * W.depth * W.vocab * 2)},
+        # per-depth beam merge: a few KB per request and depth, bound by latency
+        "pct_merge_beam": {"bound": "latency", "bytes": merge_bytes_per_step()},
     }
 
 
@@ -109,8 +127,8 @@ def source_sha(fname):
 
 
 KERNEL_SOURCE = {"pct_score_pair": "pct_umma2.cu", "pct_score_umma": "pct_umma.cu",
-                 "verify_argmax_walk": "verify.cu",
-                 "cadd_rowpass": "cadd.cu"}
+                 "verify_argmax_walk": "verify.cu", "cadd_rowpass": "cadd.cu",
+                 "drafter_topk": "pct_seed.cu", "pct_merge_beam": "pct_merge.cu"}
 
 
 def ncu_traffic(kernel):
@@ -223,6 +241,8 @@ class Round(RoundInputs):
         self.mask, self.mstat = pct.tree_ancestor_mask(self.tree.parent, self.tree.count)
         self.ver = pct.tree_verify_accept(self.tree.tok, self.tree.parent, self.tree.count, self.T,
                                           max_depth=W.depth)
+        self.walk = pct.tree_verify_walk(self.tree.tok, self.tree.parent, self.tree.count, self.T,
+                                         max_depth=W.depth)
         # preallocated workspaces so the timed region allocates nothing
         desc = pct.build_desc(W.batch, W.depth, W.vocab, W.rank, W.k, W.beam, W.n_nodes,
                               pct.PCT_BF16, pct.PCT_BF16)
@@ -234,6 +254,18 @@ class Round(RoundInputs):
         self.ws_ver = torch.empty(int(pct.lib().tree_verify_accept_workspace(W.batch, W.n_nodes)),
                                   dtype=torch.uint8, device=dev)
         torch.cuda.synchronize(dev)
+
+    def step_lazy(self):
+        """The same round with the lazy verification walk in place of the full
+        argmax (identical acceptance; only the walked rows are read)."""
+        pct = self.pct
+        pct.pct_tree_build(self.L, self.anchor, self.E, self.W, W.k, W.beam, W.n_nodes,
+                           out=self.tree, workspace=self.ws_tree)
+        pct.cadd_tree_grow(self.L, self.anchor, self.ctx, C.n_max, **COST, out=self.cadd,
+                           workspace=self.ws_cadd)
+        pct.tree_ancestor_mask(self.tree.parent, self.tree.count, mask=self.mask, status=self.mstat)
+        pct.tree_verify_walk(self.tree.tok, self.tree.parent, self.tree.count, self.T,
+                             max_depth=W.depth, out=self.walk)
 
     def step(self):
         pct = self.pct
@@ -289,64 +321,164 @@ def e2e_measure(rnd: Round, steps: int, dev):
     return ms / steps, h2d, d2h
 
 
-def oracle_round_sample(rnd: RoundInputs, req_ids, seed: int):
-    """Seconds the oracle, as it stands, spends on the given requests of the
-    round: PCTree build, CaDDTree grow, mask and verify. Inputs are the round's
-    drafter inputs; the target logits are drawn for these requests and planted
-    along the ORACLE's own trees (untimed), so nothing comes from the GPU path."""
-    import oracle
-    L = oracle.to_f64(rnd.L[req_ids])
-    E, Wm = oracle.to_f64(rnd.E), oracle.to_f64(rnd.W)
-    anc = rnd.anchor.cpu().numpy()[req_ids]
-    ctx = rnd.ctx.cpu().numpy()[req_ids]
-    t0 = time.perf_counter()
-    ref = oracle.pct_tree_build(L, anc, E, Wm, W.k, W.beam, W.n_nodes)
-    oracle.cadd_tree_grow(L, anc, ctx, C.n_max, **COST)
-    oracle.tree_ancestor_mask(ref.parent, ref.count, W.n_nodes)
-    t1 = time.perf_counter()
-    T = workloads.target_logits(len(req_ids), W.n_nodes, W.vocab,
-                                workloads.FULL_ROUND_TARGET_SIGMA, seed=seed)
-    workloads.plant_path(T, ref.tok, ref.parent, ref.count, seed=seed + 1)
-    t2 = time.perf_counter()
-    oracle.tree_verify_accept(ref.tok, ref.parent, ref.count, T, max_depth=W.depth)
-    t3 = time.perf_counter()
-    return (t1 - t0) + (t3 - t2)
-
-
 def host_cores():
     return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
 
 
-def cpu_baseline(rnd: Round, n_req: int = 1):
-    """The oracle on a bounded sample: n_req requests of the round."""
-    dt = oracle_round_sample(rnd, list(range(n_req)), seed=W.seed + 7000)
-    per_round = dt * W.batch / n_req
-    return {"value": 1.0 / per_round, "unit": "rounds/s", "cores": host_cores(), "kind": "oracle",
-            "sample": f"{n_req} of {W.batch} requests of one round (PCTree build, CaDDTree grow, "
-                      f"mask, verify), scaled to the {W.batch}-request round; {dt:.1f} s of CPU "
-                      "time; numpy float64, BLAS threads for the Markov matmul"}
+def blas_threads(n):
+    """Limit the BLAS pool of numpy to n threads inside the block (if possible)."""
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(n)
+    except ImportError:  # pragma: no cover
+        import contextlib
+        return contextlib.nullcontext()
 
 
-def roofline_entry(name, kinfo, launches, total_ms, steps, pk, pk_src):
+def oracle_requests(rnd: RoundInputs, req_ids, seed: int, threads: int):
+    """The oracle, as it stands, on the given requests of the round: PCTree
+    build, CaDDTree grow, mask and verify, one request per task over `threads`
+    host threads (BLAS one thread each). Inputs are the round's drafter inputs;
+    the target logits are drawn for these requests and planted along the
+    ORACLE's own trees (untimed), so nothing comes from the GPU path.
+    Returns (wall seconds, per-request PCTree results, per-request CaDDTree results)."""
+    from concurrent.futures import ThreadPoolExecutor
+    import oracle
+    E, Wm = oracle.to_f64(rnd.E), oracle.to_f64(rnd.W)
+    Lh = rnd.L.cpu()
+    anc = rnd.anchor.cpu().numpy()
+    ctx = rnd.ctx.cpu().numpy()
+
+    def build(b):
+        Lb = oracle.to_f64(Lh[b:b + 1])
+        ref = oracle.pct_tree_build(Lb, anc[b:b + 1], E, Wm, W.k, W.beam, W.n_nodes)
+        cad = oracle.cadd_tree_grow(Lb, anc[b:b + 1], ctx[b:b + 1], C.n_max, **COST)
+        oracle.tree_ancestor_mask(ref.parent, ref.count, W.n_nodes)
+        return ref, cad
+
+    with blas_threads(1), ThreadPoolExecutor(max_workers=threads) as ex:
+        t0 = time.perf_counter()
+        built = list(ex.map(build, req_ids))
+        t1 = time.perf_counter()
+        Ts = []
+        for j, (ref, _) in enumerate(built):       # untimed: targets along the oracle's trees
+            T = workloads.target_logits(1, W.n_nodes, W.vocab, workloads.FULL_ROUND_TARGET_SIGMA,
+                                        seed=seed + j)
+            workloads.plant_path(T, ref.tok, ref.parent, ref.count, seed=seed + 500 + j)
+            Ts.append(T)
+        t2 = time.perf_counter()
+        list(ex.map(lambda j: oracle.tree_verify_accept(built[j][0].tok, built[j][0].parent,
+                                                         built[j][0].count, Ts[j],
+                                                         max_depth=W.depth), range(len(built))))
+        t3 = time.perf_counter()
+    return (t1 - t0) + (t3 - t2), [b[0] for b in built], [b[1] for b in built]
+
+
+def _gpu_paths(tok, par, n):
+    paths, out = {0: ()}, set()
+    for i in range(1, n):
+        p = int(par[i])
+        if p < 0 or p >= i:
+            break
+        paths[i] = paths[p] + (int(tok[i]),)
+        out.add(paths[i])
+    return out
+
+
+def sample_parity(rnd, req_ids, refs, cads):
+    """The GPU's trees of the sampled requests against the oracle's (untimed):
+    node tables bit-exact, scores within 1e-4. A request the oracle marks as a
+    near tie (two candidates closer than 1e-4 at a cut, so either order is
+    correct) is compared against the oracle's tree with that tie resolved
+    toward the GPU's nodes; `excluded` counts requests matched neither way."""
+    import oracle
+    E, Wm = oracle.to_f64(rnd.E), oracle.to_f64(rnd.W)
+    Lh, anc, ctx = rnd.L.cpu(), rnd.anchor.cpu().numpy(), rnd.ctx.cpu().numpy()
+    out = {}
+    for name, gpu, res in (("pctree", rnd.tree, refs), ("caddtree", rnd.cadd, cads)):
+        tok, par, sc, cnt = (t.cpu().numpy() for t in (gpu.tok, gpu.parent, gpu.score, gpu.count))
+
+        def same(b, r):
+            n = int(r.count[0])
+            return bool(int(cnt[b]) == n and (tok[b] == r.tok[0]).all()
+                        and (par[b] == r.parent[0]).all()
+                        and np.abs(sc[b, :n] - r.score[0, :n]).max() <= 1e-4)
+
+        exact = resolved = excluded = 0
+        for b, r in zip(req_ids, res):
+            if not r.excluded[0]:
+                ok = same(b, r)
+                exact += ok
+                excluded += not ok
+                continue
+            paths = _gpu_paths(tok[b], par[b], int(cnt[b]))
+            Lb = oracle.to_f64(Lh[b:b + 1])
+            if name == "pctree":
+                alt = oracle.pct_tree_build(Lb, anc[b:b + 1], E, Wm, W.k, W.beam, W.n_nodes,
+                                            prefer=[paths])
+            else:
+                alt = oracle.cadd_tree_grow(Lb, anc[b:b + 1], ctx[b:b + 1], C.n_max, **COST,
+                                            prefer=[(paths, int(cnt[b]))])
+            ok = same(b, alt)
+            resolved += ok
+            excluded += not ok
+        out[name] = {"requests": len(req_ids), "exact": exact, "near_tie_resolved": resolved,
+                     "excluded": excluded}
+    return out
+
+
+def cpu_baseline(rnd: Round, n_multi: int = None):
+    """The oracle on a bounded sample of the round, timed two ways on the host
+    cores: one request on one thread, and one request per core on all cores."""
+    cores = host_cores()
+    n_multi = min(W.batch, cores) if n_multi is None else n_multi
+    t1, _, _ = oracle_requests(rnd, [0], seed=W.seed + 7000, threads=1)
+    ids = list(range(n_multi))
+    tm, refs, cads = oracle_requests(rnd, ids, seed=W.seed + 7000, threads=cores)
+    single = {"value": 1.0 / (t1 * W.batch), "unit": "rounds/s", "cores": 1,
+              "sample": f"request 0 of the {W.batch}-request round on one thread "
+                        f"({t1:.1f} s), scaled to the round"}
+    line = {"value": n_multi / (tm * W.batch), "unit": "rounds/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"requests 0..{n_multi - 1} of the {W.batch}-request round (PCTree build, "
+                      f"CaDDTree grow, mask, verify), one request per thread on {cores} host "
+                      f"threads ({tm:.1f} s), scaled to the round; numpy float64",
+            "single_thread": single}
+    return line, sample_parity(rnd, ids, refs, cads)
+
+
+def roofline_entry(name, launches, total_ms, steps, pk, pk_src, clocks=None):
+    """One kernel's roofline: algorithmic work per launch over its mean launch time.
+
+    Tensor-bound kernels are divided by the burst bf16 peak (the step runs for
+    milliseconds at the sampled clock); the fraction of the sustained peak is
+    given beside it. HBM-bound and latency-bound kernels are divided by the
+    measured copy bandwidth."""
     work = algorithmic_work()[name]
     per_launch_ms = total_ms / max(launches, 1)
     per_step_launches = launches / steps
+    extra = {}
     if work["bound"] == "tensor":
         units = work["flop"] / per_step_launches
         achieved = units / (per_launch_ms * 1e-3) / 1e12
-        peak = float(pk.get("bf16_tflops_sustained", pk.get("bf16_tflops")))
-        unit = "TFLOP/s"
+        peak = float(pk.get("bf16_tflops", pk.get("bf16_tflops_sustained")))
+        sus = float(pk.get("bf16_tflops_sustained", peak))
+        extra = {"frac_of_sustained": round(achieved / sus, 4), "sustained_peak": sus}
+        unit, src = "TFLOP/s", "burst bf16"
     else:
         units = work["bytes"] / per_step_launches
         achieved = units / (per_launch_ms * 1e-3) / 1e9
         peak = float(pk["hbm_gbs"])
-        unit = "GB/s"
-    return {"kernel": name, "bound": work["bound"], "achieved": round(achieved, 2),
-            "peak": peak, "unit": unit, "frac": round(achieved / peak, 4),
-            "peak_source": f"{pk_src} ({'sustained bf16' if unit == 'TFLOP/s' else 'HBM copy'})",
-            "traffic": ncu_traffic(name), "launches_per_step": per_step_launches,
-            "ms_per_launch": round(per_launch_ms, 4),
-            "algorithmic_per_launch": units}
+        unit, src = "GB/s", "HBM copy"
+    e = {"kernel": name, "bound": work["bound"], "achieved": round(achieved, 2),
+         "peak": peak, "unit": unit, "frac": round(achieved / peak, 4),
+         "peak_source": f"{pk_src} ({src})", "traffic": ncu_traffic(name),
+         "launches_per_step": per_step_launches, "ms_per_launch": round(per_launch_ms, 4),
+         "algorithmic_per_launch": units}
+    e.update(extra)
+    if clocks:
+        e["sm_mhz"] = clocks.get("sm_mhz")
+    return e
 
 
 # ---------------------------------------------------------------------------
@@ -365,99 +497,167 @@ def max_over_ranks(x: float, dist=None, dev=None) -> float:
     return float(t.item())
 
 
-def run_reference(args, rank, world, budget_s: float = 120.0):
+def run_reference(args, rank, world, budget_s: float = 150.0):
     """--impl reference: the CPU oracle on the same workload (rank 0 only).
 
-    Each step is a bounded sample of the round: one request (cycling through the
-    batch), all of its hot-path stages. Steps run until K steps or about
-    `budget_s` seconds of oracle time, whichever comes first; the line reports
-    the steps actually timed."""
+    A step is a bounded sample of the round: one request per host core (cycling
+    through the batch), every stage of the hot path, one request per thread.
+    Steps run until K steps or about `budget_s` seconds, whichever comes first;
+    the line reports the steps actually timed and the measured time per step."""
     if rank != 0:
         return 0
     if not torch.cuda.is_available():
         print(json.dumps({"impl": "reference", "unavailable": "no CUDA device to draw the inputs"}))
         return 0
     rnd = RoundInputs(torch.device("cuda", 0))
+    cores = host_cores()
+    per = min(cores, W.batch)
     times, spent = [], 0.0
     warm = min(args.warmup, 1)
     for i in range(warm + args.steps):
-        dt = oracle_round_sample(rnd, [i % W.batch], seed=W.seed + 9000 + i)
+        ids = [(i * per + j) % W.batch for j in range(per)]
+        dt, _, _ = oracle_requests(rnd, ids, seed=W.seed + 9000 + 100 * i, threads=cores)
         spent += dt
         if i >= warm:
             times.append(dt)
         if spent > budget_s and times:
             break
-    ms = statistics.mean(times) * W.batch * 1e3          # one 64-request round
-    value = 1e3 / ms
+    ms = statistics.mean(times) * 1e3                     # one step: `per` requests
+    value = per / (statistics.mean(times) * W.batch)      # 64-request rounds per second
     line = {"metric": METRIC, "value": value, "unit": "rounds/s", "n_gpus": 1,
             "steps": len(times), "steps_requested": args.steps, "warmup": warm,
-            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(),
-            "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "rounds/s", "cores": host_cores(),
-                             "kind": "oracle",
-                             "sample": f"one request of the {W.batch}-request round per step, "
-                                       f"{len(times)} steps, scaled to the round"},
+            "ms_per_step": ms, "requests_per_step": per, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "rounds/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{per} of the {W.batch} requests per step, one per "
+                                       f"thread on {cores} host threads, {len(times)} steps"},
             "e2e": {"value": value, "unit": "rounds/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
-def run_configs(args):
-    """One line per configuration of the hot path (not the default bench line):
-    GPU rounds/s over --steps timed runs after --warmup, the dominant kernel's
-    rate against the measured peak, and the oracle timed on one request of the
-    same inputs (host cores), scaled to the configuration's batch."""
+class L2Flush:
+    """Writes a buffer twice the size of L2 between timed runs (untimed)."""
+
+    def __init__(self, dev):
+        self.buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.buf.zero_()
+
+
+def warm_cold_ms(fn, dev, warm_runs, cold_runs, flush):
+    """Mean milliseconds per run: back to back (warm: inputs that fit in L2 stay
+    there) and with L2 flushed before every run (cold), each run bracketed by
+    its own events on the launch stream."""
+    fn()
+    torch.cuda.synchronize(dev)
+    warm = timed(fn, warm_runs, dev) / warm_runs
+    tot = 0.0
+    for _ in range(cold_runs):
+        flush()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        e.synchronize()
+        tot += s.elapsed_time(e)
+    return warm, tot / cold_runs
+
+
+def oracle_legs(fn, batch):
+    """The oracle on one request on one thread, and on min(batch, cores) requests
+    one per thread on all host cores; rates scaled to the configuration's batch."""
+    from concurrent.futures import ThreadPoolExecutor
+    cores = host_cores()
+    with blas_threads(1):
+        t0 = time.perf_counter()
+        fn(0)
+        t1 = time.perf_counter() - t0
+        n = min(batch, cores)
+        with ThreadPoolExecutor(max_workers=n) as ex:
+            t0 = time.perf_counter()
+            list(ex.map(fn, range(n)))
+            tm = time.perf_counter() - t0
+    return {"single_thread": {"rounds_per_s": 1.0 / (t1 * batch), "cores": 1,
+                              "sample": "1 request", "seconds": round(t1, 3)},
+            "all_cores": {"rounds_per_s": n / (tm * batch), "cores": cores,
+                          "sample": f"{n} requests, one per thread", "seconds": round(tm, 3)}}
+
+
+def config_results(dev, pk, quick=False):
+    """Every configuration of the hot path other than the full round: GPU rounds
+    per second warm and cold (L2 flushed before every round), the dominant
+    rate against its measured peak, and the oracle's rates (host cores)."""
     import oracle
     import speculative_decoding_draft_07_b200 as pct
-    dev = torch.device("cuda", 0)
-    pk, pk_src = peaks()
-    f64 = lambda t: t.detach().cpu().double().numpy() if t.dtype != torch.bfloat16 else \
-        t.detach().cpu().float().double().numpy()
-    lines = []
-
-    def gpu_rate(fn):
-        for _ in range(args.warmup):
-            fn()
-        return args.steps / (timed(fn, args.steps, dev) / 1e3)
-
-    def oracle_requests_per_s(fn):   # the oracle on one request
-        t0 = time.perf_counter()
-        fn()
-        return 1.0 / (time.perf_counter() - t0)
-
+    flush = L2Flush(dev)
+    f64 = oracle.to_f64
+    hbm, tc = float(pk["hbm_gbs"]), float(pk.get("bf16_tflops", pk.get("bf16_tflops_sustained")))
+    res = {}
     for name in ("tiny", "qwen3_4b_scale", "long_block"):
         w = workloads.WORKLOADS[name]
         d = workloads.drafter_inputs(w, device=dev)
         L, a, E, Wm = d["L"], d["anchor"], d["E"], d["W"]
-        r = gpu_rate(lambda: pct.pct_tree_build(L, a, E, Wm, w.k, w.beam, w.n_nodes))
+        out = pct.pct_tree_build(L, a, E, Wm, w.k, w.beam, w.n_nodes)
+        ws = torch.empty(pct.pct_tree_build_workspace(pct.build_desc(
+            w.batch, w.depth, w.vocab, w.rank, w.k, w.beam, w.n_nodes,
+            pct.PCT_BF16 if L.dtype == torch.bfloat16 else pct.PCT_F32,
+            pct.PCT_BF16 if E.dtype == torch.bfloat16 else pct.PCT_F32)), dtype=torch.uint8,
+            device=dev)
+        fn = lambda: pct.pct_tree_build(L, a, E, Wm, w.k, w.beam, w.n_nodes, out=out, workspace=ws)
+        runs = 20 if name == "long_block" else 200
+        warm, cold = warm_cold_ms(fn, dev, runs, max(runs // 4, 10), flush)
         F = [1]
         for _ in range(w.depth):
             F.append(min(w.beam, F[-1] * w.k))
-        rows = sum(w.batch * F[d_ - 1] for d_ in range(1, w.depth + 1))
+        rows = sum(w.batch * F[i - 1] for i in range(1, w.depth + 1))
         flop = 2.0 * w.rank * w.vocab * rows
-        wbytes = float(w.rank * w.vocab * (2 if w.dtype == "bf16" else 4) * w.depth)
-        o_rate = oracle_requests_per_s(lambda: oracle.pct_tree_build(
-            f64(L[:1]), a[:1].cpu().numpy(), f64(E), f64(Wm), w.k, w.beam, w.n_nodes))
-        lines.append({"config": name, "rounds_per_s": r, "requests": w.batch,
-                      "tflops": flop * r / 1e12, "frac_bf16_sustained": flop * r / 1e12 /
-                      float(pk["bf16_tflops_sustained"]),
-                      "w_stream_gbs": wbytes * r / 1e9,
-                      "frac_hbm": wbytes * r / 1e9 / float(pk["hbm_gbs"]),
-                      "oracle_rounds_per_s": o_rate / w.batch, "oracle_sample": "1 request"})
+        esz = 2 if w.dtype == "bf16" else 4
+        wbytes = float(w.depth * (w.rank * w.vocab + w.batch * w.vocab) * esz)   # W per depth + L
+        e = {"workload": name, "requests": w.batch, "rounds_per_s_warm": 1e3 / warm,
+             "rounds_per_s_cold": 1e3 / cold, "ms_per_round_cold": cold,
+             "tflops_cold": flop / cold / 1e9, "frac_bf16_burst_cold": flop / cold / 1e9 / tc,
+             "stream_gbs_cold": wbytes / cold / 1e6, "frac_hbm_cold": wbytes / cold / 1e6 / hbm,
+             "stream_gbs_warm": wbytes / warm / 1e6,
+             "bound": "tensor" if name == "long_block" else ("hbm" if name != "tiny" else "launch")}
+        if not quick:
+            Lh, Eh, Wh, ah = L.cpu(), f64(E), f64(Wm), a.cpu().numpy()
+            e["oracle"] = oracle_legs(lambda b: oracle.pct_tree_build(
+                f64(Lh[b:b + 1]), ah[b:b + 1], Eh, Wh, w.k, w.beam, w.n_nodes), w.batch)
+        res[name] = e
+        del d, L, E, Wm, out, ws
     for ell in C.ells:
         d = workloads.cadd_inputs(C, ell, device=dev)
         L, a, ctx = d["L"], d["anchor"], d["ctx_len"]
-        r = gpu_rate(lambda: pct.cadd_tree_grow(L, a, ctx, C.n_max, **COST))
+        out = pct.cadd_tree_grow(L, a, ctx, C.n_max, **COST)
+        fn = lambda: pct.cadd_tree_grow(L, a, ctx, C.n_max, **COST, out=out)
+        warm, cold = warm_cold_ms(fn, dev, 100, 25, flush)
         nbytes = float(L.numel() * L.element_size())
-        o_rate = oracle_requests_per_s(lambda: oracle.cadd_tree_grow(
-            f64(L[:1]), a[:1].cpu().numpy(), ctx[:1].cpu().numpy(), C.n_max, **COST))
-        lines.append({"config": f"caddtree_l{ell}", "rounds_per_s": r, "requests": C.batch,
-                      "gbs": nbytes * r / 1e9, "frac_hbm": nbytes * r / 1e9 / float(pk["hbm_gbs"]),
-                      "oracle_rounds_per_s": o_rate / C.batch, "oracle_sample": "1 request"})
-    for ln in lines:
-        print(json.dumps({k: (round(v, 6) if isinstance(v, float) else v) for k, v in ln.items()}))
+        e = {"workload": f"caddtree_l{ell}", "requests": C.batch, "rounds_per_s_warm": 1e3 / warm,
+             "rounds_per_s_cold": 1e3 / cold, "ms_per_round_cold": cold,
+             "gbs_cold": nbytes / cold / 1e6, "frac_hbm_cold": nbytes / cold / 1e6 / hbm,
+             "mean_nodes": float(out.count.float().mean()), "bound": "hbm"}
+        if not quick:
+            Lh, ah, ch = L.cpu(), a.cpu().numpy(), ctx.cpu().numpy()
+            e["oracle"] = oracle_legs(lambda b: oracle.cadd_tree_grow(
+                f64(Lh[b:b + 1]), ah[b:b + 1], ch[b:b + 1], C.n_max, **COST), C.batch)
+        res[f"caddtree_l{ell}"] = e
+        del d, L, out
+    del flush
+    torch.cuda.empty_cache()
+    return {k: {kk: (round(vv, 6) if isinstance(vv, float) else vv) for kk, vv in v.items()}
+            for k, v in res.items()}
+
+
+def run_configs(args):
+    """--configs: one line per configuration (not the default bench line)."""
+    dev = torch.device("cuda", 0)
+    pk, _ = peaks()
+    for name, e in config_results(dev, pk).items():
+        print(json.dumps(e))
     return 0
 
 
@@ -487,6 +687,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="leave the per-configuration results out of the bench line")
     ap.add_argument("--requests", type=int, default=W.batch,
                     help="requests per round (smaller only for profiling captures)")
     ap.add_argument("--profile-stage", default=None, choices=["pctree", "cadd"],
@@ -535,13 +737,27 @@ def main():
     time.sleep(0.3)
     if dist is not None:
         dist.barrier()
+    torch.cuda.cudart().cudaProfilerStart()   # a profiler started with capture off records only this
     ms = timed(rnd.step, args.steps, dev)
+    torch.cuda.cudart().cudaProfilerStop()
     clocks = sampler.stop()
     kernels = pct.trace_read()
     pct.trace_enable(False)
     ms = max_over_ranks(ms, dist, dev)
     ms_step = ms / args.steps
     value = world * 1e3 / ms_step
+
+    # the same round with the lazy verification walk (argmax of the walked rows only)
+    for _ in range(3):
+        rnd.step_lazy()
+    pct.trace_enable(True)
+    pct.trace_reset()
+    if dist is not None:
+        dist.barrier()
+    ms_lazy = max_over_ranks(timed(rnd.step_lazy, args.steps, dev), dist, dev) / args.steps
+    kl = pct.trace_read()
+    pct.trace_enable(False)
+    walked_rows = int((rnd.walk.accept_len.to(torch.int64) + 1).sum().item())
 
     # end-to-end through the public API with host buffers
     e2e_ms, h2d, d2h = e2e_measure(rnd, args.e2e_steps, dev)
@@ -550,7 +766,7 @@ def main():
     if rank == 0:
         pk, pk_src = peaks()
         launches = sum(v[0] for v in kernels.values())
-        roofs = [roofline_entry(n, None, kernels[n][0], kernels[n][1], args.steps, pk, pk_src)
+        roofs = [roofline_entry(n, kernels[n][0], kernels[n][1], args.steps, pk, pk_src, clocks)
                  for n in algorithmic_work() if n in kernels]
         dominant = max(kernels, key=lambda n: kernels[n][1]) if kernels else None
         main_roof = next((r for r in roofs if r["kernel"] == dominant), roofs[0] if roofs else None)
@@ -568,8 +784,22 @@ def main():
             "e2e": {"value": world * 1e3 / e2e_ms, "unit": "rounds/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
         }
+        wl = kl.get("verify_walk", (1, 0.0))
+        walk_bytes = float(walked_rows * W.vocab * 2)
+        line["lazy_verify"] = {
+            "value": world * 1e3 / ms_lazy, "unit": "rounds/s", "ms_per_step": ms_lazy,
+            "note": "the round with tree_verify_walk in place of the full argmax: same "
+                    "acceptance, only the rows the walk reaches are read",
+            "verify_walk_ms_per_step": wl[1] / args.steps,
+            "walked_rows_per_step": walked_rows, "bytes_read_per_step": walk_bytes,
+            "walk_gbs": walk_bytes / (wl[1] / args.steps * 1e-3) / 1e9 if wl[1] > 0 else None,
+            "full_argmax_bytes_per_step": algorithmic_work()["verify_argmax_walk"]["bytes"]}
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(rnd, n_req=2)
+            line["cpu_baseline"], line["parity_sample"] = cpu_baseline(rnd)
+            line["excluded"] = line["parity_sample"]["pctree"]["excluded"] + \
+                line["parity_sample"]["caddtree"]["excluded"]
+        if world == 1 and not args.no_configs:
+            line["configs"] = config_results(dev, pk)
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()

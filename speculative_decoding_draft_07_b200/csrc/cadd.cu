@@ -30,6 +30,7 @@
 //    parent insertion index, rank) so that one warp max-reduction pops the
 //    best node under the library's total order; the stop test is evaluated in
 //    log form, s > log((1 + Phi) dC(n) / C(n)), before each insertion.
+#include <algorithm>
 #include <climits>
 
 #include "common.cuh"
@@ -458,9 +459,24 @@ __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
   asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
-__device__ __forceinline__ float group_max(const uint4& q) {
-  const uint32_t mx = bf16x2_max(bf16x2_max(q.x, q.y), bf16x2_max(q.z, q.w));
-  return fmaxf(bf16_lo(mx), bf16_hi(mx));
+// Per half: 0xffff where a > b (bf16 compare), else 0.
+__device__ __forceinline__ uint32_t bf16x2_gt(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("set.gt.u32.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+// The largest bf16 value not above t, in both halves. For any bf16 x: x > t
+// exactly when x > that value. A NaN t gives +inf (no x passes, as no x > NaN).
+__device__ __forceinline__ uint32_t bf16_pair_round_down(float t) {
+  uint32_t h;
+  if (t != t) {
+    h = 0x7f80u;
+  } else {
+    const uint32_t u = __float_as_uint(t);
+    h = u >> 16;                               // truncation: toward zero (infinities exact)
+    if ((u & 0xffffu) != 0u && (u & 0x80000000u)) h += 1u;   // negative: one step further down
+  }
+  return h | (h << 16);
 }
 
 // Sum of s_i 2^((m_i - M) log2 e) with M the block-wide max of m_i, in a fixed
@@ -531,77 +547,115 @@ struct SegWs {
   unsigned long long* surv;    // [rows][S][kSegCap] survivor keys
 };
 
-__global__ __launch_bounds__(kSegThreads, 6) void cadd_seg_rowpass_kernel(
-    CaddParams p, const __nv_bfloat16* __restrict__ L, const int64_t* __restrict__ ctx, SegWs w) {
-  __shared__ float2 wred[kSegThreads / 32];
-  __shared__ uint4 stg_v[kSegThreads / 32][kSegG * 32];   // candidate groups, per warp
-  __shared__ int stg_g[kSegThreads / 32][kSegG * 32];
-  __shared__ int s_cnt;
-
-  const int V = p.V;
-  const int S = seg_count(V);
-  const int row = blockIdx.x / S, seg = blockIdx.x - row * S;
-  const int b = row / p.D;
-  const int K = p.n_max - 1;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// One (row, segment) work item of the row pass.
+struct SegItem {
+  int row, seg, g0, ng;
+};
+__device__ __forceinline__ SegItem seg_item(int item, int V, int S) {
+  SegItem it;
+  it.row = item / S;
+  it.seg = item - it.row * S;
   const int ngroups = V >> 3;
   const int g_per = (ngroups + S - 1) / S;
-  const int g0 = min(ngroups, seg * g_per);
-  const int ng = min(ngroups, g0 + g_per) - g0;
-  const uint4* src = reinterpret_cast<const uint4*>(L + (size_t)row * V) + g0;
-
-  // the whole segment in flight: kSegG independent 16-byte loads per thread
-  // (groups past the segment read as -inf)
-  uint4 q[kSegG];
+  it.g0 = min(ngroups, it.seg * g_per);
+  it.ng = min(ngroups, it.g0 + g_per) - it.g0;
+  return it;
+}
+// The item's segment into registers: kSegG independent 16-byte loads per
+// thread (groups past the segment read as -inf).
+__device__ __forceinline__ void seg_load(const __nv_bfloat16* __restrict__ L, int V,
+                                         const SegItem& it, uint4 (&q)[kSegG]) {
+  const uint4* src = reinterpret_cast<const uint4*>(L + (size_t)it.row * V) + it.g0;
 #pragma unroll
   for (int j = 0; j < kSegG; ++j) {
     const int g = j * kSegThreads + threadIdx.x;
-    q[j] = g < ng ? ld_stream16(src + g) : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+    q[j] = g < it.ng ? ld_stream16(src + g)
+                     : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
   }
+}
+
+struct SegSmem {
+  float2 wred[kSegThreads / 32];
+  uint4 stg_v[kSegThreads / 32][kSegG * 32];   // candidate groups, per warp
+  int stg_g[kSegThreads / 32][kSegG * 32];
+  int s_cnt;
+};
+
+// Everything after the loads for one item: partial log-sum-exp, the local
+// filter, and the item's slot in the workspace.
+__device__ __forceinline__ void seg_process(const CaddParams& p, const int64_t* __restrict__ ctx,
+                                            const SegWs& w, const SegItem& it,
+                                            const uint4 (&q)[kSegG], SegSmem& sm) {
+  float2* wred = sm.wred;
+  auto& stg_v = sm.stg_v;
+  auto& stg_g = sm.stg_g;
+  int& s_cnt = sm.s_cnt;
+  const int S = seg_count(p.V);
+  const int row = it.row, seg = it.seg, g0 = it.g0;
+  const int b = row / p.D;
+  const int K = p.n_max - 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) s_cnt = 0;
   const float lnth = cadd_ln_theta_closed(p, (float)ctx[b]) - kThetaSlack;
 
-  // partial log-sum-exp against the thread's own maximum (no rescaling)
-  float m = neg_inf();
+  // packed maxima: gm[j] holds the larger of each half-pair of group j's words,
+  // so max(lo, hi) of gm[j] is the group's maximum; their tree gives the thread's
+  uint32_t gm[kSegG];
 #pragma unroll
-  for (int j = 0; j < kSegG; ++j) m = fmaxf(m, group_max(q[j]));
+  for (int j = 0; j < kSegG; ++j)
+    gm[j] = bf16x2_max(bf16x2_max(q[j].x, q[j].y), bf16x2_max(q[j].z, q[j].w));
+  uint32_t tmx = gm[0];
+#pragma unroll
+  for (int j = 1; j < kSegG; ++j) tmx = bf16x2_max(tmx, gm[j]);
+  const float m = fmaxf(bf16_lo(tmx), bf16_hi(tmx));
+
+  // partial log-sum-exp against the thread's own maximum (no rescaling), four
+  // independent scalar sums
   float s = 0.f;
   if (m != neg_inf()) {
-    const float2 nmb = make_float2(-m * kLog2e, -m * kLog2e);
-    const float2 l2e = make_float2(kLog2e, kLog2e);
-    float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+    const float nmb = -m * kLog2e;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
     for (int j = 0; j < kSegG; ++j) {
       const uint4 v = q[j];
-      const float2 a0 = f2_fma(make_float2(bf16_lo(v.x), bf16_hi(v.x)), l2e, nmb);
-      const float2 a1 = f2_fma(make_float2(bf16_lo(v.y), bf16_hi(v.y)), l2e, nmb);
-      const float2 a2 = f2_fma(make_float2(bf16_lo(v.z), bf16_hi(v.z)), l2e, nmb);
-      const float2 a3 = f2_fma(make_float2(bf16_lo(v.w), bf16_hi(v.w)), l2e, nmb);
-      acc0 = f2_add(acc0, f2_add(make_float2(ex2(a0.x), ex2(a0.y)), make_float2(ex2(a1.x), ex2(a1.y))));
-      acc1 = f2_add(acc1, f2_add(make_float2(ex2(a2.x), ex2(a2.y)), make_float2(ex2(a3.x), ex2(a3.y))));
+      a0 += ex2(fmaf(bf16_lo(v.x), kLog2e, nmb));
+      a1 += ex2(fmaf(bf16_hi(v.x), kLog2e, nmb));
+      a2 += ex2(fmaf(bf16_lo(v.y), kLog2e, nmb));
+      a3 += ex2(fmaf(bf16_hi(v.y), kLog2e, nmb));
+      a0 += ex2(fmaf(bf16_lo(v.z), kLog2e, nmb));
+      a1 += ex2(fmaf(bf16_hi(v.z), kLog2e, nmb));
+      a2 += ex2(fmaf(bf16_lo(v.w), kLog2e, nmb));
+      a3 += ex2(fmaf(bf16_hi(v.w), kLog2e, nmb));
     }
-    const float2 acc = f2_add(acc0, acc1);
-    s = acc.x + acc.y;
+    s = (a0 + a1) + (a2 + a3);
   }
   const float2 ps = block_lse_fixed(m, s, wred);
   const float lse_seg = (ps.x == neg_inf()) ? neg_inf() : ps.x + logf(ps.y);
   const float t_loc = (K <= 0) ? __int_as_float(0x7f800000) : lse_seg + lnth - kSegMargin;
 
-  // the segment's values above its own threshold, into its slot. Groups whose
-  // max reaches it are first packed per warp into shared memory (ballot
-  // compaction), then tested value by value one group per lane, so the rare
+  // the segment's values above its own threshold, into its slot. A bf16 value
+  // exceeds t_loc exactly when it exceeds t_loc rounded down to bf16, so each
+  // group is tested with one packed compare of its maxima. Groups that pass are
+  // packed per warp into shared memory (ballot compaction, only in warps that
+  // have any), then tested value by value one group per lane, so the rare
   // candidates cost no divergent passes over the registers.
-  int nst = 0;   // staged groups of this warp
+  const uint32_t tpair = bf16_pair_round_down(t_loc);
+  uint32_t hits = 0;
 #pragma unroll
-  for (int j = 0; j < kSegG; ++j) {
-    const bool c = group_max(q[j]) > t_loc;
-    const unsigned ball = __ballot_sync(0xffffffffu, c);
-    if (c) {
-      const int at = nst + __popc(ball & ((1u << lane) - 1u));
-      stg_v[warp][at] = q[j];
-      stg_g[warp][at] = g0 + j * kSegThreads + threadIdx.x;
+  for (int j = 0; j < kSegG; ++j) hits |= (bf16x2_gt(gm[j], tpair) != 0u ? 1u : 0u) << j;
+  int nst = 0;   // staged groups of this warp
+  if (__any_sync(0xffffffffu, hits != 0u)) {
+#pragma unroll
+    for (int j = 0; j < kSegG; ++j) {
+      const bool c = (hits >> j) & 1u;
+      const unsigned ball = __ballot_sync(0xffffffffu, c);
+      if (c) {
+        const int at = nst + __popc(ball & ((1u << lane) - 1u));
+        stg_v[warp][at] = q[j];
+        stg_g[warp][at] = g0 + j * kSegThreads + threadIdx.x;
+      }
+      nst += __popc(ball);
     }
-    nst += __popc(ball);
   }
   __syncwarp();
   const size_t slot = (size_t)row * S + seg;
@@ -644,6 +698,18 @@ __global__ __launch_bounds__(kSegThreads, 6) void cadd_seg_rowpass_kernel(
     w.cnt[slot] = s_cnt;
     if (seg == 0) w.lnth[row] = lnth;
   }
+}
+
+// One CTA per (row, segment) item, with the whole segment's loads in flight at
+// once (measured: persistent CTAs double-buffering two items in registers fit
+// half as many CTAs per SM and were slower, 109 us against 79 us at 960 rows).
+__global__ __launch_bounds__(kSegThreads, 6) void cadd_seg_rowpass_kernel(
+    CaddParams p, const __nv_bfloat16* __restrict__ L, const int64_t* __restrict__ ctx, SegWs w) {
+  __shared__ SegSmem sm;
+  const SegItem it = seg_item(blockIdx.x, p.V, seg_count(p.V));
+  uint4 q[kSegG];
+  seg_load(L, p.V, it, q);
+  seg_process(p, ctx, w, it, q, sm);
 }
 
 __global__ __launch_bounds__(kSegThreads) void cadd_seg_finish_kernel(
@@ -763,6 +829,7 @@ __device__ __forceinline__ unsigned long long pool_key(float s, int depth, int p
          ((unsigned long long)(1023 - pidx) << 10) | (unsigned long long)(1023 - rank);
 }
 
+template <bool STAGED>
 __global__ __launch_bounds__(32) void cadd_bestfirst_kernel(
     CaddParams p, const int32_t* __restrict__ anchor, const int64_t* __restrict__ ctx,
     const int32_t* __restrict__ cand_cnt, const float* __restrict__ cand_q,
@@ -771,23 +838,66 @@ __global__ __launch_bounds__(32) void cadd_bestfirst_kernel(
     float* __restrict__ ophi, int32_t* __restrict__ status) {
   extern __shared__ unsigned long long pool[];          // [n_max + 1]
   const int nmax = p.n_max;
+  const int D = p.D, K1 = max(nmax - 1, 1);
   int* ntok = reinterpret_cast<int*>(pool + nmax + 1);  // [n_max] each
   int* npar = ntok + nmax;
   int* ndep = npar + nmax;
   float* ns = reinterpret_cast<float*>(ndep + nmax);
   int* canon = reinterpret_cast<int*>(ns + nmax);
   int* order = canon + nmax;
-  __shared__ int dstart[66], dfill[66];
+  float* sq = reinterpret_cast<float*>(order + nmax);   // [D][K1] the request's candidates
+  int* stk = reinterpret_cast<int*>(sq + (size_t)D * K1);
+  __shared__ int dstart[66], dfill[66], scnt[64];
 
   const int b = blockIdx.x, lane = threadIdx.x;
-  const int D = p.D, K1 = max(nmax - 1, 1);
   const size_t row0 = (size_t)b * D;
   const int a0 = anchor[b];
   if (lane == 0 && (a0 < 0 || a0 >= p.V)) atomicOr(&status[b], PCT_DEV_BAD_TOKEN);
   if (lane == 0) { ntok[0] = a0; npar[0] = -1; ndep[0] = 0; ns[0] = 0.f; }
 
-  auto cnt_at = [&](int depth) { return cand_cnt[row0 + depth - 1]; };
-  auto q_at = [&](int depth, int rank) { return cand_q[(row0 + depth - 1) * K1 + rank]; };
+  // the request's candidate lists, staged once when they fit in shared memory:
+  // the growth below reads them one pop after another, so each read would
+  // otherwise be a dependent trip to L2 on the sequential path
+  for (int dd = lane; dd < D; dd += 32) scnt[dd] = min(max(cand_cnt[row0 + dd], 0), K1);
+  __syncwarp();
+  if (STAGED) {
+    // all rows' candidates as one index space (row offsets in dstart), eight
+    // loads per lane issued before any is stored
+    if (lane == 0) {
+      int acc = 0;
+      for (int dd = 0; dd < D; ++dd) { dstart[dd] = acc; acc += scnt[dd]; }
+      dstart[D] = acc;
+    }
+    __syncwarp();
+    const int total = dstart[D];
+    constexpr int U = 8;
+    for (int base = 0; base < total; base += 32 * U) {
+      float qv[U];
+      int tv[U], at[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int f = base + u * 32 + lane;
+        at[u] = -1;
+        if (f < total) {
+          int dd = 0;
+          while (dstart[dd + 1] <= f) ++dd;
+          const int j = f - dstart[dd];
+          const size_t g = (row0 + dd) * K1 + j;
+          qv[u] = cand_q[g];
+          tv[u] = cand_tok[g];
+          at[u] = dd * K1 + j;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (at[u] >= 0) { sq[at[u]] = qv[u]; stk[at[u]] = tv[u]; }
+    }
+    __syncwarp();
+  }
+  auto cnt_at = [&](int depth) { return scnt[depth - 1]; };
+  auto q_at = [&](int depth, int rank) {
+    return STAGED ? sq[(depth - 1) * K1 + rank] : cand_q[(row0 + depth - 1) * K1 + rank];
+  };
   int pool_n = 0;
   if (D >= 1 && nmax > 1 && cnt_at(1) > 0) {
     if (lane == 0) pool[0] = pool_key(q_at(1, 0), 1, 0, 0);
@@ -820,7 +930,7 @@ __global__ __launch_bounds__(32) void cadd_bestfirst_kernel(
     const float dC = p.c + p.e * (2.f * fn + 1.f);
     const float thr = dC > 0.f ? logf((1.f + phi) * dC / Cn) : neg_inf();
     if (!(s > thr)) break;
-    const int tk = cand_tok[(row0 + depth - 1) * K1 + rank];
+    const int tk = STAGED ? stk[(depth - 1) * K1 + rank] : cand_tok[(row0 + depth - 1) * K1 + rank];
     const int np = pidx;
     unsigned long long sib = 0ull, child = 0ull;
     if (rank + 1 < cnt_at(depth)) sib = pool_key(ns[np] + q_at(depth, rank + 1), depth, np, rank + 1);
@@ -937,15 +1047,18 @@ cudaError_t launch_cadd(const CaddParams& p, const void* L, const int32_t* ancho
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  const size_t smem = (size_t)(p.n_max + 1) * 8 + (size_t)p.n_max * 4 * 6;
+  const size_t base = (size_t)(p.n_max + 1) * 8 + (size_t)p.n_max * 4 * 6;
+  const size_t staged = base + (size_t)p.D * std::max(p.n_max - 1, 1) * 8;
+  const bool stage = staged <= 160 * 1024;
+  const size_t smem = stage ? staged : base;
+  auto kern = stage ? cadd_bestfirst_kernel<true> : cadd_bestfirst_kernel<false>;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(cadd_bestfirst_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
   TraceScope t(s, "cadd_bestfirst");
-  cadd_bestfirst_kernel<<<p.batch, 32, smem, s>>>(p, anchor, ctx, cand_cnt, cand_q, cand_tok, tok,
-                                                  parent, depth, score, count, phi, status);
+  kern<<<p.batch, 32, smem, s>>>(p, anchor, ctx, cand_cnt, cand_q, cand_tok, tok, parent, depth,
+                                 score, count, phi, status);
   return cudaGetLastError();
 }
 

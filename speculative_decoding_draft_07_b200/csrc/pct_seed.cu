@@ -37,6 +37,13 @@ __device__ __forceinline__ void load8<float>(const float* p, float (&x)[8]) {
   x[6] = __uint_as_float(b.z); x[7] = __uint_as_float(b.w);
 }
 
+// Elementwise max of two packed bf16 pairs.
+__device__ __forceinline__ uint32_t bf16x2_max2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 __device__ __forceinline__ float max8(const float (&x)[8]) {
   return fmaxf(fmax3(x[0], x[1], x[2]), fmax3(fmax3(x[3], x[4], x[5]), x[6], x[7]));
 }
@@ -56,6 +63,24 @@ __global__ void __launch_bounds__(kSeedThreads) drafter_topk_kernel(
   float best = neg_inf();
   int bg = -1;
   constexpr int U = 8;   // 16-byte groups in flight per thread
+  if constexpr (sizeof(TL) == 2) {
+    // bf16: every load of a pass issued before any is used, maxima on packed pairs
+    for (int g0 = threadIdx.x; g0 < G; g0 += U * kSeedThreads) {
+      uint4 q[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int g = g0 + u * kSeedThreads;
+        q[u] = g < G ? ld_stream16(row + (size_t)g * 8)
+                     : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t mx = bf16x2_max2(bf16x2_max2(q[u].x, q[u].y), bf16x2_max2(q[u].z, q[u].w));
+        const float gm = fmaxf(bf16_lo(mx), bf16_hi(mx));
+        if (gm > best) { best = gm; bg = g0 + u * kSeedThreads; }
+      }
+    }
+  } else
   for (int g0 = threadIdx.x; g0 < G; g0 += U * kSeedThreads) {
     float x[U][8];
 #pragma unroll

@@ -294,8 +294,13 @@ int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t*
   if (P.chain && aligned(E, 16) && aligned(W, 16) && aligned(L, 16)) {
     // every depth in one persistent launch, then the global top-N
     int32_t* cerr = nullptr;
+    int32_t* ccol = reinterpret_cast<int32_t*>(ws + P.o_scol);
+    float* clval = reinterpret_cast<float*>(ws + P.o_slval);
+    float* cwmax = reinterpret_cast<float*>(ws + P.o_swmax);
+    PCT_CU(launch_drafter_topk(P.batch * P.D, P.V, P.k, P.ldt, L, W, P.r, P.r_pad, ccol, clval,
+                               cwmax, ws + P.o_swcol, s));
     PCT_CU(launch_chain(chain_shape(P), L, anchor, E, W, ws + P.o_chain, ltok, lppos, ls, &cerr,
-                        dev_status, s));
+                        dev_status, ccol, clval, cwmax, ws + P.o_swcol, s));
     FinalArgs f;
     f.batch = P.batch; f.D = P.D; f.beam = P.beam; f.N = P.N;
     for (int d = 0; d <= P.D; ++d) f.F[d] = P.F[d];

@@ -140,9 +140,13 @@ struct ChainShape {
 };
 bool chain_eligible(const ChainShape& c);           // shape and current device
 size_t chain_workspace(const ChainShape& c);
+// Seeds: [batch][D][k] columns, L_d and max|W| there, W's columns [..][r_pad]
+// (launch_drafter_topk's output).
 cudaError_t launch_chain(const ChainShape& c, const void* L, const int32_t* anchor, const void* E,
                          const void* W, void* ws, int32_t* lvl_tok, int32_t* lvl_ppos, float* lvl_s,
-                         int32_t** err_out, int32_t* status, cudaStream_t s);
+                         int32_t** err_out, int32_t* status, const int32_t* scol,
+                         const float* slval, const float* swmax, const void* swcol,
+                         cudaStream_t s);
 
 struct FinalArgs {
   int batch, D, beam, N;

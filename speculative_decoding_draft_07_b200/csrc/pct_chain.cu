@@ -45,6 +45,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "seed.cuh"
 #include "select.cuh"
 #include "umma.cuh"
 
@@ -68,6 +69,10 @@ constexpr int C_MAXBEAM = 32;
 constexpr int C_KEYS = 2048;                         // rows x k beam candidates
 constexpr int C_CH = 32;                             // accumulator columns per TMEM load
 constexpr int C_TMEM_COLS = 2 * C_BN;
+// the next depth's seed data, prefetched while the current depth is scored
+// when every request's fits: W columns (k x r_pad bf16 per request), then the
+// columns, L_d there and max|W| there (k each per request)
+constexpr int C_PRE = 8192 + 3 * 4 * 256;
 
 // kind::f16 instruction descriptor: D f32, A = B = bf16, A K-major, B
 // MN-major, N = 128, M = 128.
@@ -77,7 +82,7 @@ constexpr uint32_t C_IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (
 template <int KMAX>
 constexpr size_t chain_smem_bytes() {
   return 1024 + (size_t)C_KBMAX * C_A_KB + (size_t)C_STAGES * C_B_STAGE + 2 * (size_t)C_LPART +
-         C_ONEHOT + C_KEYS * 8 + C_ROWS * (8 + 8 * KMAX) + C_ROWS * 12 + 64 + 256;
+         C_ONEHOT + C_KEYS * 8 + C_ROWS * (8 + 8 * KMAX) + C_ROWS * 16 + C_PRE + 64 + 256;
 }
 
 struct ChainParams {
@@ -95,6 +100,12 @@ struct ChainParams {
   int32_t* lvl_ppos;
   float* lvl_s;
   int32_t* status;                // [batch]
+  // admission seeds per (request, depth): the k best drafter-logit columns,
+  // L_d and max|W| there, and W's columns (bf16, r_pad wide)
+  const int32_t* scol;
+  const float* slval;
+  const float* swmax;
+  const __nv_bfloat16* swcol;
 };
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
@@ -103,6 +114,15 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+// Tile load of W kept in L2 (evict-last): W is read again at every depth.
+__device__ __forceinline__ void tma_load_2d_keep(void* dst, const CUtensorMap* map, int x, int y,
+                                                 uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
 __device__ __forceinline__ void epi_sync() {
@@ -127,9 +147,11 @@ __device__ void build_a_tile(const ChainParams& p, int M, int Fd, const int* fto
                              uint8_t* sOneHot) {
   const int t = threadIdx.x - 64;                  // 0..127
   const int R = copies_for(M), rpc = C_BM / R;
+  // every (row, chunk) of the M rows is loaded once and stored to each of the
+  // R copies; the rest of the tile (rows past M in each copy) is zero
   const int per_row = p.kblocks * 8;               // 16-byte chunks per A row
-  const int total = C_BM * per_row;
-  constexpr int B = 16;                            // chunks in flight per thread
+  const int total = M * per_row;
+  constexpr int B = 8;                             // chunks in flight per thread
   for (int i0 = t; i0 < total; i0 += B * C_EPI * 32) {
     uint4 v[B];
 #pragma unroll
@@ -137,10 +159,9 @@ __device__ void build_a_tile(const ChainParams& p, int M, int Fd, const int* fto
       const int idx = i0 + j * C_EPI * 32;
       v[j] = make_uint4(0u, 0u, 0u, 0u);
       if (idx < total) {
-        const int a = idx / per_row, rem = idx - a * per_row;
+        const int r = idx / per_row, rem = idx - r * per_row;
         const int kk = (rem >> 3) * C_BK + (rem & 7) * 8;
-        const int r = a - (a / rpc) * rpc;
-        if (r < M && kk < p.r) {
+        if (kk < p.r) {
           const int tok = (unsigned)ftok[r] < (unsigned)p.V ? ftok[r] : 0;
           v[j] = __ldg(reinterpret_cast<const uint4*>(p.E + (size_t)tok * p.r + kk));
         }
@@ -150,11 +171,21 @@ __device__ void build_a_tile(const ChainParams& p, int M, int Fd, const int* fto
     for (int j = 0; j < B; ++j) {
       const int idx = i0 + j * C_EPI * 32;
       if (idx < total) {
-        const int a = idx / per_row, rem = idx - a * per_row;
+        const int r = idx / per_row, rem = idx - r * per_row;
         const int kb = rem >> 3, c8 = rem & 7;
-        *reinterpret_cast<uint4*>(sA + kb * C_A_KB + a * 128 + ((c8 ^ (a & 7)) << 4)) = v[j];
+        for (int cp = 0; cp < R; ++cp) {
+          const int a = cp * rpc + r;
+          *reinterpret_cast<uint4*>(sA + kb * C_A_KB + a * 128 + ((c8 ^ (a & 7)) << 4)) = v[j];
+        }
       }
     }
+  }
+  for (int idx = t; idx < C_BM * per_row; idx += C_EPI * 32) {
+    const int a = idx / per_row, rem = idx - a * per_row;
+    if (a - (a / rpc) * rpc < M) continue;
+    const int kb = rem >> 3, c8 = rem & 7;
+    *reinterpret_cast<uint4*>(sA + kb * C_A_KB + a * 128 + ((c8 ^ (a & 7)) << 4)) =
+        make_uint4(0u, 0u, 0u, 0u);
   }
   {
     // one-hot row a (K-major, 32-byte swizzle: the two 16-byte halves of a row
@@ -176,6 +207,100 @@ __device__ void build_a_tile(const ChainParams& p, int M, int Fd, const int* fto
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Seed gates of the M rows of depth dd (frontier of Fd per request, A tile
+// built): row r's gate is a lower bound of its k-th value, the least of the
+// exact z at the request's k seed columns less the rounding allowance of the
+// tensor-core sum (seed.cuh); ordered keys, 0 where there is no seed. Every
+// epilogue thread takes (row, column) pairs; the parent embedding is read from
+// copy 0 of the row in the A tile.
+// Whether depth dd's seed data of every request fits the prefetch buffer.
+__device__ __forceinline__ bool seed_prefetchable(const ChainParams& p) {
+  return p.batch * p.k * p.r_pad * 2 <= 8192 && p.batch * p.k <= 256;
+}
+// Every epilogue thread: asynchronous copies of depth dd's seed data into pre
+// (layout above); seed_wait() before use.
+__device__ void seed_prefetch_depth(const ChainParams& p, int dd, uint8_t* pre) {
+  const int t = threadIdx.x - 64;
+  const int k = p.k, n16 = k * p.r_pad / 8;
+  for (int i = t; i < p.batch * n16; i += C_EPI * 32) {
+    const int b = i / n16, j = i - b * n16;
+    const size_t e0 = ((size_t)b * p.D + (dd - 1)) * k;
+    const uint32_t dst = smem_u32(pre + (size_t)i * 16);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
+                 "l"(p.swcol + e0 * p.r_pad + (size_t)j * 8) : "memory");
+  }
+  for (int i = t; i < 3 * p.batch * k; i += C_EPI * 32) {
+    const int w = i / (p.batch * k), bc = i - w * p.batch * k;
+    const int b = bc / k, c = bc - b * k;
+    const size_t e = ((size_t)b * p.D + (dd - 1)) * k + c;
+    const void* src = w == 0 ? static_cast<const void*>(p.scol + e)
+                             : w == 1 ? static_cast<const void*>(p.slval + e)
+                                      : static_cast<const void*>(p.swmax + e);
+    const uint32_t dst = smem_u32(pre + 8192 + (size_t)i * 4);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ void chain_seeds(const ChainParams& p, int dd, int M, int Fd, const uint8_t* sA,
+                            uint32_t* sseed, __nv_bfloat16* swc, const uint8_t* pre) {
+  const int t = threadIdx.x - 64;
+  for (int r = t; r < C_ROWS; r += C_EPI * 32) sseed[r] = 0xffffffffu;
+  const int k = p.k;
+  if (pre != nullptr) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    epi_sync();
+  }
+  const int32_t* pcol = reinterpret_cast<const int32_t*>(pre + 8192);
+  const float* plval = reinterpret_cast<const float*>(pre + 8192) + p.batch * k;
+  const float* pwmax = plval + p.batch * k;
+  for (int b = 0; b < p.batch; ++b) {
+    const size_t e0 = ((size_t)b * p.D + (dd - 1)) * k;
+    const __nv_bfloat16* wsrc;
+    if (pre != nullptr) {
+      wsrc = reinterpret_cast<const __nv_bfloat16*>(pre) + (size_t)b * k * p.r_pad;
+    } else {
+      // the request's k W columns for this depth, once per CTA (k x r_pad bf16)
+      const int n16 = k * p.r_pad / 8;
+      for (int i = t; i < n16; i += C_EPI * 32)
+        reinterpret_cast<uint4*>(swc)[i] = __ldg(reinterpret_cast<const uint4*>(p.swcol + e0 * p.r_pad) + i);
+      epi_sync();
+      wsrc = swc;
+    }
+    for (int pr = t; pr < Fd * k; pr += C_EPI * 32) {
+      const int i = pr / k, c = pr - i * k;
+      const int r = b * Fd + i;
+      const size_t e = e0 + c;
+      const int col = pre != nullptr ? pcol[b * k + c] : p.scol[e];
+      uint32_t key = 0u;
+      if (col >= 0) {
+        const __nv_bfloat16* wc = wsrc + (size_t)c * p.r_pad;
+        float dot = 0.f, e1 = 0.f;
+        for (int j0 = 0; j0 < p.r; j0 += 8) {
+          const int kb = j0 / C_BK, c8 = (j0 % C_BK) >> 3;
+          const uint4 ev = *reinterpret_cast<const uint4*>(sA + kb * C_A_KB + r * 128 + ((c8 ^ (r & 7)) << 4));
+          const uint4 wv = *reinterpret_cast<const uint4*>(wc + j0);
+          const float ee[8] = {bf16_lo(ev.x), bf16_hi(ev.x), bf16_lo(ev.y), bf16_hi(ev.y),
+                               bf16_lo(ev.z), bf16_hi(ev.z), bf16_lo(ev.w), bf16_hi(ev.w)};
+          const float ww[8] = {bf16_lo(wv.x), bf16_hi(wv.x), bf16_lo(wv.y), bf16_hi(wv.y),
+                               bf16_lo(wv.z), bf16_hi(wv.z), bf16_lo(wv.w), bf16_hi(wv.w)};
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            dot = fmaf(ee[q], ww[q], dot);
+            e1 += fabsf(ee[q]);
+          }
+        }
+        const float l = pre != nullptr ? plval[b * k + c] : p.slval[e];
+        const float wm = pre != nullptr ? pwmax[b * k + c] : p.swmax[e];
+        const float lo = (l + dot) - (fabsf(l) + e1 * wm) * kSeedSlack;
+        key = (lo == lo && lo != __int_as_float(0x7f800000) && lo > neg_inf()) ? f2ord(lo) : 0u;
+      }
+      atomicMin(&sseed[r], key);
+    }
+    if (pre == nullptr || b + 1 == p.batch) epi_sync();
+  }
+}
+
 template <int KMAX>
 __global__ void __launch_bounds__(C_THREADS, 1)
     pct_chain_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmL,
@@ -194,8 +319,10 @@ __global__ void __launch_bounds__(C_THREADS, 1)
   int* xi = reinterpret_cast<int*>(xv + C_ROWS * KMAX);      // [C_ROWS][KMAX]
   int* ftok = xi + C_ROWS * KMAX;                            // [C_ROWS] frontier tokens
   float* fs = reinterpret_cast<float*>(ftok + C_ROWS);       // [C_ROWS] frontier scores
-  int* misc = reinterpret_cast<int*>(fs + C_ROWS);           // [16]
-  uint64_t* full = reinterpret_cast<uint64_t*>(misc + 16);
+  uint32_t* sseed = reinterpret_cast<uint32_t*>(fs + C_ROWS); // [C_ROWS] seed gates (ordered keys)
+  int* misc = reinterpret_cast<int*>(sseed + C_ROWS);         // [16]
+  uint8_t* spre = reinterpret_cast<uint8_t*>(misc + 16);       // [C_PRE] (16-byte aligned)
+  uint64_t* full = reinterpret_cast<uint64_t*>(spre + C_PRE);
   uint64_t* empty = full + C_STAGES;
   uint64_t* lfull = empty + C_STAGES;    // [2]
   uint64_t* lempty = lfull + 2;          // [2]
@@ -240,6 +367,8 @@ __global__ void __launch_bounds__(C_THREADS, 1)
     }
     epi_sync();
     build_a_tile(p, p.batch, 1, ftok, sA, sOneHot);
+    epi_sync();
+    chain_seeds(p, 1, p.batch, 1, sA, sseed, reinterpret_cast<__nv_bfloat16*>(mkeys), nullptr);
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -261,6 +390,8 @@ __global__ void __launch_bounds__(C_THREADS, 1)
       uint32_t phase = 0;
       int git = 0;
       bool ok = true;
+      uint64_t keep;
+      asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep));
       for (int d = 1; d <= p.D && ok; ++d) {
         for (int it = 0; it < ntiles && ok; ++it, ++git) {
           const int n0 = (t_begin + it) * C_BN;
@@ -273,8 +404,8 @@ __global__ void __launch_bounds__(C_THREADS, 1)
             if (!wait_bar(&empty[stage], phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
             mbar_expect_tx(&full[stage], (uint32_t)C_B_STAGE);
             uint8_t* dst = sB + stage * C_B_STAGE;
-            tma_load_2d(dst, &tmB, n0, kb * C_BK, &full[stage]);
-            tma_load_2d(dst + C_B_STAGE / 2, &tmB, n0 + 64, kb * C_BK, &full[stage]);
+            tma_load_2d_keep(dst, &tmB, n0, kb * C_BK, &full[stage], keep);
+            tma_load_2d_keep(dst + C_B_STAGE / 2, &tmB, n0 + 64, kb * C_BK, &full[stage], keep);
             armed |= 1u << stage;
             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
             if (++stage == C_STAGES) { stage = 0; phase ^= 1u; }
@@ -346,7 +477,11 @@ __global__ void __launch_bounds__(C_THREADS, 1)
       float m = neg_inf(), s = 0.f;
       TopK<KMAX> tk;
       tk.init(k);
-      float gth = neg_inf();
+      if (d < p.D && seed_prefetchable(p)) seed_prefetch_depth(p, d + 1, spre);
+      const uint32_t seed_key = valid ? sseed[r] : 0u;
+      const float seed_gate =
+          (seed_key > f2ord(neg_inf()) && seed_key != 0xffffffffu) ? ord2f(seed_key) : neg_inf();
+      float gth = seed_gate;
       bool ok = true;
       for (int it = 0; it < ntiles; ++it, ++git) {
         const int buf = git & 1;
@@ -431,7 +566,7 @@ __global__ void __launch_bounds__(C_THREADS, 1)
         p.ms[((size_t)par * C_ROWS + r) * p.G + cta] = make_float2(m, s);
         // entries at or above the row's gate join the row's candidates
         const uint32_t g = *reinterpret_cast<volatile uint32_t*>(thr);
-        const float gate = g > f2ord(neg_inf()) ? ord2f(g) : neg_inf();
+        const float gate = fmaxf(g > f2ord(neg_inf()) ? ord2f(g) : neg_inf(), seed_gate);
         int n = 0;
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) n += (j < k && tk.v[j] != neg_inf() && tk.v[j] >= gate);
@@ -484,6 +619,14 @@ __global__ void __launch_bounds__(C_THREADS, 1)
           const int rr = r0 + q * C_EPI;
           ncand[q] = rr < M ? __ldcg(p.cand_cnt + (size_t)(d - 1) * C_ROWS + rr) : 0;
         }
+        // the first 32 candidates of each row are loaded with the counts
+        unsigned long long first[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int rr = r0 + q * C_EPI;
+          first[q] = (rr < M && lane < p.cap)
+                         ? __ldcg(p.cand + ((size_t)par * C_ROWS + rr) * p.cap + lane) : 0ull;
+        }
         for (int c0 = 0; c0 < p.G; c0 += 32 * PL) {
           float2 v[4][PL];
 #pragma unroll
@@ -501,14 +644,9 @@ __global__ void __launch_bounds__(C_THREADS, 1)
 #pragma unroll
             for (int i = 0; i < PL; ++i) lse_combine(lm[q], lsum[q], v[q][i].x, v[q][i].y);
         }
-        unsigned long long first[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int rr = r0 + q * C_EPI;
-          const int n = min(ncand[q], p.cap);
-          first[q] = (rr < M && lane < n)
-                         ? __ldcg(p.cand + ((size_t)par * C_ROWS + rr) * p.cap + lane) : 0ull;
-        }
+        for (int q = 0; q < 4; ++q)
+          if (lane >= min(ncand[q], p.cap)) first[q] = 0ull;   // entries past the count are stale
 #pragma unroll 1
         for (int q = 0; q < 4; ++q) {
           const int rr = r0 + q * C_EPI;
@@ -578,6 +716,8 @@ __global__ void __launch_bounds__(C_THREADS, 1)
         build_a_tile(p, p.batch * Fn, Fn, ftok, sA, sOneHot);
         epi_sync();
         if (threadIdx.x == 64) mbar_arrive(aready);
+        chain_seeds(p, d + 1, p.batch * Fn, Fn, sA, sseed, reinterpret_cast<__nv_bfloat16*>(mkeys),
+                    seed_prefetchable(p) ? spre : nullptr);
       }
     }
   }
@@ -665,7 +805,9 @@ size_t chain_workspace(const ChainShape& c) {
 
 cudaError_t launch_chain(const ChainShape& c, const void* L, const int32_t* anchor, const void* E,
                          const void* W, void* ws, int32_t* lvl_tok, int32_t* lvl_ppos, float* lvl_s,
-                         int32_t** err_out, int32_t* status, cudaStream_t s) {
+                         int32_t** err_out, int32_t* status, const int32_t* scol,
+                         const float* slval, const float* swmax, const void* swcol,
+                         cudaStream_t s) {
   const int G = chain_grid(c.V);
   const size_t cap = (size_t)G * c.k;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
@@ -691,6 +833,8 @@ cudaError_t launch_chain(const ChainShape& c, const void* L, const int32_t* anch
   p.err = reinterpret_cast<int32_t*>(w + (size_t)c.D * C_ROWS * 8 + (size_t)c.D * 4);
   p.lvl_tok = lvl_tok; p.lvl_ppos = lvl_ppos; p.lvl_s = lvl_s;
   p.status = status;
+  p.scol = scol; p.slval = slval; p.swmax = swmax;
+  p.swcol = static_cast<const __nv_bfloat16*>(swcol);
   *err_out = p.err;
   CUtensorMap tmB, tmL;
   if (!encode_2d_bf16(&tmB, W, (uint64_t)c.V, (uint64_t)c.r, 64, C_BK)) return cudaErrorInvalidValue;

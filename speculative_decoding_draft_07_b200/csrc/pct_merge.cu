@@ -102,9 +102,10 @@ __device__ __forceinline__ float merge_row(const Partials& part, size_t row, int
     lse_combine(m, s, m2, s2);
   }
   const float lse = (m == neg_inf()) ? neg_inf() : m + logf(s);
-#pragma unroll
-  for (int j = 0; j < KMAX; ++j) {
-    if (j >= k) break;
+  // rolled: this code runs once per launch, so its size (instruction fetch)
+  // costs more than the loop
+#pragma unroll 1
+  for (int j = 0; j < k; ++j) {
     float v = tk.v[0];
     int i = tk.i[0];
 #pragma unroll
@@ -282,11 +283,11 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
     // next depth's admission seeds for this request's new parents
     seed_prefetch_wait();   // also orders the Eg rows written above
     if (stash && vec)
-      seed_rows(kept, [&](int t) { return reinterpret_cast<const __nv_bfloat16*>(egs + t * a.r_pad); },
-                &seed_sm, a.seed.ks, a.r_pad, a.seed.thr + (size_t)b * Fn);
+      seed_rows<KMAX>(kept, [&](int t) { return reinterpret_cast<const __nv_bfloat16*>(egs + t * a.r_pad); },
+                      &seed_sm, a.seed.ks, a.r_pad, a.seed.thr + (size_t)b * Fn);
     else
-      seed_rows(kept, [&](int t) { return static_cast<const __nv_bfloat16*>(Eg) + ((size_t)b * Fn + t) * a.r_pad; },
-                &seed_sm, a.seed.ks, a.r_pad, a.seed.thr + (size_t)b * Fn);
+      seed_rows<KMAX>(kept, [&](int t) { return static_cast<const __nv_bfloat16*>(Eg) + ((size_t)b * Fn + t) * a.r_pad; },
+                      &seed_sm, a.seed.ks, a.r_pad, a.seed.thr + (size_t)b * Fn);
   }
 }
 

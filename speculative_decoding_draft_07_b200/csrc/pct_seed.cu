@@ -48,18 +48,51 @@ __device__ __forceinline__ float max8(const float (&x)[8]) {
   return fmaxf(fmax3(x[0], x[1], x[2]), fmax3(fmax3(x[3], x[4], x[5]), x[6], x[7]));
 }
 
-// One block per row of L ([rows][V], V % 8 == 0, 16-byte aligned rows).
-// Per row: cols[ks] distinct columns, best first (-1 where fewer than ks
-// thread winners exist), lval[ks] = L at them, wcol[ks][r_pad] = W[.][col]
-// (bf16, zero past r), wmax[ks] = max_j |W[j][col]|.
-template <typename TL>
+__device__ __forceinline__ uint32_t seed_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void seed_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// Descending bitonic sort of keys[0..P) by the block (P a power of two).
+__device__ void seed_sort_desc(unsigned long long* keys, int P) {
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const int t = threadIdx.x;
+      if (t < P / 2) {
+        const int lo = 2 * t - (t & (stride - 1));
+        const int hi = lo + stride;
+        const bool desc = ((lo & size) == 0);
+        const unsigned long long a = keys[lo], b = keys[hi];
+        if (desc ? (a < b) : (a > b)) { keys[lo] = b; keys[hi] = a; }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// One row of L ([rows][V], V % 8 == 0, 16-byte aligned rows) per block, or per
+// cluster of CL blocks when there are few rows (each block scans a fixed
+// 1/CL of the row; rank 0 merges the blocks' candidates through distributed
+// shared memory). Per row: cols[ks] distinct columns, best first (-1 where
+// fewer than ks thread winners exist), lval[ks] = L at them,
+// wcol[ks][r_pad] = W[.][col] (bf16, zero past r), wmax[ks] = max_j |W[j][col]|.
+template <typename TL, int CL>
 __global__ void __launch_bounds__(kSeedThreads) drafter_topk_kernel(
     int V, int ks, const TL* __restrict__ L, const __nv_bfloat16* __restrict__ W, int r,
     int r_pad, int32_t* __restrict__ cols, float* __restrict__ lval, float* __restrict__ wmax,
     __nv_bfloat16* __restrict__ wcol) {
   __shared__ unsigned long long keys[kSeedThreads];
-  const TL* row = L + (size_t)blockIdx.x * V;
-  const int G = V / 8;
+  const int rowi = (int)blockIdx.x / CL;
+  const uint32_t rank = CL > 1 ? seed_ctarank() : 0u;
+  const TL* row = L + (size_t)rowi * V;
+  const int Gall = V / 8;
+  const int gbeg = (int)((long long)Gall * rank / CL), gend = (int)((long long)Gall * (rank + 1) / CL);
+  row += (size_t)gbeg * 8;
+  const int G = gend - gbeg;
   float best = neg_inf();
   int bg = -1;
   constexpr int U = 8;   // 16-byte groups in flight per thread
@@ -105,28 +138,40 @@ __global__ void __launch_bounds__(kSeedThreads) drafter_topk_kernel(
     load8<TL>(row + (size_t)bg * 8, x);
 #pragma unroll
     for (int j = 7; j >= 0; --j)
-      if (x[j] == best) col = bg * 8 + j;
+      if (x[j] == best) col = (gbeg + bg) * 8 + j;
   }
   keys[threadIdx.x] =
       col >= 0 ? ((unsigned long long)f2ord(best) << 32) | (unsigned long long)(0xffffffffu - (uint32_t)col)
                : 0ull;
   __syncthreads();
   // descending bitonic sort of the 256 thread winners
-  for (int size = 2; size <= kSeedThreads; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      const int t = threadIdx.x;
-      if (t < kSeedThreads / 2) {
-        const int lo = 2 * t - (t & (stride - 1));
-        const int hi = lo + stride;
-        const bool desc = ((lo & size) == 0);
-        const unsigned long long a = keys[lo], b = keys[hi];
-        if (desc ? (a < b) : (a > b)) { keys[lo] = b; keys[hi] = a; }
+  seed_sort_desc(keys, kSeedThreads);
+  if constexpr (CL > 1) {
+    // rank 0 takes every block's ks best (distinct columns) and sorts them
+    __shared__ unsigned long long others[CL * kSeedMaxK];
+    seed_cluster_sync();
+    if (rank == 0) {
+      for (int i = threadIdx.x; i < (CL - 1) * ks; i += blockDim.x) {
+        const uint32_t src = 1u + (uint32_t)(i / ks);
+        uint32_t a;
+        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+                     : "=r"(a) : "r"((uint32_t)__cvta_generic_to_shared(keys + (i % ks))), "r"(src));
+        unsigned long long v;
+        asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(a) : "memory");
+        others[i] = v;
       }
-      __syncthreads();
     }
+    seed_cluster_sync();   // no block leaves while rank 0 reads its keys
+    if (rank != 0) return;
+    for (int i = threadIdx.x; i < (CL - 1) * ks; i += blockDim.x) keys[ks + i] = others[i];
+    int P = 1;
+    while (P < CL * ks) P <<= 1;
+    for (int i = CL * ks + threadIdx.x; i < P; i += blockDim.x) keys[i] = 0ull;
+    __syncthreads();
+    seed_sort_desc(keys, P);
   }
   // W columns of the seed columns: 16 threads per column (a half warp)
-  const size_t e0 = (size_t)blockIdx.x * ks;
+  const size_t e0 = (size_t)rowi * ks;
   const int c = threadIdx.x >> 4, sub = threadIdx.x & 15;
   const unsigned long long key = c < ks ? keys[c] : 0ull;
   const int cc = key ? (int)(0xffffffffu - (uint32_t)(key & 0xffffffffull)) : -1;
@@ -166,11 +211,34 @@ cudaError_t launch_drafter_topk(int rows, int V, int ks, int logits_dtype, const
   TraceScope t(s, "drafter_topk");
   const __nv_bfloat16* Wb = static_cast<const __nv_bfloat16*>(W);
   __nv_bfloat16* wc = static_cast<__nv_bfloat16*>(wcol);
+  // few rows: a cluster of 8 blocks per row keeps more of the GPU streaming
+  if ((long long)rows * 8 <= 2LL * num_sms() && V / 8 >= 8 * kSeedThreads) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)rows * 8);
+    cfg.blockDim = dim3(kSeedThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 8;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (logits_dtype == PCT_BF16)
+      e = cudaLaunchKernelEx(&cfg, drafter_topk_kernel<__nv_bfloat16, 8>, V, ks,
+                             static_cast<const __nv_bfloat16*>(L), Wb, r, r_pad, cols, lval, wmax, wc);
+    else
+      e = cudaLaunchKernelEx(&cfg, drafter_topk_kernel<float, 8>, V, ks, static_cast<const float*>(L),
+                             Wb, r, r_pad, cols, lval, wmax, wc);
+    if (e != cudaSuccess) (void)cudaGetLastError();
+    return e;
+  }
   if (logits_dtype == PCT_BF16)
-    drafter_topk_kernel<__nv_bfloat16><<<rows, kSeedThreads, 0, s>>>(
+    drafter_topk_kernel<__nv_bfloat16, 1><<<rows, kSeedThreads, 0, s>>>(
         V, ks, static_cast<const __nv_bfloat16*>(L), Wb, r, r_pad, cols, lval, wmax, wc);
   else
-    drafter_topk_kernel<float><<<rows, kSeedThreads, 0, s>>>(
+    drafter_topk_kernel<float, 1><<<rows, kSeedThreads, 0, s>>>(
         V, ks, static_cast<const float*>(L), Wb, r, r_pad, cols, lval, wmax, wc);
   return cudaGetLastError();
 }

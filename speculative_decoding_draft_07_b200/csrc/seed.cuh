@@ -77,14 +77,16 @@ __device__ __forceinline__ void seed_prefetch_wait() {
 // eg_row(t) (bf16, r_pad wide, zero padded, 16-byte aligned) written by this
 // block before a __syncthreads. sm holds the seed entry (seed_prefetch).
 // Writes thr[t] = ordered key of the row's bound, 0 when there is none.
-template <typename EgFn>
+// KS bounds ks at compile time (the unrolled per-column work).
+template <int KS = kSeedMaxK, typename EgFn>
 __device__ __forceinline__ void seed_rows(int nrows, EgFn eg_row, const SeedSmem* sm, int ks,
                                           int r_pad, uint32_t* __restrict__ thr) {
+  static_assert(KS <= kSeedMaxK, "seed columns");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const __nv_bfloat16* ws = sm->wcol;
   bool usable = true;
 #pragma unroll
-  for (int c = 0; c < kSeedMaxK; ++c) usable &= (c >= ks) || sm->cols[c] >= 0;
+  for (int c = 0; c < KS; ++c) usable &= (c >= ks) || sm->cols[c] >= 0;
   for (int t = warp; t < nrows; t += nw) {
     const int j0 = 8 * lane;
     float e[8];
@@ -99,9 +101,9 @@ __device__ __forceinline__ void seed_rows(int nrows, EgFn eg_row, const SeedSmem
     float e1 = 0.f;
 #pragma unroll
     for (int q = 0; q < 8; ++q) e1 += fabsf(e[q]);
-    float d[kSeedMaxK];
+    float d[KS];
 #pragma unroll
-    for (int c = 0; c < kSeedMaxK; ++c) {
+    for (int c = 0; c < KS; ++c) {
       d[c] = 0.f;
       if (c < ks && j0 < r_pad) {
         const uint4 w = *reinterpret_cast<const uint4*>(ws + c * r_pad + j0);
@@ -115,13 +117,13 @@ __device__ __forceinline__ void seed_rows(int nrows, EgFn eg_row, const SeedSmem
     for (int o = 16; o > 0; o >>= 1) {
       e1 += __shfl_xor_sync(0xffffffffu, e1, o);
 #pragma unroll
-      for (int c = 0; c < kSeedMaxK; ++c)
+      for (int c = 0; c < KS; ++c)
         if (c < ks) d[c] += __shfl_xor_sync(0xffffffffu, d[c], o);
     }
     float lo_min = __int_as_float(0x7f800000);
     bool finite = usable;
 #pragma unroll
-    for (int c = 0; c < kSeedMaxK; ++c) {
+    for (int c = 0; c < KS; ++c) {
       if (c < ks) {
         const float l = sm->lval[c];
         const float lo = (l + d[c]) - (fabsf(l) + e1 * sm->wmax[c]) * kSeedSlack;

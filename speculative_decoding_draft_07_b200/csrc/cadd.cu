@@ -425,33 +425,43 @@ __global__ __launch_bounds__(kRowThreads, 3) void cadd_rowpass_kernel(
 // ---------------------------------------------------------------------------
 // Segmented row pass (bf16 rows, 16-byte aligned, V % 8 == 0), two kernels.
 //  * cadd_seg_rowpass_kernel: every row is cut into S segments of at most
-//    kSegG * kSegThreads 16-byte groups, one kSegThreads-thread block per
-//    (row, segment), with no dependence between blocks. The segment is loaded
-//    straight into registers (kSegG 16-byte loads per thread in flight), folded
-//    into a partial log-sum-exp against each thread's own maximum, and filtered
-//    against the segment's own threshold lse_seg + ln(theta): since lse_seg <=
-//    lse of the row, that keeps a superset of the row's survivors. They go to
-//    the segment's slot of a buffer in global memory, with the partial and the
-//    count beside them.
+//    kSegPer 16-byte groups, one kSegThreads-thread block per (row, segment),
+//    with no dependence between blocks. The segment is loaded straight into
+//    registers (kSegG 16-byte loads per thread in flight) and folded into a
+//    partial log-sum-exp; a bitmap then marks each group whose maximum exceeds
+//    the segment's own threshold lse_seg + ln(theta). Since lse_seg <= lse of
+//    the row, the marks cover every value the row keeps.
 //  * cadd_seg_finish_kernel, one block per row: combines the S partials into
-//    the row's lse, keeps the buffered values above the exact threshold
-//    lse + ln(theta), sorts them (value desc, token asc) and writes the first
-//    n_max - 1; if a segment's slot overflowed (theta tiny) it selects them
-//    exactly over the row instead.
-// HBM sees every row once; the survivors add a few KB per row.
+//    the row's lse, reads the marked groups again, keeps their values above
+//    the exact threshold lse + ln(theta), sorts them (value desc, token asc)
+//    and writes the first n_max - 1; if too many groups are marked or too
+//    many values pass (theta tiny) it selects them exactly over the row.
+// HBM sees every row once; the bitmap adds 1 bit per 16 bytes, the marked
+// groups a few KB per row.
 
 constexpr int kSegThreads = 128;
+constexpr int kFinThreads = 128;          // finish kernel block
 constexpr int kSegG = 10;                 // 16-byte groups per thread (80 values)
-constexpr int kSegCap = 256;              // survivors buffered per segment
+constexpr int kSegBlocks = 6;             // resident blocks per SM (register bound)
+constexpr int kSegPer = kSegG * kSegThreads;   // 16-byte groups per segment
+constexpr int kSegWords = kSegPer / 32;         // bitmap words per segment
+static_assert(kSegThreads == 128 && kSegWords <= 64 && kSegWords % 8 == 0,
+              "bitmap words of a block: two sets of at most 64 threads, whole sectors");
 constexpr int kSegFinCap = 1024;          // exact survivors sorted per row (>= n_max - 1)
+constexpr int kFinGroups = 4096;          // marked groups listed per row
+constexpr int kFinBatch = 4;              // 16-byte loads in flight per thread (finish)
+constexpr int kFinMaxSegs = 256;          // segments per row that may use the tight bitmap
 constexpr float kSegMargin = 1e-3f;       // covers the rounding of lse_seg against lse
 
 // Segments of a row of V values (V % 8 == 0).
 __host__ __device__ __forceinline__ int seg_count(int V) {
   const int ngroups = V / 8;
-  const int per = kSegG * kSegThreads;
-  return ngroups < per ? 1 : (ngroups + per - 1) / per;
+  return ngroups <= kSegPer ? 1 : (ngroups + kSegPer - 1) / kSegPer;
 }
+// 32-bit words of a row's candidate-group bitmap: one bit per 16-byte group,
+// rounded up to whole 32-byte sectors (the row's last segment writes the
+// padding words, as zeros).
+__host__ __device__ __forceinline__ int seg_words(int V) { return ((V / 8 + 31) / 32 + 7) & ~7; }
 
 // Elementwise max of two packed bf16 pairs.
 __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
@@ -492,7 +502,7 @@ __device__ float2 block_lse_fixed(float m, float s, float2* wred) {
   for (int o = 16; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
   if (lane == 0) wred[warp] = make_float2(M, sc);
   __syncthreads();
-  constexpr int nw = kSegThreads / 32;
+  constexpr int nw = kFinThreads / 32;
   float BM = neg_inf();
 #pragma unroll
   for (int w = 0; w < nw; ++w) BM = fmaxf(BM, wred[w].x);
@@ -543,60 +553,64 @@ __device__ __forceinline__ float cadd_ln_theta_closed(const CaddParams& p, float
 struct SegWs {
   float* lnth;                 // [rows] filter offset ln(theta) - slack
   float2* part;                // [rows][S] partial (max, sum)
-  int* cnt;                    // [rows][S] survivors of the segment (may exceed kSegCap)
-  unsigned long long* surv;    // [rows][S][kSegCap] survivor keys
+  float* t2;                   // [rows][S] threshold of the tight bitmap
+  uint32_t* mask;              // [2][rows][seg_words(V)] candidate groups (loose, tight),
+                               // bit g % 32 of word g / 32
 };
 
-// One (row, segment) work item of the row pass.
+// One (row, segment) work item of the row pass: segment seg of a row covers
+// the 16-byte groups [seg * kSegPer, min(ngroups, (seg + 1) * kSegPer)), so
+// every segment but a row's last is full.
 struct SegItem {
   int row, seg, g0, ng;
 };
-__device__ __forceinline__ SegItem seg_item(int item, int V, int S) {
+__device__ __forceinline__ SegItem seg_item(int row, int seg, int V) {
   SegItem it;
-  it.row = item / S;
-  it.seg = item - it.row * S;
-  const int ngroups = V >> 3;
-  const int g_per = (ngroups + S - 1) / S;
-  it.g0 = min(ngroups, it.seg * g_per);
-  it.ng = min(ngroups, it.g0 + g_per) - it.g0;
+  it.row = row;
+  it.seg = seg;
+  it.g0 = seg * kSegPer;
+  it.ng = min(V >> 3, it.g0 + kSegPer) - it.g0;
   return it;
 }
 // The item's segment into registers: kSegG independent 16-byte loads per
-// thread (groups past the segment read as -inf).
+// thread (groups past a short segment read as -inf).
 __device__ __forceinline__ void seg_load(const __nv_bfloat16* __restrict__ L, int V,
                                          const SegItem& it, uint4 (&q)[kSegG]) {
   const uint4* src = reinterpret_cast<const uint4*>(L + (size_t)it.row * V) + it.g0;
+  if (it.ng == kSegPer) {
 #pragma unroll
-  for (int j = 0; j < kSegG; ++j) {
-    const int g = j * kSegThreads + threadIdx.x;
-    q[j] = g < it.ng ? ld_stream16(src + g)
-                     : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+    for (int j = 0; j < kSegG; ++j) q[j] = ld_stream16(src + j * kSegThreads + threadIdx.x);
+  } else {
+#pragma unroll
+    for (int j = 0; j < kSegG; ++j) {
+      const int g = j * kSegThreads + threadIdx.x;
+      q[j] = g < it.ng ? ld_stream16(src + g)
+                       : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+    }
   }
 }
 
 struct SegSmem {
   float2 wred[kSegThreads / 32];
-  uint4 stg_v[kSegThreads / 32][kSegG * 32];   // candidate groups, per warp
-  int stg_g[kSegThreads / 32][kSegG * 32];
-  int s_cnt;
+  uint32_t words[2][kSegWords];                // the block's bitmap words (loose, tight)
+  uint32_t tpair, tpair2;
 };
 
-// Everything after the loads for one item: partial log-sum-exp, the local
-// filter, and the item's slot in the workspace.
+// Everything after the loads for one item: the partial log-sum-exp, then two
+// bits per 16-byte group. The loose bit is set when the group's maximum
+// exceeds the segment's own threshold t = lse_seg + ln(theta): lse_seg <= lse
+// of the row, so these bits cover every value the row keeps. The tight bit
+// uses t2 = t + ln(S) - 1/2, about where the row's threshold falls when the S
+// segments hold similar mass; it covers the row's values whenever the row's
+// threshold is at least t2, which the finishing kernel checks per segment
+// before it tests only the groups one of the two bitmaps marks.
 __device__ __forceinline__ void seg_process(const CaddParams& p, const int64_t* __restrict__ ctx,
                                             const SegWs& w, const SegItem& it,
                                             const uint4 (&q)[kSegG], SegSmem& sm) {
-  float2* wred = sm.wred;
-  auto& stg_v = sm.stg_v;
-  auto& stg_g = sm.stg_g;
-  int& s_cnt = sm.s_cnt;
   const int S = seg_count(p.V);
   const int row = it.row, seg = it.seg, g0 = it.g0;
-  const int b = row / p.D;
-  const int K = p.n_max - 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) s_cnt = 0;
-  const float lnth = cadd_ln_theta_closed(p, (float)ctx[b]) - kThetaSlack;
+  const size_t slot = (size_t)row * S + seg;
 
   // packed maxima: gm[j] holds the larger of each half-pair of group j's words,
   // so max(lo, hi) of gm[j] is the group's maximum; their tree gives the thread's
@@ -609,119 +623,113 @@ __device__ __forceinline__ void seg_process(const CaddParams& p, const int64_t* 
   for (int j = 1; j < kSegG; ++j) tmx = bf16x2_max(tmx, gm[j]);
   const float m = fmaxf(bf16_lo(tmx), bf16_hi(tmx));
 
-  // partial log-sum-exp against the thread's own maximum (no rescaling), four
-  // independent scalar sums
+  // partial log-sum-exp against the thread's own maximum (no rescaling), two
+  // packed pairs of fp32 sums
   float s = 0.f;
   if (m != neg_inf()) {
     const float nmb = -m * kLog2e;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    float2 p0 = make_float2(0.f, 0.f), p1 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < kSegG; ++j) {
       const uint4 v = q[j];
-      a0 += ex2(fmaf(bf16_lo(v.x), kLog2e, nmb));
-      a1 += ex2(fmaf(bf16_hi(v.x), kLog2e, nmb));
-      a2 += ex2(fmaf(bf16_lo(v.y), kLog2e, nmb));
-      a3 += ex2(fmaf(bf16_hi(v.y), kLog2e, nmb));
-      a0 += ex2(fmaf(bf16_lo(v.z), kLog2e, nmb));
-      a1 += ex2(fmaf(bf16_hi(v.z), kLog2e, nmb));
-      a2 += ex2(fmaf(bf16_lo(v.w), kLog2e, nmb));
-      a3 += ex2(fmaf(bf16_hi(v.w), kLog2e, nmb));
+      const float2 l2 = make_float2(kLog2e, kLog2e), n2 = make_float2(nmb, nmb);
+      const float2 t0 = f2_fma(make_float2(bf16_lo(v.x), bf16_hi(v.x)), l2, n2);
+      const float2 t1 = f2_fma(make_float2(bf16_lo(v.y), bf16_hi(v.y)), l2, n2);
+      const float2 t2 = f2_fma(make_float2(bf16_lo(v.z), bf16_hi(v.z)), l2, n2);
+      const float2 t3 = f2_fma(make_float2(bf16_lo(v.w), bf16_hi(v.w)), l2, n2);
+      p0 = f2_add(p0, make_float2(ex2(t0.x), ex2(t0.y)));
+      p1 = f2_add(p1, make_float2(ex2(t1.x), ex2(t1.y)));
+      p0 = f2_add(p0, make_float2(ex2(t2.x), ex2(t2.y)));
+      p1 = f2_add(p1, make_float2(ex2(t3.x), ex2(t3.y)));
     }
-    s = (a0 + a1) + (a2 + a3);
+    s = (p0.x + p1.x) + (p0.y + p1.y);
   }
-  const float2 ps = block_lse_fixed(m, s, wred);
-  const float lse_seg = (ps.x == neg_inf()) ? neg_inf() : ps.x + logf(ps.y);
-  const float t_loc = (K <= 0) ? __int_as_float(0x7f800000) : lse_seg + lnth - kSegMargin;
 
-  // the segment's values above its own threshold, into its slot. A bf16 value
-  // exceeds t_loc exactly when it exceeds t_loc rounded down to bf16, so each
-  // group is tested with one packed compare of its maxima. Groups that pass are
-  // packed per warp into shared memory (ballot compaction, only in warps that
-  // have any), then tested value by value one group per lane, so the rare
-  // candidates cost no divergent passes over the registers.
-  const uint32_t tpair = bf16_pair_round_down(t_loc);
-  uint32_t hits = 0;
+  // the block's (max, sum) in a fixed order (lane tree, then warps in order);
+  // one thread turns it into the segment's threshold and publishes it with
+  // the partial, so the per-row scalar work runs once per block
+  {
+    float M = m;
 #pragma unroll
-  for (int j = 0; j < kSegG; ++j) hits |= (bf16x2_gt(gm[j], tpair) != 0u ? 1u : 0u) << j;
-  int nst = 0;   // staged groups of this warp
-  if (__any_sync(0xffffffffu, hits != 0u)) {
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float sc = (m == neg_inf()) ? 0.f : s * ex2((m - M) * kLog2e);
 #pragma unroll
-    for (int j = 0; j < kSegG; ++j) {
-      const bool c = (hits >> j) & 1u;
-      const unsigned ball = __ballot_sync(0xffffffffu, c);
-      if (c) {
-        const int at = nst + __popc(ball & ((1u << lane) - 1u));
-        stg_v[warp][at] = q[j];
-        stg_g[warp][at] = g0 + j * kSegThreads + threadIdx.x;
-      }
-      nst += __popc(ball);
-    }
-  }
-  __syncwarp();
-  const size_t slot = (size_t)row * S + seg;
-  unsigned long long* out = w.surv + slot * kSegCap;
-  for (int r0 = 0; r0 < nst; r0 += 32) {
-    const int i = r0 + lane;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    int g = 0;
-    uint32_t vm = 0;
-    if (i < nst) {
-      v = stg_v[warp][i];
-      g = stg_g[warp][i];
-      vm = (uint32_t)(bf16_lo(v.x) > t_loc) | (uint32_t)(bf16_hi(v.x) > t_loc) << 1 |
-           (uint32_t)(bf16_lo(v.y) > t_loc) << 2 | (uint32_t)(bf16_hi(v.y) > t_loc) << 3 |
-           (uint32_t)(bf16_lo(v.z) > t_loc) << 4 | (uint32_t)(bf16_hi(v.z) > t_loc) << 5 |
-           (uint32_t)(bf16_lo(v.w) > t_loc) << 6 | (uint32_t)(bf16_hi(v.w) > t_loc) << 7;
-    }
-    const int cnt = __popc(vm);
-    int incl = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int base = 0;
-    if (lane == 31 && incl > 0) base = atomicAdd(&s_cnt, incl);
-    int pos = __shfl_sync(0xffffffffu, base, 31) + (incl - cnt);
-    while (vm) {
-      const int e = __ffs(vm) - 1;
-      vm &= vm - 1;
-      const uint32_t wd = (e >> 1) == 0 ? v.x : (e >> 1) == 1 ? v.y : (e >> 1) == 2 ? v.z : v.w;
-      const float z = (e & 1) ? bf16_hi(wd) : bf16_lo(wd);
-      if (pos < kSegCap) out[pos] = cand_key(z, g * 8 + e);
-      ++pos;
-    }
+    for (int o = 16; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+    if (lane == 0) sm.wred[warp] = make_float2(M, sc);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    w.part[slot] = ps;
-    w.cnt[slot] = s_cnt;
+    constexpr int nw = kSegThreads / 32;
+    float BM = neg_inf();
+#pragma unroll
+    for (int i = 0; i < nw; ++i) BM = fmaxf(BM, sm.wred[i].x);
+    float BS = 0.f;
+#pragma unroll
+    for (int i = 0; i < nw; ++i) {
+      const float2 e = sm.wred[i];
+      if (e.x != neg_inf()) BS += e.y * ex2((e.x - BM) * kLog2e);
+    }
+    const float lnth = cadd_ln_theta_closed(p, (float)ctx[row / p.D]) - kThetaSlack;
+    const float lse_seg = (BM == neg_inf()) ? neg_inf() : BM + logf(BS);
+    const float t = (p.n_max <= 1) ? __int_as_float(0x7f800000) : lse_seg + lnth - kSegMargin;
+    const float t2 = t + (S > 1 ? logf((float)S) - 0.5f : 0.f);
+    sm.tpair = bf16_pair_round_down(t);
+    sm.tpair2 = bf16_pair_round_down(t2);
+    w.t2[slot] = t2;
+    w.part[slot] = make_float2(BM, BS);
     if (seg == 0) w.lnth[row] = lnth;
   }
+  __syncthreads();
+
+  // A bf16 value exceeds t exactly when it exceeds t rounded down to bf16, so
+  // a group is tested with one packed compare of its maximum. Group
+  // g0 + j * kSegThreads + 32 * warp + lane is bit lane of one word (kSegPer,
+  // kSegThreads and g0 are multiples of 32): the warp's ballot is the word.
+  // The block's kSegWords words of each bitmap are contiguous (and start on
+  // a 32-byte boundary): staged in shared memory, they leave in whole sectors.
+  const uint32_t tpair = sm.tpair, tpair2 = sm.tpair2;
+#pragma unroll
+  for (int j = 0; j < kSegG; ++j) {
+    const unsigned ball = __ballot_sync(0xffffffffu, bf16x2_gt(gm[j], tpair) != 0u);
+    const unsigned ball2 = __ballot_sync(0xffffffffu, bf16x2_gt(gm[j], tpair2) != 0u);
+    if (lane == 0) {
+      sm.words[0][j * (kSegThreads / 32) + warp] = ball;
+      sm.words[1][j * (kSegThreads / 32) + warp] = ball2;
+    }
+  }
+  __syncthreads();
+  const int nwr = seg_words(p.V);
+  const int w0 = g0 >> 5;
+  const int i = threadIdx.x & 63, which = threadIdx.x >> 6;
+  if (which < 2 && i < kSegWords && w0 + i < nwr)
+    w.mask[((size_t)which * p.batch * p.D + row) * nwr + w0 + i] = sm.words[which][i];
 }
 
-// One CTA per (row, segment) item, with the whole segment's loads in flight at
-// once (measured: persistent CTAs double-buffering two items in registers fit
-// half as many CTAs per SM and were slower, 109 us against 79 us at 960 rows).
-__global__ __launch_bounds__(kSegThreads, 6) void cadd_seg_rowpass_kernel(
+// One CTA per (row, segment) item (grid: rows x segments), with the whole
+// segment's loads in flight at once. Measured at 1024 rows of V = 151936:
+// persistent CTAs double-buffering two items in registers fit half as many
+// CTAs per SM, and segments staged in shared memory by bulk copies keep fewer
+// bytes in flight; both were slower.
+__global__ __launch_bounds__(kSegThreads, kSegBlocks) void cadd_seg_rowpass_kernel(
     CaddParams p, const __nv_bfloat16* __restrict__ L, const int64_t* __restrict__ ctx, SegWs w) {
   __shared__ SegSmem sm;
-  const SegItem it = seg_item(blockIdx.x, p.V, seg_count(p.V));
+  const SegItem it = seg_item(blockIdx.x, blockIdx.y, p.V);
   uint4 q[kSegG];
   seg_load(L, p.V, it, q);
   seg_process(p, ctx, w, it, q, sm);
 }
 
-__global__ __launch_bounds__(kSegThreads) void cadd_seg_finish_kernel(
+__global__ __launch_bounds__(kFinThreads) void cadd_seg_finish_kernel(
     CaddParams p, const __nv_bfloat16* __restrict__ L, const int64_t* __restrict__ ctx, SegWs w,
     float* __restrict__ row_lse, int32_t* __restrict__ cand_cnt, float* __restrict__ cand_q,
     int32_t* __restrict__ cand_tok, int32_t* __restrict__ status) {
-  __shared__ float2 wred[kSegThreads / 32];
+  __shared__ float2 wred[kFinThreads / 32];
   __shared__ unsigned long long keys[kSegFinCap];
-  __shared__ int cnt_sm[kSegThreads];
+  __shared__ int glist[kFinGroups];
   __shared__ int hist[256];
   __shared__ int sbuf[32];
-  __shared__ int s_n;
+  __shared__ int s_n, s_ng;
+  __shared__ bool use_tight[kFinMaxSegs];
 
   const int V = p.V;
   const int S = seg_count(V);
@@ -734,54 +742,71 @@ __global__ __launch_bounds__(kSegThreads) void cadd_seg_finish_kernel(
   // C(n) <= 0 for some n: reported once per request
   if (d == 0 && warp == 1) (void)cadd_ln_theta(p, (double)ctx[b], lane, true, &status[b]);
 
-  // one round trip for the partials, the counts and the threshold offset;
   // the row's lse from the partials in a fixed order
-  if (threadIdx.x == 0) s_n = 0;
+  if (threadIdx.x == 0) {
+    s_n = 0;
+    s_ng = 0;
+  }
   const float lnth = w.lnth[row];
   float pm = neg_inf(), pss = 0.f;
-  int over = 0;   // some segment's slot overflowed
-  for (int g = threadIdx.x; g < S; g += kSegThreads) {
+  for (int g = threadIdx.x; g < S; g += kFinThreads) {
     const float2 e = w.part[(size_t)row * S + g];
-    const int c = w.cnt[(size_t)row * S + g];
-    if (g < kSegThreads) cnt_sm[g] = c;
-    over |= c > kSegCap;
     lse_combine(pm, pss, e.x, e.y);
   }
-  const float2 rl = block_lse_fixed(pm, pss, wred);   // its barriers publish cnt_sm
+  const float2 rl = block_lse_fixed(pm, pss, wred);   // its barriers publish s_n, s_ng
   const float lse = (rl.x == neg_inf()) ? neg_inf() : rl.x + logf(rl.y);
   const float t = (K <= 0) ? __int_as_float(0x7f800000) : lse + lnth;
 
-  // buffered survivors above the exact threshold, kFinSegs segments per batch
-  // of loads (a window of kSegThreads segments' counts at a time)
-  int n = 0;
+  // per segment, the tight bitmap when the row's threshold is at least the
+  // segment's t2, else the loose one
+  for (int g = threadIdx.x; g < S; g += kFinThreads)
+    if (g < kFinMaxSegs) use_tight[g] = t >= w.t2[(size_t)row * S + g];
+  __syncthreads();
+
+  // the marked groups (list in shared memory), then their values above the
+  // row's threshold, kFinBatch independent 16-byte loads per thread at a time
+  int n = 0, over = 0;
   if (K > 0) {
-    constexpr int kFinSegs = 16;
-    constexpr int kSlots = kSegCap / kSegThreads;   // keys per thread per segment
-    for (int w0 = 0; w0 < S; w0 += kSegThreads) {
-      const int nwin = min(kSegThreads, S - w0);
-      if (w0 > 0) {
-        __syncthreads();
-        if (threadIdx.x < nwin) cnt_sm[threadIdx.x] = w.cnt[(size_t)row * S + w0 + threadIdx.x];
-        __syncthreads();
+    const int nw = seg_words(V);
+    const uint32_t* mrow = w.mask + (size_t)row * nw;
+    const uint32_t* mrow2 = mrow + (size_t)(p.batch * p.D) * nw;
+    for (int i = threadIdx.x; i < nw; i += kFinThreads) {
+      const int sg = i / (kSegPer / 32);
+      uint32_t bits = (sg < kFinMaxSegs && use_tight[sg]) ? mrow2[i] : mrow[i];
+      if (bits == 0u) continue;
+      const int at = atomicAdd(&s_ng, __popc(bits));
+      for (int k = at; bits; ++k) {
+        const int e = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (k < kFinGroups) glist[k] = 32 * i + e;
       }
-      for (int s0 = 0; s0 < nwin; s0 += kFinSegs) {
-        unsigned long long kk[kFinSegs * kSlots];
+    }
+    __syncthreads();
+    const int ng = s_ng;
+    if (ng > kFinGroups) {
+      over = 1;
+    } else {
+      const uint4* xg = reinterpret_cast<const uint4*>(x);
+      for (int i0 = 0; i0 < ng; i0 += kFinBatch * kFinThreads) {
+        uint4 v[kFinBatch];
+        int g[kFinBatch];
 #pragma unroll
-        for (int u = 0; u < kFinSegs; ++u) {
-          const int sg = s0 + u;
-          const int c = sg < nwin ? min(cnt_sm[sg], kSegCap) : 0;
-          const unsigned long long* in = w.surv + ((size_t)row * S + w0 + sg) * kSegCap;
-#pragma unroll
-          for (int h = 0; h < kSlots; ++h) {
-            const int j = h * kSegThreads + threadIdx.x;
-            kk[u * kSlots + h] = j < c ? in[j] : 0ull;
-          }
+        for (int u = 0; u < kFinBatch; ++u) {
+          const int i = i0 + u * kFinThreads + threadIdx.x;
+          g[u] = i < ng ? glist[i] : -1;
+          v[u] = g[u] >= 0 ? ld_stream16(xg + g[u])
+                           : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
         }
 #pragma unroll
-        for (int u = 0; u < kFinSegs * kSlots; ++u) {
-          if (kk[u] != 0ull && ord2f((unsigned)(kk[u] >> 32)) > t) {
-            const int at = atomicAdd(&s_n, 1);
-            if (at < kSegFinCap) keys[at] = kk[u];
+        for (int u = 0; u < kFinBatch; ++u) {
+          const uint32_t wd[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float z = (e & 1) ? bf16_hi(wd[e >> 1]) : bf16_lo(wd[e >> 1]);
+            if (z > t) {
+              const int at = atomicAdd(&s_n, 1);
+              if (at < kSegFinCap) keys[at] = cand_key(z, 8 * g[u] + e);
+            }
           }
         }
       }
@@ -804,13 +829,13 @@ __global__ __launch_bounds__(kSegThreads) void cadd_seg_finish_kernel(
   } else {
     int P = 1;
     while (P < n) P <<= 1;
-    for (int j = n + threadIdx.x; j < P; j += kSegThreads) keys[j] = 0ull;
+    for (int j = n + threadIdx.x; j < P; j += kFinThreads) keys[j] = 0ull;
     __syncthreads();
     bitonic_desc(keys, P);
   }
   const int keep = min(n, max(K, 0));
   const size_t cbase = (size_t)row * (size_t)max(K, 1);
-  for (int j = threadIdx.x; j < keep; j += kSegThreads) {
+  for (int j = threadIdx.x; j < keep; j += kFinThreads) {
     const unsigned long long kk = keys[j];
     cand_q[cbase + j] = ord2f((unsigned)(kk >> 32)) - lse;
     cand_tok[cbase + j] = (int)(~(unsigned)(kk & 0xffffffffu));
@@ -1004,7 +1029,7 @@ size_t cadd_seg_workspace(int batch, int D, int V, int dtype) {
   if (dtype != PCT_BF16 || V % 8 != 0) return 0;
   const size_t rows = (size_t)batch * D, slots = rows * seg_count(V);
   return align256(rows * sizeof(float)) + align256(slots * sizeof(float2)) +
-         align256(slots * sizeof(int)) + slots * kSegCap * sizeof(unsigned long long);
+         align256(slots * sizeof(float)) + 2 * rows * seg_words(V) * sizeof(uint32_t);
 }
 
 cudaError_t launch_cadd(const CaddParams& p, const void* L, const int32_t* anchor,
@@ -1020,18 +1045,19 @@ cudaError_t launch_cadd(const CaddParams& p, const void* L, const int32_t* ancho
     SegWs w;
     w.lnth = reinterpret_cast<float*>(c);              c += align256(rows * sizeof(float));
     w.part = reinterpret_cast<float2*>(c);             c += align256(slots * sizeof(float2));
-    w.cnt = reinterpret_cast<int*>(c);                 c += align256(slots * sizeof(int));
-    w.surv = reinterpret_cast<unsigned long long*>(c);
-    if (slots > 0x7fffffffu) return cudaErrorInvalidConfiguration;
+    w.t2 = reinterpret_cast<float*>(c);                c += align256(slots * sizeof(float));
+    w.mask = reinterpret_cast<uint32_t*>(c);
+    if (rows > 0x7fffffffu || seg_count(p.V) > 65535) return cudaErrorInvalidConfiguration;
     const __nv_bfloat16* Lb = static_cast<const __nv_bfloat16*>(L);
     {
       TraceScope t(s, "cadd_rowpass");
-      cadd_seg_rowpass_kernel<<<(unsigned)slots, kSegThreads, 0, s>>>(p, Lb, ctx, w);
+      const dim3 grid((unsigned)rows, (unsigned)seg_count(p.V));
+      cadd_seg_rowpass_kernel<<<grid, kSegThreads, 0, s>>>(p, Lb, ctx, w);
       cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
     TraceScope t(s, "cadd_finish");
-    cadd_seg_finish_kernel<<<(unsigned)rows, kSegThreads, 0, s>>>(p, Lb, ctx, w, row_lse, cand_cnt,
+    cadd_seg_finish_kernel<<<(unsigned)rows, kFinThreads, 0, s>>>(p, Lb, ctx, w, row_lse, cand_cnt,
                                                                  cand_q, cand_tok, status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -81,16 +81,20 @@ def test_workspace_grows_with_problem():
 
 def test_cadd_workspace_holds_the_segment_buffers():
     """bf16 rows with V % 8 == 0 take the segmented row pass: V / 8 16-byte groups per
-    row cut into ceil(groups / 1280) segments, each with a 256-key survivor slot, a
-    partial and a count; fp32 rows (single-block row pass) need none of it."""
+    row cut into ceil(groups / 1280) segments, each with a partial (max, sum) and a
+    tight threshold, and two bitmaps of one bit per group (rows padded to whole
+    32-byte sectors); fp32 rows (single-block row pass) need none of it."""
     def ws(dtype, V):
         c = pct.cadd_desc(64, 15, V, 512, dtype, 1.0, 2.0, 1e-4, 5e-3, 1e-5)
         return pct.lib().cadd_tree_grow_workspace(ctypes.byref(c))
     rows, V = 64 * 15, 151936
     S = -(-(V // 8) // 1280)
     assert S == 15
+    words = -(-(V // 8) // 32)
+    words += -words % 8
+    assert words == 600
     bf, f32 = ws(pct.PCT_BF16, V), ws(pct.PCT_F32, V)
-    assert bf - f32 >= rows * S * (256 * 8 + 8 + 4) + rows * 4
+    assert bf - f32 >= rows * S * (8 + 4) + rows * 4 + 2 * rows * words * 4
     assert ws(pct.PCT_BF16, V + 4) == ws(pct.PCT_F32, V + 4)     # V % 8 != 0: no segments
 
 

@@ -90,10 +90,9 @@ def test_stop_disabled_uses_exact_selection_fallback():
 
 
 def test_many_rows_mixed_overflow():
-    """240 rows, so each cluster of the row pass walks several rows through its two
-    segment buffers; flat rows (std 0.05) overflow the survivor buffer and take the
-    exact selection, sharply peaked rows (std 2, peak +40) keep one survivor, the two
-    interleaved at random in row order."""
+    """240 rows of one segment each: in flat rows (std 0.05) more values pass than the
+    finishing kernel sorts, so they take the exact selection; sharply peaked rows (std
+    2, peak +40) keep one survivor; the two interleaved at random in row order."""
     batch, D, V = 16, 15, 4096
     L = _sharp_logits(batch, D, V, seed=21, sigma=0.05, peak=(0.0, 0.5)).float()
     g = torch.Generator().manual_seed(22)
@@ -112,20 +111,32 @@ def test_many_rows_mixed_overflow():
 
 @pytest.mark.parametrize("seed", [51, 52])
 def test_multi_segment_rows(seed):
-    """V = 20488: each row splits into three segments of the row pass (854, 854 and 853
-    16-byte groups), so the survivors of every segment's own threshold are merged and
-    filtered again against the row's."""
-    batch, D, V = 8, 6, 20488
+    """V = 47784: each row splits into five segments of the row pass (four of 1280
+    16-byte groups and one of 853), each marking the groups above its own threshold
+    for the finishing kernel to test against the row's; the short last segment takes
+    the bounds-checked loads."""
+    batch, D, V = 8, 6, 47784
     L = _sharp_logits(batch, D, V, seed=seed, sigma=2.0, peak=(0.0, 6.0))
     ctx = np.array([512, 4096, 32768, 0, 100, 2000, 50000, 7])
     out, ref = _run(L, np.arange(batch), ctx, 128, COST, label=f"segments {seed}")
     assert ref.count.max() > 30
 
 
+@pytest.mark.parametrize("V", [20488, 183520])
+def test_segment_edges(V):
+    """V = 20488: a last segment of one 16-byte group; V = 183520: eighteen segments,
+    a bitmap of 717 words per row."""
+    batch, D = 2, 3
+    L = _sharp_logits(batch, D, V, seed=V % 97, sigma=2.0, peak=(0.0, 6.0))
+    ctx = np.array([4096, 32768])
+    out, ref = _run(L, np.arange(batch), ctx, 128, COST, label=f"segment edges V={V}")
+    assert ref.count.max() > 30
+
+
 def test_multi_segment_overflow():
-    """Three segments per row with flat rows whose segments overflow their slots (exact
-    selection over the row) interleaved with sharply peaked rows."""
-    batch, D, V = 6, 5, 20488
+    """Five segments per row: flat rows mark more groups than the finishing kernel lists
+    (exact selection over the row), interleaved with sharply peaked rows."""
+    batch, D, V = 6, 5, 47784
     L = _sharp_logits(batch, D, V, seed=41, sigma=0.05, peak=(0.0, 0.5)).float()
     g = torch.Generator().manual_seed(42)
     sharp = torch.rand((batch, D), generator=g) < 0.5

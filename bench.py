@@ -289,6 +289,30 @@ def timed(fn, steps, dev):
     return s.elapsed_time(e)
 
 
+def graph_step_ms(fn, steps, dev):
+    """Milliseconds per step of fn captured once in a CUDA graph and replayed
+    back to back (None if the capture fails)."""
+    try:
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        torch.cuda.synchronize(dev)
+        for _ in range(3):
+            g.replay()
+        ms = timed(g.replay, steps, dev) / steps
+        del g
+        return ms
+    except Exception:
+        torch.cuda.synchronize(dev)
+        return None
+
+
 def e2e_measure(rnd: Round, steps: int, dev):
     """Same metric through the public API with host buffers: every step copies its
     inputs from pinned host memory and reads its results back."""
@@ -729,9 +753,7 @@ def main():
         rnd.step()
     torch.cuda.synchronize(dev)
 
-    # timed region: per-kernel events on the launch stream, clocks sampled alongside
-    pct.trace_enable(True)
-    pct.trace_reset()
+    # timed region: the rounds back to back on the launch stream, clocks sampled alongside
     sampler = ClockSampler(gpu_ids(dev))
     sampler.start()
     time.sleep(0.3)
@@ -740,21 +762,36 @@ def main():
     torch.cuda.cudart().cudaProfilerStart()   # a profiler started with capture off records only this
     ms = timed(rnd.step, args.steps, dev)
     torch.cuda.cudart().cudaProfilerStop()
-    clocks = sampler.stop()
-    kernels = pct.trace_read()
-    pct.trace_enable(False)
-    ms = max_over_ranks(ms, dist, dev)
-    ms_step = ms / args.steps
-    value = world * 1e3 / ms_step
-
-    # the same round with the lazy verification walk (argmax of the walked rows only)
-    for _ in range(3):
-        rnd.step_lazy()
+    # the same rounds again with every kernel bracketed by two events on its
+    # stream: the per-kernel durations of the rooflines (the events lengthen
+    # the round, so the headline comes from the region above)
     pct.trace_enable(True)
     pct.trace_reset()
     if dist is not None:
         dist.barrier()
+    ms_traced = timed(rnd.step, args.steps, dev)
+    clocks = sampler.stop()
+    kernels = pct.trace_read()
+    pct.trace_enable(False)
+    ms = max_over_ranks(ms, dist, dev)
+    ms_traced = max_over_ranks(ms_traced, dist, dev)
+    ms_step = ms / args.steps
+    value = world * 1e3 / ms_step
+    graph_ms = graph_step_ms(rnd.step, args.steps, dev)
+    if graph_ms is not None:
+        graph_ms = max_over_ranks(graph_ms, dist, dev)
+
+    # the same round with the lazy verification walk (argmax of the walked rows only)
+    for _ in range(3):
+        rnd.step_lazy()
+    if dist is not None:
+        dist.barrier()
     ms_lazy = max_over_ranks(timed(rnd.step_lazy, args.steps, dev), dist, dev) / args.steps
+    pct.trace_enable(True)
+    pct.trace_reset()
+    if dist is not None:
+        dist.barrier()
+    timed(rnd.step_lazy, args.steps, dev)
     kl = pct.trace_read()
     pct.trace_enable(False)
     walked_rows = int((rnd.walk.accept_len.to(torch.int64) + 1).sum().item())
@@ -780,6 +817,10 @@ def main():
             "kernels": {n: {"launches_per_step": c / args.steps, "ms_per_step": t / args.steps}
                         for n, (c, t) in kernels.items()},
             "gpu_launches": launches,
+            "traced_ms_per_step": ms_traced / args.steps,
+            "cuda_graph": None if graph_ms is None else {
+                "value": world * 1e3 / graph_ms, "unit": "rounds/s", "ms_per_step": graph_ms,
+                "note": "the same round captured once in a CUDA graph and replayed"},
             "clocks": clocks,
             "e2e": {"value": world * 1e3 / e2e_ms, "unit": "rounds/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},

@@ -293,6 +293,8 @@ int32_t tree_verify_accept_noalloc(int32_t batch, int32_t n_stride, int32_t voca
  * and the elapsed time is accumulated per kernel name. Not for use inside
  * CUDA-graph capture.
  * ------------------------------------------------------------------------ */
+/* Enabling creates a pool of 16384 events up front, so a traced region spends
+ * no host time creating them (a region that records more creates the rest). */
 int32_t pct_trace_enable(int32_t on);   /* returns the previous setting */
 int32_t pct_trace_reset(void);
 /* Waits for the recorded events, then writes up to max_entries rows: a

@@ -49,6 +49,7 @@ struct Rec {
 std::vector<Rec> g_recs;
 std::vector<std::string> g_names;
 std::vector<cudaEvent_t> g_pool;
+constexpr size_t kTracePool = 16384;   // events kept ready while tracing is on
 
 cudaEvent_t take_event() {
   if (!g_pool.empty()) {
@@ -103,7 +104,7 @@ struct PctPlan {
   int S[66];
   int Mmax, M_pad;
   size_t max_ps;
-  size_t o_eg, o_ms, o_val, o_idx, o_ltok, o_lppos, o_ls, o_err, o_thr, o_scol, o_slval, o_swmax, o_swcol, total;
+  size_t o_eg, o_ms, o_val, o_idx, o_ltok, o_lppos, o_ls, o_err, o_thr, o_scol, o_slval, o_swmax, o_swcol, o_sdk, total;
   bool chain;             // small frontiers: one persistent launch (pct_chain.cu)
   size_t o_chain;
 };
@@ -159,6 +160,7 @@ int make_plan(const pct_build_desc* d, PctPlan* P) {
   P->o_slval = o; o += align_up(seeds * sizeof(float));
   P->o_swmax = o; o += align_up(seeds * sizeof(float));
   P->o_swcol = o; o += P->mdt == PCT_BF16 ? align_up(seeds * P->r_pad * 2) : 0;
+  P->o_sdk = o;   o += P->mdt == PCT_BF16 ? align_up(drafter_topk_scratch(P->batch * P->D)) : 0;
   P->chain = chain_eligible(chain_shape(*P));
   P->o_chain = o; o += P->chain ? align_up(chain_workspace(chain_shape(*P))) : 0;
   P->total = o;
@@ -219,6 +221,13 @@ int32_t pct_trace_enable(int32_t on) {
   std::lock_guard<std::mutex> lk(g_mu);
   const int32_t prev = g_on ? 1 : 0;
   g_on = on != 0;
+  // events are created here, not while a traced region launches: creating
+  // them there costs host time that delays the launches being timed
+  while (g_on && g_pool.size() + 2 * g_recs.size() < kTracePool) {
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) break;
+    g_pool.push_back(e);
+  }
   return prev;
 }
 
@@ -298,7 +307,7 @@ int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t*
     float* clval = reinterpret_cast<float*>(ws + P.o_slval);
     float* cwmax = reinterpret_cast<float*>(ws + P.o_swmax);
     PCT_CU(launch_drafter_topk(P.batch * P.D, P.V, P.k, P.ldt, L, W, P.r, P.r_pad, ccol, clval,
-                               cwmax, ws + P.o_swcol, s));
+                               cwmax, ws + P.o_swcol, ws + P.o_sdk, s));
     PCT_CU(launch_chain(chain_shape(P), L, anchor, E, W, ws + P.o_chain, ltok, lppos, ls, &cerr,
                         dev_status, ccol, clval, cwmax, ws + P.o_swcol, s));
     FinalArgs f;
@@ -335,7 +344,7 @@ int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t*
   };
   if (seeded)
     PCT_CU(launch_drafter_topk(P.batch * P.D, P.V, P.k, P.ldt, L, W, P.r, P.r_pad, scol, slval,
-                               swmax, swcol, s));
+                               swmax, swcol, ws + P.o_sdk, s));
   PCT_CU(launch_gather_rows(P.batch, anchor, P.V, P.r, P.r_pad, P.mdt, E, Eg, dev_status, 1,
                             seed_for(0), s));
   for (int d = 1; d <= P.D; ++d) {

@@ -110,10 +110,12 @@ cudaError_t launch_gather_rows(int rows, const int32_t* toks, int V, int r, int 
 
 // Seed data for every row of the logits [rows][V] (V % 8 == 0, bf16 W [r][V]):
 // the ks best columns (approximately), L at them, W's columns (bf16, zero
-// padded to r_pad) and their largest magnitude.
+// padded to r_pad) and their largest magnitude. scratch: drafter_topk_scratch
+// bytes (256-byte aligned), any contents.
+size_t drafter_topk_scratch(int rows);
 cudaError_t launch_drafter_topk(int rows, int V, int ks, int logits_dtype, const void* L,
                                 const void* W, int r, int r_pad, int32_t* cols, float* lval,
-                                float* wmax, void* wcol, cudaStream_t s);
+                                float* wmax, void* wcol, void* scratch, cudaStream_t s);
 
 struct MergeArgs {
   int batch, F_prev, F_new, k, beam, S, V, r, r_pad, markov_dtype, depth;

@@ -6,19 +6,23 @@
 // L_d is largest are the natural place to look for each parent's top-k. The
 // columns found here only seed a lower bound (the bound is exact whatever
 // columns are chosen), so the search need not be exact either: each thread
-// keeps the best 8-column group of its strided share of the row, the column of
-// that group's maximum is recovered with one reload, and the block keeps the
-// ks best of its 256 thread winners. One streaming pass over L (HBM bound).
+// keeps the best 8-column group of its strided share of a slice of the row,
+// the column of that group's maximum is recovered with one reload, each block
+// keeps the ks best of its 256 thread winners and the row's last block merges
+// the slices' picks. One streaming pass over L (HBM bound).
+#include <algorithm>
 #include <climits>
 
 #include "common.cuh"
 #include "internal.h"
 #include "seed.cuh"
+#include "select.cuh"
 
 namespace pct {
 namespace {
 
 constexpr int kSeedThreads = 256;
+constexpr int kSeedParts = 8;   // most slices of a row
 
 template <typename TL>
 __device__ __forceinline__ void load8(const TL* p, float (&x)[8]);
@@ -48,49 +52,28 @@ __device__ __forceinline__ float max8(const float (&x)[8]) {
   return fmaxf(fmax3(x[0], x[1], x[2]), fmax3(fmax3(x[3], x[4], x[5]), x[6], x[7]));
 }
 
-__device__ __forceinline__ uint32_t seed_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void seed_cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
-// Descending bitonic sort of keys[0..P) by the block (P a power of two).
-__device__ void seed_sort_desc(unsigned long long* keys, int P) {
-  for (int size = 2; size <= P; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      const int t = threadIdx.x;
-      if (t < P / 2) {
-        const int lo = 2 * t - (t & (stride - 1));
-        const int hi = lo + stride;
-        const bool desc = ((lo & size) == 0);
-        const unsigned long long a = keys[lo], b = keys[hi];
-        if (desc ? (a < b) : (a > b)) { keys[lo] = b; keys[hi] = a; }
-      }
-      __syncthreads();
-    }
-  }
-}
-
-// One row of L ([rows][V], V % 8 == 0, 16-byte aligned rows) per block, or per
-// cluster of CL blocks when there are few rows (each block scans a fixed
-// 1/CL of the row; rank 0 merges the blocks' candidates through distributed
-// shared memory). Per row: cols[ks] distinct columns, best first (-1 where
-// fewer than ks thread winners exist), lval[ks] = L at them,
-// wcol[ks][r_pad] = W[.][col] (bf16, zero past r), wmax[ks] = max_j |W[j][col]|.
-template <typename TL, int CL>
+// One row of L ([rows][V], V % 8 == 0, 16-byte aligned rows) cut into `parts`
+// fixed slices, one block per (row, slice): grid (rows, parts). Each block
+// keeps the ks best of its 256 thread winners; with more than one part it
+// writes them to pkeys and the last block of the row to finish (a counter per
+// row, reset by that block) merges the parts' keys. Nothing waits on another
+// block; the counters start at zero (the launcher clears them). Per row: cols[ks] distinct columns, best first (-1 where fewer than
+// ks thread winners exist), lval[ks] = L at them, wcol[ks][r_pad] = W[.][col]
+// (bf16, zero past r), wmax[ks] = max_j |W[j][col]|.
+template <typename TL>
 __global__ void __launch_bounds__(kSeedThreads) drafter_topk_kernel(
     int V, int ks, const TL* __restrict__ L, const __nv_bfloat16* __restrict__ W, int r,
     int r_pad, int32_t* __restrict__ cols, float* __restrict__ lval, float* __restrict__ wmax,
-    __nv_bfloat16* __restrict__ wcol) {
+    __nv_bfloat16* __restrict__ wcol, unsigned* __restrict__ cnt,
+    unsigned long long* __restrict__ pkeys) {
   __shared__ unsigned long long keys[kSeedThreads];
-  const int rowi = (int)blockIdx.x / CL;
-  const uint32_t rank = CL > 1 ? seed_ctarank() : 0u;
+  __shared__ int s_last;
+  const int rowi = (int)blockIdx.x;
+  const int parts = (int)gridDim.y, part = (int)blockIdx.y;
   const TL* row = L + (size_t)rowi * V;
   const int Gall = V / 8;
-  const int gbeg = (int)((long long)Gall * rank / CL), gend = (int)((long long)Gall * (rank + 1) / CL);
+  const int gbeg = (int)((long long)Gall * part / parts);
+  const int gend = (int)((long long)Gall * (part + 1) / parts);
   row += (size_t)gbeg * 8;
   const int G = gend - gbeg;
   float best = neg_inf();
@@ -140,35 +123,50 @@ __global__ void __launch_bounds__(kSeedThreads) drafter_topk_kernel(
     for (int j = 7; j >= 0; --j)
       if (x[j] == best) col = (gbeg + bg) * 8 + j;
   }
-  keys[threadIdx.x] =
-      col >= 0 ? ((unsigned long long)f2ord(best) << 32) | (unsigned long long)(0xffffffffu - (uint32_t)col)
-               : 0ull;
-  __syncthreads();
-  // descending bitonic sort of the 256 thread winners
-  seed_sort_desc(keys, kSeedThreads);
-  if constexpr (CL > 1) {
-    // rank 0 takes every block's ks best (distinct columns) and sorts them
-    __shared__ unsigned long long others[CL * kSeedMaxK];
-    seed_cluster_sync();
-    if (rank == 0) {
-      for (int i = threadIdx.x; i < (CL - 1) * ks; i += blockDim.x) {
-        const uint32_t src = 1u + (uint32_t)(i / ks);
-        uint32_t a;
-        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
-                     : "=r"(a) : "r"((uint32_t)__cvta_generic_to_shared(keys + (i % ks))), "r"(src));
-        unsigned long long v;
-        asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(a) : "memory");
-        others[i] = v;
-      }
-    }
-    seed_cluster_sync();   // no block leaves while rank 0 reads its keys
-    if (rank != 0) return;
-    for (int i = threadIdx.x; i < (CL - 1) * ks; i += blockDim.x) keys[ks + i] = others[i];
-    int P = 1;
-    while (P < CL * ks) P <<= 1;
-    for (int i = CL * ks + threadIdx.x; i < P; i += blockDim.x) keys[i] = 0ull;
+  // the 32 best of the 256 thread winners, sorted: a warp sort each, then
+  // warp 0 merges the eight sorted lists
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  {
+    unsigned long long x =
+        col >= 0 ? ((unsigned long long)f2ord(best) << 32) | (unsigned long long)(0xffffffffu - (uint32_t)col)
+                 : 0ull;
+    keys[threadIdx.x] = warp_sort_desc(x, lane);
     __syncthreads();
-    seed_sort_desc(keys, P);
+    if (warp == 0) {
+      unsigned long long acc = keys[lane];
+#pragma unroll
+      for (int w = 1; w < kSeedThreads / 32; ++w) acc = warp_merge_top(acc, keys[32 * w + 31 - lane], lane);
+      keys[lane] = acc;   // lanes read only keys[32..] after their first read
+    }
+    __syncthreads();
+  }
+  if (parts > 1) {
+    // publish this part's ks best; the row's last block to arrive merges
+    unsigned long long* pk = pkeys + (size_t)rowi * kSeedParts * kSeedMaxK;
+    if (threadIdx.x < ks) pk[part * kSeedMaxK + threadIdx.x] = keys[threadIdx.x];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(&cnt[rowi], 1u) == (unsigned)(parts - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (warp == 0) {
+      // every part's sorted list (ks <= 16 entries, padded with zero keys) in
+      // registers at once, then merged pairwise
+      unsigned long long b[kSeedParts];
+#pragma unroll
+      for (int q = 0; q < kSeedParts; ++q) {
+        const int j = q == 0 ? lane : 31 - lane;
+        b[q] = (q < parts && j < ks) ? __ldcg(pk + q * kSeedMaxK + j) : 0ull;
+      }
+      unsigned long long acc = b[0];
+#pragma unroll
+      for (int q = 1; q < kSeedParts; ++q)
+        if (q < parts) acc = warp_merge_top(acc, b[q], lane);
+      keys[lane] = acc;
+      if (lane == 0) cnt[rowi] = 0u;   // ready for the next launch
+    }
+    __syncthreads();
   }
   // W columns of the seed columns: 16 threads per column (a half warp)
   const size_t e0 = (size_t)rowi * ks;
@@ -202,44 +200,40 @@ __global__ void __launch_bounds__(kSeedThreads) drafter_topk_kernel(
 
 }  // namespace
 
+size_t drafter_topk_scratch(int rows) {
+  return ((size_t)rows * sizeof(unsigned) + 255) / 256 * 256 +
+         (size_t)rows * kSeedParts * kSeedMaxK * sizeof(unsigned long long);
+}
+
 cudaError_t launch_drafter_topk(int rows, int V, int ks, int logits_dtype, const void* L,
                                 const void* W, int r, int r_pad, int32_t* cols, float* lval,
-                                float* wmax, void* wcol, cudaStream_t s) {
+                                float* wmax, void* wcol, void* scratch, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   if (ks > kSeedMaxK || r > kSeedMaxR || r_pad > kSeedMaxR || r_pad % 8 != 0 || V % 8 != 0)
     return cudaErrorInvalidValue;
-  TraceScope t(s, "drafter_topk");
   const __nv_bfloat16* Wb = static_cast<const __nv_bfloat16*>(W);
   __nv_bfloat16* wc = static_cast<__nv_bfloat16*>(wcol);
-  // few rows: a cluster of 8 blocks per row keeps more of the GPU streaming
-  if ((long long)rows * 8 <= 2LL * num_sms() && V / 8 >= 8 * kSeedThreads) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)rows * 8);
-    cfg.blockDim = dim3(kSeedThreads);
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 8;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e;
-    if (logits_dtype == PCT_BF16)
-      e = cudaLaunchKernelEx(&cfg, drafter_topk_kernel<__nv_bfloat16, 8>, V, ks,
-                             static_cast<const __nv_bfloat16*>(L), Wb, r, r_pad, cols, lval, wmax, wc);
-    else
-      e = cudaLaunchKernelEx(&cfg, drafter_topk_kernel<float, 8>, V, ks, static_cast<const float*>(L),
-                             Wb, r, r_pad, cols, lval, wmax, wc);
-    if (e != cudaSuccess) (void)cudaGetLastError();
-    return e;
+  // parts of at least two passes of loads each (one when there are few rows),
+  // up to kSeedParts per row: the grid then covers the SMs in many short
+  // blocks instead of one wave of rows and a tail
+  const int passes = V / 8 / (8 * kSeedThreads);
+  int parts = std::max(1, std::min(kSeedParts, passes / 2));
+  if ((long long)rows * parts < 2LL * num_sms()) parts = std::max(1, std::min(kSeedParts, passes));
+  unsigned* cnt = static_cast<unsigned*>(scratch);
+  unsigned long long* pkeys = reinterpret_cast<unsigned long long*>(
+      static_cast<char*>(scratch) + ((size_t)rows * sizeof(unsigned) + 255) / 256 * 256);
+  if (parts > 1) {
+    cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(unsigned) * (size_t)rows, s);
+    if (e != cudaSuccess) return e;
   }
+  TraceScope t(s, "drafter_topk");
+  const dim3 grid((unsigned)rows, (unsigned)parts);
   if (logits_dtype == PCT_BF16)
-    drafter_topk_kernel<__nv_bfloat16, 1><<<rows, kSeedThreads, 0, s>>>(
-        V, ks, static_cast<const __nv_bfloat16*>(L), Wb, r, r_pad, cols, lval, wmax, wc);
+    drafter_topk_kernel<__nv_bfloat16><<<grid, kSeedThreads, 0, s>>>(
+        V, ks, static_cast<const __nv_bfloat16*>(L), Wb, r, r_pad, cols, lval, wmax, wc, cnt, pkeys);
   else
-    drafter_topk_kernel<float, 1><<<rows, kSeedThreads, 0, s>>>(
-        V, ks, static_cast<const float*>(L), Wb, r, r_pad, cols, lval, wmax, wc);
+    drafter_topk_kernel<float><<<grid, kSeedThreads, 0, s>>>(
+        V, ks, static_cast<const float*>(L), Wb, r, r_pad, cols, lval, wmax, wc, cnt, pkeys);
   return cudaGetLastError();
 }
 

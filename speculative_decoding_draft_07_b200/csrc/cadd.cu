@@ -234,6 +234,8 @@ __global__ __launch_bounds__(kRowThreads, 3) void cadd_rowpass_kernel(
     CaddParams p, const T* __restrict__ L, const int64_t* __restrict__ ctx,
     float* __restrict__ row_lse, int32_t* __restrict__ cand_cnt, float* __restrict__ cand_q,
     int32_t* __restrict__ cand_tok, int32_t* __restrict__ status) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ unsigned long long keys[kCap];
   __shared__ float sm[32], ss[32];
   __shared__ int sbuf[32];
@@ -712,6 +714,8 @@ __device__ __forceinline__ void seg_process(const CaddParams& p, const int64_t* 
 // bytes in flight; both were slower.
 __global__ __launch_bounds__(kSegThreads, kSegBlocks) void cadd_seg_rowpass_kernel(
     CaddParams p, const __nv_bfloat16* __restrict__ L, const int64_t* __restrict__ ctx, SegWs w) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ SegSmem sm;
   const SegItem it = seg_item(blockIdx.x, blockIdx.y, p.V);
   uint4 q[kSegG];
@@ -723,6 +727,8 @@ __global__ __launch_bounds__(kFinThreads) void cadd_seg_finish_kernel(
     CaddParams p, const __nv_bfloat16* __restrict__ L, const int64_t* __restrict__ ctx, SegWs w,
     float* __restrict__ row_lse, int32_t* __restrict__ cand_cnt, float* __restrict__ cand_q,
     int32_t* __restrict__ cand_tok, int32_t* __restrict__ status) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float2 wred[kFinThreads / 32];
   __shared__ unsigned long long keys[kSegFinCap];
   __shared__ int glist[kFinGroups];
@@ -861,6 +867,8 @@ __global__ __launch_bounds__(32) void cadd_bestfirst_kernel(
     const int32_t* __restrict__ cand_tok, int32_t* __restrict__ otok, int32_t* __restrict__ opar,
     int32_t* __restrict__ odep, float* __restrict__ oscore, int32_t* __restrict__ ocount,
     float* __restrict__ ophi, int32_t* __restrict__ status) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ unsigned long long pool[];          // [n_max + 1]
   const int nmax = p.n_max;
   const int D = p.D, K1 = max(nmax - 1, 1);
@@ -1052,25 +1060,25 @@ cudaError_t launch_cadd(const CaddParams& p, const void* L, const int32_t* ancho
     {
       TraceScope t(s, "cadd_rowpass");
       const dim3 grid((unsigned)rows, (unsigned)seg_count(p.V));
-      cadd_seg_rowpass_kernel<<<grid, kSegThreads, 0, s>>>(p, Lb, ctx, w);
-      cudaError_t e = cudaGetLastError();
+      cudaError_t e = launch_pdl(cadd_seg_rowpass_kernel, grid, dim3(kSegThreads), 0, s, 1, p, Lb,
+                                 ctx, w);
       if (e != cudaSuccess) return e;
     }
     TraceScope t(s, "cadd_finish");
-    cadd_seg_finish_kernel<<<(unsigned)rows, kFinThreads, 0, s>>>(p, Lb, ctx, w, row_lse, cand_cnt,
-                                                                 cand_q, cand_tok, status);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(cadd_seg_finish_kernel, dim3((unsigned)rows), dim3(kFinThreads), 0, s,
+                               1, p, Lb, ctx, w, row_lse, cand_cnt, cand_q, cand_tok, status);
     if (e != cudaSuccess) return e;
   } else {
     dim3 grid(p.D, p.batch);
     TraceScope t(s, "cadd_rowpass");
-    if (p.dtype == PCT_BF16)
-      cadd_rowpass_kernel<__nv_bfloat16><<<grid, kRowThreads, 0, s>>>(
-          p, static_cast<const __nv_bfloat16*>(L), ctx, row_lse, cand_cnt, cand_q, cand_tok, status);
-    else
-      cadd_rowpass_kernel<float><<<grid, kRowThreads, 0, s>>>(
-          p, static_cast<const float*>(L), ctx, row_lse, cand_cnt, cand_q, cand_tok, status);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e =
+        p.dtype == PCT_BF16
+            ? launch_pdl(cadd_rowpass_kernel<__nv_bfloat16>, grid, dim3(kRowThreads), 0, s, 1, p,
+                         static_cast<const __nv_bfloat16*>(L), ctx, row_lse, cand_cnt, cand_q,
+                         cand_tok, status)
+            : launch_pdl(cadd_rowpass_kernel<float>, grid, dim3(kRowThreads), 0, s, 1, p,
+                         static_cast<const float*>(L), ctx, row_lse, cand_cnt, cand_q, cand_tok,
+                         status);
     if (e != cudaSuccess) return e;
   }
   const size_t base = (size_t)(p.n_max + 1) * 8 + (size_t)p.n_max * 4 * 6;
@@ -1083,9 +1091,8 @@ cudaError_t launch_cadd(const CaddParams& p, const void* L, const int32_t* ancho
     if (e != cudaSuccess) return e;
   }
   TraceScope t(s, "cadd_bestfirst");
-  kern<<<p.batch, 32, smem, s>>>(p, anchor, ctx, cand_cnt, cand_q, cand_tok, tok, parent, depth,
-                                 score, count, phi, status);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(p.batch), dim3(32), smem, s, 1, p, anchor, ctx, cand_cnt, cand_q,
+                    cand_tok, tok, parent, depth, score, count, phi, status);
 }
 
 }  // namespace pct

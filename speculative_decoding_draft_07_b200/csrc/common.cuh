@@ -13,6 +13,49 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
 
+// Programmatic dependent launch. A kernel started by launch_pdl may begin while
+// the previous kernel of its stream is still running: pdl_wait() returns once
+// that kernel has completed and its memory operations are visible, so it comes
+// before every global-memory access of the kernel (reads and writes). Only
+// set-up that touches shared memory, TMEM or the kernel's parameters runs
+// before it. pdl_trigger() lets the next kernel start launching; its own
+// pdl_wait() still waits for this one to complete. Every launch_pdl kernel
+// calls pdl_wait() then pdl_trigger() at its start, so a dependent grid can
+// start only once every block of this grid is resident or done: its early
+// blocks never hold resources that blocks of this grid still need.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch with programmatic stream serialization allowed (and a cluster shape
+// when cluster_x > 1).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster_x > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  if (e != cudaSuccess) (void)cudaGetLastError();
+  return e;
+}
+
 // 2^x on the special-function unit (hardware approximation, flushes subnormal
 // results to zero; relative error a few ulp), used for the softmax sums.
 __device__ __forceinline__ float ex2(float x) {

@@ -36,6 +36,8 @@ template <typename TE>
 __global__ void gather_rows_kernel(int rows, const int32_t* __restrict__ toks, int V, int r,
                                    int r_pad, const TE* __restrict__ E, TE* __restrict__ Eg,
                                    int32_t* __restrict__ status, int status_div, SeedArgs seed) {
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.x;
   if (row >= rows) return;
   int t = toks[row];
@@ -141,6 +143,8 @@ __device__ void bitonic_desc_block(unsigned long long* keys, int P) {
 
 template <int KMAX, typename TE>
 __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ unsigned long long keys[kMaxCand];
   __shared__ unsigned long long ck[256];
   __shared__ float kept_s[256];
@@ -295,6 +299,8 @@ constexpr int kFinalThreads = 1024;
 constexpr int kMaxUnion = 4096;
 
 __global__ __launch_bounds__(kFinalThreads) void final_kernel(FinalArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float us[kMaxUnion];
   __shared__ int oidx[kMaxUnion];
   __shared__ int off[66];
@@ -402,6 +408,8 @@ template <int KMAX>
 __global__ void rows_finalize_kernel(int rows, int k, int S, Partials part, float* lse_out,
                                      int32_t* top_tok, float* top_logpi, const int32_t* err,
                                      int32_t* status, int n_par) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float wv[8][16];
   __shared__ int wi[8][16];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -429,14 +437,12 @@ cudaError_t launch_gather_rows(int rows, const int32_t* toks, int V, int r, int 
     return cudaErrorInvalidValue;
   TraceScope t(s, "gather_rows");
   if (markov_dtype == PCT_BF16)
-    gather_rows_kernel<__nv_bfloat16><<<rows, 128, 0, s>>>(
-        rows, toks, V, r, r_pad, static_cast<const __nv_bfloat16*>(E),
-        static_cast<__nv_bfloat16*>(Eg), status, status_div, seed);
-  else
-    gather_rows_kernel<float><<<rows, 128, 0, s>>>(rows, toks, V, r, r_pad,
-                                                   static_cast<const float*>(E),
-                                                   static_cast<float*>(Eg), status, status_div, seed);
-  return cudaGetLastError();
+    return launch_pdl(gather_rows_kernel<__nv_bfloat16>, dim3(rows), dim3(128), 0, s, 1, rows, toks,
+                      V, r, r_pad, static_cast<const __nv_bfloat16*>(E),
+                      static_cast<__nv_bfloat16*>(Eg), status, status_div, seed);
+  return launch_pdl(gather_rows_kernel<float>, dim3(rows), dim3(128), 0, s, 1, rows, toks, V, r,
+                    r_pad, static_cast<const float*>(E), static_cast<float*>(Eg), status,
+                    status_div, seed);
 }
 
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s) {
@@ -445,34 +451,33 @@ cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
   TraceScope t(s, "pct_merge_beam");
   const bool bf = a.markov_dtype == PCT_BF16;
-#define PCT_MERGE(KM)                                                                  \
-  (bf ? (merge_kernel<KM, __nv_bfloat16><<<a.batch, kMergeThreads, 0, s>>>(a), 0)      \
-      : (merge_kernel<KM, float><<<a.batch, kMergeThreads, 0, s>>>(a), 0))
-  if (a.k <= 4) PCT_MERGE(4);
-  else if (a.k <= 8) PCT_MERGE(8);
-  else PCT_MERGE(16);
+#define PCT_MERGE(KM)                                                                        \
+  (bf ? launch_pdl(merge_kernel<KM, __nv_bfloat16>, dim3(a.batch), dim3(kMergeThreads), 0, s, 1, a) \
+      : launch_pdl(merge_kernel<KM, float>, dim3(a.batch), dim3(kMergeThreads), 0, s, 1, a))
+  if (a.k <= 4) return PCT_MERGE(4);
+  if (a.k <= 8) return PCT_MERGE(8);
+  return PCT_MERGE(16);
 #undef PCT_MERGE
-  return cudaGetLastError();
 }
 
 cudaError_t launch_final(const FinalArgs& a, cudaStream_t s) {
   TraceScope t(s, "pct_global_topn");
-  final_kernel<<<a.batch, kFinalThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(final_kernel, dim3(a.batch), dim3(kFinalThreads), 0, s, 1, a);
 }
 
 cudaError_t launch_rows_finalize(int rows, int k, int S, Partials part, float* lse,
                                  int32_t* top_tok, float* top_logpi, const int32_t* err,
                                  int32_t* status, int n_par, cudaStream_t s) {
   TraceScope t(s, "pct_rows_finalize");
-  const int grid = (rows + 7) / 8;
+  const dim3 grid((rows + 7) / 8);
   if (k <= 4)
-    rows_finalize_kernel<4><<<grid, 256, 0, s>>>(rows, k, S, part, lse, top_tok, top_logpi, err, status, n_par);
-  else if (k <= 8)
-    rows_finalize_kernel<8><<<grid, 256, 0, s>>>(rows, k, S, part, lse, top_tok, top_logpi, err, status, n_par);
-  else
-    rows_finalize_kernel<16><<<grid, 256, 0, s>>>(rows, k, S, part, lse, top_tok, top_logpi, err, status, n_par);
-  return cudaGetLastError();
+    return launch_pdl(rows_finalize_kernel<4>, grid, dim3(256), 0, s, 1, rows, k, S, part, lse,
+                      top_tok, top_logpi, err, status, n_par);
+  if (k <= 8)
+    return launch_pdl(rows_finalize_kernel<8>, grid, dim3(256), 0, s, 1, rows, k, S, part, lse,
+                      top_tok, top_logpi, err, status, n_par);
+  return launch_pdl(rows_finalize_kernel<16>, grid, dim3(256), 0, s, 1, rows, k, S, part, lse,
+                    top_tok, top_logpi, err, status, n_par);
 }
 
 }  // namespace pct

@@ -66,6 +66,8 @@ __global__ void __launch_bounds__(kSeedThreads) drafter_topk_kernel(
     int r_pad, int32_t* __restrict__ cols, float* __restrict__ lval, float* __restrict__ wmax,
     __nv_bfloat16* __restrict__ wcol, unsigned* __restrict__ cnt,
     unsigned long long* __restrict__ pkeys) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ unsigned long long keys[kSeedThreads];
   __shared__ int s_last;
   const int rowi = (int)blockIdx.x;
@@ -229,12 +231,11 @@ cudaError_t launch_drafter_topk(int rows, int V, int ks, int logits_dtype, const
   TraceScope t(s, "drafter_topk");
   const dim3 grid((unsigned)rows, (unsigned)parts);
   if (logits_dtype == PCT_BF16)
-    drafter_topk_kernel<__nv_bfloat16><<<grid, kSeedThreads, 0, s>>>(
-        V, ks, static_cast<const __nv_bfloat16*>(L), Wb, r, r_pad, cols, lval, wmax, wc, cnt, pkeys);
-  else
-    drafter_topk_kernel<float><<<grid, kSeedThreads, 0, s>>>(
-        V, ks, static_cast<const float*>(L), Wb, r, r_pad, cols, lval, wmax, wc, cnt, pkeys);
-  return cudaGetLastError();
+    return launch_pdl(drafter_topk_kernel<__nv_bfloat16>, grid, dim3(kSeedThreads), 0, s, 1, V, ks,
+                      static_cast<const __nv_bfloat16*>(L), Wb, r, r_pad, cols, lval, wmax, wc, cnt,
+                      pkeys);
+  return launch_pdl(drafter_topk_kernel<float>, grid, dim3(kSeedThreads), 0, s, 1, V, ks,
+                    static_cast<const float*>(L), Wb, r, r_pad, cols, lval, wmax, wc, cnt, pkeys);
 }
 
 }  // namespace pct

@@ -20,6 +20,8 @@ constexpr int kSimtThreads = 128;
 
 template <typename TL, int KMAX>
 __global__ __launch_bounds__(kSimtThreads) void score_simt_kernel(ScoreArgs a, int cols_per_slice) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float eg[];                       // [r]
   __shared__ float rm[kSimtThreads / 32], rs[kSimtThreads / 32];
   __shared__ float bv[kSimtThreads / 32];
@@ -84,14 +86,17 @@ cudaError_t launch_score_simt(const ScoreArgs& a, cudaStream_t s) {
   dim3 grid(rows, a.S);
   const size_t smem = (size_t)a.r * sizeof(float);
   TraceScope t(s, "pct_score_simt");
-#define PCT_SIMT(TL, KM) score_simt_kernel<TL, KM><<<grid, kSimtThreads, smem, s>>>(a, cps)
+#define PCT_SIMT(TL, KM) \
+  launch_pdl(score_simt_kernel<TL, KM>, grid, dim3(kSimtThreads), smem, s, 1, a, cps)
   if (a.logits_dtype == PCT_BF16) {
-    if (a.k <= 4) PCT_SIMT(__nv_bfloat16, 4); else if (a.k <= 8) PCT_SIMT(__nv_bfloat16, 8); else PCT_SIMT(__nv_bfloat16, 16);
-  } else {
-    if (a.k <= 4) PCT_SIMT(float, 4); else if (a.k <= 8) PCT_SIMT(float, 8); else PCT_SIMT(float, 16);
+    if (a.k <= 4) return PCT_SIMT(__nv_bfloat16, 4);
+    if (a.k <= 8) return PCT_SIMT(__nv_bfloat16, 8);
+    return PCT_SIMT(__nv_bfloat16, 16);
   }
+  if (a.k <= 4) return PCT_SIMT(float, 4);
+  if (a.k <= 8) return PCT_SIMT(float, 8);
+  return PCT_SIMT(float, 16);
 #undef PCT_SIMT
-  return cudaGetLastError();
 }
 
 }  // namespace pct

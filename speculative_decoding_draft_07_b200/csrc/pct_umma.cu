@@ -174,6 +174,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();   // the set-up above touches only shared memory and TMEM
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -553,7 +555,8 @@ cudaError_t launch_score(const ScoreArgs& a, cudaStream_t s) {
       (void)cudaGetLastError();                                                                 \
       return e;                                                                                 \
     }                                                                                           \
-    kern<<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, tmL, p);                                   \
+    e = launch_pdl(kern, grid, dim3(THREADS), SMEM_BYTES, s, 1, tmA, tmB, tmL, p);             \
+    if (e != cudaSuccess) return e;                                                             \
   } while (0)
 #define PCT_UMMA_K(TL, LM)                                    \
   do {                                                        \

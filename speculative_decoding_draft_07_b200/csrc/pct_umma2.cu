@@ -204,6 +204,8 @@ __global__ void __launch_bounds__(P_THREADS, 1)
   cluster_sync_all();   // barriers, one-hot tiles and TMEM of both CTAs are ready
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();   // the set-up above touches only shared memory and TMEM
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -496,18 +498,7 @@ cudaError_t launch_score_pair(const ScoreArgs& a, cudaStream_t s) {
   } else {
     tmL = tmB;   // unused
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * a.S, mtiles);
-  cfg.blockDim = dim3(P_THREADS);
-  cfg.dynamicSmemBytes = P_SMEM;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  const dim3 grid(2 * a.S, mtiles);
   TraceScope t(s, "pct_score_pair");
 #define PCT_PAIR(TL, KM, FD)                                                                  \
   do {                                                                                        \
@@ -518,11 +509,8 @@ cudaError_t launch_score_pair(const ScoreArgs& a, cudaStream_t s) {
       (void)cudaGetLastError();                                                               \
       return e;                                                                               \
     }                                                                                         \
-    e = cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmL, p);                                     \
-    if (e != cudaSuccess) {                                                                   \
-      (void)cudaGetLastError(); /* leave no launch error behind for later calls */            \
-      return e;                                                                               \
-    }                                                                                         \
+    e = launch_pdl(kern, grid, dim3(P_THREADS), P_SMEM, s, 2, tmA, tmB, tmL, p);              \
+    if (e != cudaSuccess) return e;                                                           \
   } while (0)
 #define PCT_PAIR_K(TL, FD)                        \
   do {                                            \

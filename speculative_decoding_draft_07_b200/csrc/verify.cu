@@ -35,6 +35,8 @@ constexpr int kUnroll = 8;
 __global__ void ancestor_mask_kernel(int n_stride, int words, const int32_t* __restrict__ parent,
                                      const int32_t* __restrict__ count, uint32_t* __restrict__ mask,
                                      int32_t* __restrict__ status) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.y;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= n_stride * words) return;
@@ -198,6 +200,8 @@ __global__ __launch_bounds__(kVerifyThreads) void verify_kernel(
     const void* __restrict__ target, int32_t* __restrict__ argmax, int32_t* __restrict__ alen,
     int32_t* __restrict__ apath, int32_t* __restrict__ corr, int32_t* __restrict__ status,
     unsigned* __restrict__ arrive) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float sv[32];
   __shared__ int si[32];
   __shared__ int s_last;
@@ -279,8 +283,8 @@ cudaError_t launch_ancestor_mask(int batch, int n_stride, const int32_t* parent,
   const int total = n_stride * words;
   dim3 grid((total + 255) / 256, batch);
   TraceScope t(s, "ancestor_mask");
-  ancestor_mask_kernel<<<grid, 256, 0, s>>>(n_stride, words, parent, count, mask, status);
-  return cudaGetLastError();
+  return launch_pdl(ancestor_mask_kernel, grid, dim3(256), 0, s, 1, n_stride, words, parent, count,
+                    mask, status);
 }
 
 cudaError_t launch_verify(int batch, int n_stride, int vocab, int max_depth, const int32_t* tok,
@@ -290,22 +294,23 @@ cudaError_t launch_verify(int batch, int n_stride, int vocab, int max_depth, con
   dim3 grid(n_stride, batch);
   const bool aligned16 = (reinterpret_cast<uintptr_t>(target) & 15u) == 0;
   TraceScope t(s, "verify_argmax_walk");
+  cudaError_t e;
   if (dtype == PCT_BF16) {
     if (aligned16 && vocab % 8 == 0)
-      verify_kernel<0><<<grid, kVerifyThreads, 0, s>>>(n_stride, vocab, max_depth, tok, parent, count,
-                                                      target, argmax, alen, apath, corr, status, arrive);
+      e = launch_pdl(verify_kernel<0>, grid, dim3(kVerifyThreads), 0, s, 1, n_stride, vocab,
+                     max_depth, tok, parent, count, target, argmax, alen, apath, corr, status, arrive);
     else
-      verify_kernel<1><<<grid, kVerifyThreads, 0, s>>>(n_stride, vocab, max_depth, tok, parent, count,
-                                                      target, argmax, alen, apath, corr, status, arrive);
+      e = launch_pdl(verify_kernel<1>, grid, dim3(kVerifyThreads), 0, s, 1, n_stride, vocab,
+                     max_depth, tok, parent, count, target, argmax, alen, apath, corr, status, arrive);
   } else {
     if (aligned16 && vocab % 4 == 0)
-      verify_kernel<2><<<grid, kVerifyThreads, 0, s>>>(n_stride, vocab, max_depth, tok, parent, count,
-                                                      target, argmax, alen, apath, corr, status, arrive);
+      e = launch_pdl(verify_kernel<2>, grid, dim3(kVerifyThreads), 0, s, 1, n_stride, vocab,
+                     max_depth, tok, parent, count, target, argmax, alen, apath, corr, status, arrive);
     else
-      verify_kernel<3><<<grid, kVerifyThreads, 0, s>>>(n_stride, vocab, max_depth, tok, parent, count,
-                                                      target, argmax, alen, apath, corr, status, arrive);
+      e = launch_pdl(verify_kernel<3>, grid, dim3(kVerifyThreads), 0, s, 1, n_stride, vocab,
+                     max_depth, tok, parent, count, target, argmax, alen, apath, corr, status, arrive);
   }
-  return cudaGetLastError();
+  return e;
 }
 
 // ---------------------------------------------------------------------------
@@ -415,6 +420,8 @@ __global__ __launch_bounds__(kWalkThreads) void verify_walk_kernel(
     const int32_t* __restrict__ parent, const int32_t* __restrict__ count,
     const void* __restrict__ target, int32_t* __restrict__ argmax, int32_t* __restrict__ alen,
     int32_t* __restrict__ apath, int32_t* __restrict__ corr, int32_t* __restrict__ status) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int32_t walk_tree[];          // [n_stride] tokens, then [n_stride] parents
   __shared__ float part_v[2];
   __shared__ int part_i[2];
@@ -511,28 +518,19 @@ cudaError_t launch_verify_walk(int batch, int n_stride, int vocab, int max_depth
   int mode;
   if (dtype == PCT_BF16) mode = (aligned16 && vocab % 8 == 0) ? 0 : 1;
   else mode = (aligned16 && vocab % 4 == 0) ? 2 : 3;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(batch * kWalkCluster);
-  cfg.blockDim = dim3(kWalkThreads);
-  cfg.dynamicSmemBytes = 2 * sizeof(int32_t) * (size_t)n_stride;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kWalkCluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  const dim3 grid(batch * kWalkCluster), block(kWalkThreads);
+  const size_t smem = 2 * sizeof(int32_t) * (size_t)n_stride;
   TraceScope t(s, "verify_walk");
-  cudaError_t e;
+#define PCT_WALK(M)                                                                              \
+  launch_pdl(verify_walk_kernel<M>, grid, block, smem, s, kWalkCluster, n_stride, vocab,         \
+             max_depth, tok, parent, count, target, argmax, alen, apath, corr, status)
   switch (mode) {
-    case 0: e = cudaLaunchKernelEx(&cfg, verify_walk_kernel<0>, n_stride, vocab, max_depth, tok, parent, count, target, argmax, alen, apath, corr, status); break;
-    case 1: e = cudaLaunchKernelEx(&cfg, verify_walk_kernel<1>, n_stride, vocab, max_depth, tok, parent, count, target, argmax, alen, apath, corr, status); break;
-    case 2: e = cudaLaunchKernelEx(&cfg, verify_walk_kernel<2>, n_stride, vocab, max_depth, tok, parent, count, target, argmax, alen, apath, corr, status); break;
-    default: e = cudaLaunchKernelEx(&cfg, verify_walk_kernel<3>, n_stride, vocab, max_depth, tok, parent, count, target, argmax, alen, apath, corr, status); break;
+    case 0: return PCT_WALK(0);
+    case 1: return PCT_WALK(1);
+    case 2: return PCT_WALK(2);
+    default: return PCT_WALK(3);
   }
-  if (e != cudaSuccess) (void)cudaGetLastError();
-  return e;
+#undef PCT_WALK
 }
 
 }  // namespace pct

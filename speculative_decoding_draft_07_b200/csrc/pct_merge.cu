@@ -142,7 +142,7 @@ __device__ void bitonic_desc_block(unsigned long long* keys, int P) {
 }
 
 template <int KMAX, typename TE>
-__global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
+__global__ __launch_bounds__(kMergeThreads, 1) void merge_kernel(MergeArgs a) {
   pdl_wait();
   pdl_trigger();
   __shared__ unsigned long long keys[kMaxCand];
@@ -150,8 +150,12 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
   __shared__ float kept_s[256];
   __shared__ float wv[kMergeThreads / 32][32];
   __shared__ int wi[kMergeThreads / 32][32];
-  // the next depth's parent embeddings (bf16), kept for the seeds (up to 32 rows)
-  __shared__ __align__(16) uint16_t egs[32 * kSeedMaxR];
+  // the next depth's parent embeddings (bf16), kept for the seeds (up to 32
+  // rows; the row stride's extra 16 bytes keep the seed product's fragment
+  // loads free of bank conflicts)
+  constexpr int kEgsStride = kSeedMaxR + 8;
+  __shared__ __align__(16) uint16_t egs[kSeedMmaRows * kEgsStride];
+  __shared__ float e1s[kSeedMmaRows];
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = kMergeThreads / 32;
@@ -175,10 +179,10 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
     for (int i0 = 2 * warp; i0 < F; i0 += 2 * nwarps) {
       const int i = i0 + h;
       const size_t row = (size_t)b * F + min(i, F - 1);   // both halves take part in the shuffles
+      const float sp = (a.prev_s && i < F) ? a.prev_s[(size_t)b * a.prev_stride + i] : 0.f;
       const float lse = merge_row<KMAX, 16>(a.part, row, a.S, k, wv[warp] + 16 * h, wi[warp] + 16 * h);
       __syncwarp();
       if (i < F) {
-        const float sp = a.prev_s ? a.prev_s[(size_t)b * a.prev_stride + i] : 0.f;
         for (int j = gl; j < k; j += 16)
           keys[i * k + j] = beam_key(sp + (wv[warp][16 * h + j] - lse), i, wi[warp][16 * h + j]);
       }
@@ -187,9 +191,9 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
   } else {
     for (int i = warp; i < F; i += nwarps) {
       const size_t row = (size_t)b * F + i;
+      const float sp = a.prev_s ? a.prev_s[(size_t)b * a.prev_stride + i] : 0.f;
       const float lse = merge_row<KMAX, 32>(a.part, row, a.S, k, wv[warp], wi[warp]);
       __syncwarp();
-      const float sp = a.prev_s ? a.prev_s[(size_t)b * a.prev_stride + i] : 0.f;
       for (int j = lane; j < k; j += 32) keys[i * k + j] = beam_key(sp + (wv[warp][j] - lse), i, wi[warp][j]);
       __syncwarp();
     }
@@ -271,7 +275,7 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
       const uint4 val = j < rv ? reinterpret_cast<const uint4*>(E + (size_t)tok * a.r)[j]
                                : make_uint4(0u, 0u, 0u, 0u);
       reinterpret_cast<uint4*>(Eg + ((size_t)b * Fn + t) * a.r_pad)[j] = val;
-      if (stash) reinterpret_cast<uint4*>(egs + t * a.r_pad)[j] = val;
+      if (stash) reinterpret_cast<uint4*>(egs + t * kEgsStride)[j] = val;
     }
   } else {
     for (int idx = threadIdx.x; idx < kept * a.r_pad; idx += blockDim.x) {
@@ -286,8 +290,11 @@ __global__ __launch_bounds__(kMergeThreads) void merge_kernel(MergeArgs a) {
     if (a.seed.thr == nullptr) return;
     // next depth's admission seeds for this request's new parents
     seed_prefetch_wait();   // also orders the Eg rows written above
-    if (stash && vec)
-      seed_rows<KMAX>(kept, [&](int t) { return reinterpret_cast<const __nv_bfloat16*>(egs + t * a.r_pad); },
+    if (stash && vec && a.seed.ks <= kSeedMmaCols && a.r_pad % 16 == 0)
+      seed_rows_mma(kept, reinterpret_cast<const __nv_bfloat16*>(egs), kEgsStride, &seed_sm,
+                    a.seed.ks, a.r_pad, a.seed.thr + (size_t)b * Fn, e1s);
+    else if (stash && vec)
+      seed_rows<KMAX>(kept, [&](int t) { return reinterpret_cast<const __nv_bfloat16*>(egs + t * kEgsStride); },
                       &seed_sm, a.seed.ks, a.r_pad, a.seed.thr + (size_t)b * Fn);
     else
       seed_rows<KMAX>(kept, [&](int t) { return static_cast<const __nv_bfloat16*>(Eg) + ((size_t)b * Fn + t) * a.r_pad; },

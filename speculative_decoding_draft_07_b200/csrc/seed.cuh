@@ -135,4 +135,86 @@ __device__ __forceinline__ void seed_rows(int nrows, EgFn eg_row, const SeedSmem
   }
 }
 
+// The same bounds for up to 32 rows and ks <= 8 columns at once, for the merge
+// kernel (the rows are a request's new parents). The products E_t . W[:, c]
+// form a [32 x r_pad] x [r_pad x 8] matrix product, done with mma.sync
+// m16n8k16 (bf16 operands, fp32 accumulation) by warps 0 and 1, one 16-row
+// half each: far too small for the tcgen05 path's set-up to pay. The slack
+// covers any accumulation order, so the bound is the one seed_rows computes.
+// eg: shared memory, row t at eg + t * eg_stride (eg_stride >= r_pad, a
+// multiple of 8; rows nrows..31 may hold anything); r_pad % 16 == 0;
+// e1s: 32 floats of shared memory. Every thread of the block calls it.
+constexpr int kSeedMmaRows = 32;
+constexpr int kSeedMmaCols = 8;
+__device__ __forceinline__ uint32_t seed_lds32(const __nv_bfloat16* p) {
+  return *reinterpret_cast<const uint32_t*>(p);
+}
+__device__ __forceinline__ void seed_rows_mma(int nrows, const __nv_bfloat16* eg, int eg_stride, const SeedSmem* sm,
+                              int ks, int r_pad, uint32_t* __restrict__ thr, float* e1s) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  // sum_j |E_tj| per row: one warp per row at a time, 8 values per lane
+  for (int t = warp; t < nrows; t += nw) {
+    float e1 = 0.f;
+    for (int j0 = 8 * lane; j0 < r_pad; j0 += 256) {
+      const uint4 w = *reinterpret_cast<const uint4*>(eg + t * eg_stride + j0);
+      e1 += fabsf(bf16_lo(w.x)) + fabsf(bf16_hi(w.x)) + fabsf(bf16_lo(w.y)) + fabsf(bf16_hi(w.y)) +
+            fabsf(bf16_lo(w.z)) + fabsf(bf16_hi(w.z)) + fabsf(bf16_lo(w.w)) + fabsf(bf16_hi(w.w));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) e1 += __shfl_xor_sync(0xffffffffu, e1, o);
+    if (lane == 0) e1s[t] = e1;
+  }
+  __syncthreads();
+  if (warp >= 2) return;
+  // D = A . B with A = rows 16 * warp .. +15 of eg and B[k][n] = W[k][col n]
+  // (the seed columns, stored n-major: a column-major B fragment)
+  const int g = lane >> 2, q = lane & 3;
+  const __nv_bfloat16* a_lo = eg + (16 * warp + g) * eg_stride + 2 * q;
+  const __nv_bfloat16* a_hi = a_lo + 8 * eg_stride;
+  const __nv_bfloat16* bcol = sm->wcol + g * r_pad + 2 * q;   // column g (zero where g >= ks)
+  float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
+#pragma unroll 4
+  for (int k0 = 0; k0 < r_pad; k0 += 16) {
+    const uint32_t a0 = seed_lds32(a_lo + k0), a1 = seed_lds32(a_hi + k0);
+    const uint32_t a2 = seed_lds32(a_lo + k0 + 8), a3 = seed_lds32(a_hi + k0 + 8);
+    const uint32_t b0 = g < ks ? seed_lds32(bcol + k0) : 0u;
+    const uint32_t b1 = g < ks ? seed_lds32(bcol + k0 + 8) : 0u;
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c0), "+f"(c1), "+f"(c2), "+f"(c3)
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+  // lane (g, q) holds rows 16w + g (c0, c1) and 16w + g + 8 (c2, c3), columns
+  // 2q and 2q + 1; the row's minimum over columns is across the quad
+  bool usable = true;
+#pragma unroll
+  for (int c = 0; c < kSeedMmaCols; ++c) usable &= (c >= ks) || sm->cols[c] >= 0;
+  const float d[4] = {c0, c1, c2, c3};
+  float lo_min[2] = {__int_as_float(0x7f800000), __int_as_float(0x7f800000)};
+  bool fin[2] = {usable, usable};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int hrow = i >> 1, c = 2 * q + (i & 1);
+    const int t = 16 * warp + g + 8 * hrow;
+    if (c < ks && t < nrows) {
+      const float l = sm->lval[c];
+      const float lo = (l + d[i]) - (fabsf(l) + e1s[t] * sm->wmax[c]) * kSeedSlack;
+      fin[hrow] = fin[hrow] && (lo == lo) && lo != __int_as_float(0x7f800000);
+      lo_min[hrow] = fminf(lo_min[hrow], lo);
+    }
+  }
+#pragma unroll
+  for (int hrow = 0; hrow < 2; ++hrow) {
+#pragma unroll
+    for (int o = 1; o < 4; o <<= 1) {
+      lo_min[hrow] = fminf(lo_min[hrow], __shfl_xor_sync(0xffffffffu, lo_min[hrow], o));
+      fin[hrow] = __shfl_xor_sync(0xffffffffu, (int)fin[hrow], o) && fin[hrow];
+    }
+    const int t = 16 * warp + g + 8 * hrow;
+    if (q == 0 && t < nrows)
+      thr[t] = (fin[hrow] && lo_min[hrow] > neg_inf()) ? f2ord(lo_min[hrow]) : 0u;
+  }
+}
+
 }  // namespace pct

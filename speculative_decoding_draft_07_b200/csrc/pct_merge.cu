@@ -332,27 +332,35 @@ __global__ __launch_bounds__(kFinalThreads) void final_kernel(FinalArgs a) {
   }
   __syncthreads();
   // selection flag: rank under (score desc, depth asc, position asc) < N - 1;
-  // the flattened index u is depth-major, so (depth, position) order is u order
+  // the flattened index u is depth-major, so (depth, position) order is u order.
+  // The U x U comparisons are spread over every thread: S threads per u, each
+  // over a stride-S share of the v (counts added in shared memory)
   constexpr int PER = kMaxUnion / kFinalThreads;
+  const bool all_kept = U <= keepN;
+  if (!all_kept) {
+    for (int u = threadIdx.x; u < U; u += blockDim.x) oidx[u] = 0;
+    __syncthreads();
+    const int S = max(1, (int)blockDim.x / U);
+    for (int task = threadIdx.x; task < U * S; task += blockDim.x) {
+      const int u = task % U, part = task / U;
+      const float su = us[u];
+      int rank = 0;
+#pragma unroll 4
+      for (int v = part; v < U; v += S) rank += (us[v] > su) || (us[v] == su && v < u);
+      if (rank) atomicAdd(&oidx[u], rank);
+    }
+    __syncthreads();
+  }
   int flag[PER];
   int mine = 0;
 #pragma unroll
   for (int q = 0; q < PER; ++q) {
     const int u = threadIdx.x * PER + q;
-    int f = 0;
-    if (u < U) {
-      if (U <= keepN) {
-        f = 1;
-      } else {
-        const float su = us[u];
-        int rank = 0;
-        for (int v = 0; v < U; ++v) rank += (us[v] > su) || (us[v] == su && v < u);
-        f = rank < keepN;
-      }
-    }
+    const int f = u < U && (all_kept || oidx[u] < keepN);
     flag[q] = f;
     mine += f;
   }
+  __syncthreads();   // oidx is rewritten below
   // exclusive scan of the per-thread counts (threads own consecutive u)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int incl = mine;

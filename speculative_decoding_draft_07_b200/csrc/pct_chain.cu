@@ -267,8 +267,10 @@ __device__ void chain_seeds(const ChainParams& p, int dd, int M, int Fd, const u
       epi_sync();
       wsrc = swc;
     }
+    // column-major tasks: a warp's lanes share one or two W columns (broadcast
+    // reads) and take consecutive rows (conflict-free in the swizzled A tile)
     for (int pr = t; pr < Fd * k; pr += C_EPI * 32) {
-      const int i = pr / k, c = pr - i * k;
+      const int c = pr / Fd, i = pr - c * Fd;
       const int r = b * Fd + i;
       const size_t e = e0 + c;
       const int col = pre != nullptr ? pcol[b * k + c] : p.scol[e];

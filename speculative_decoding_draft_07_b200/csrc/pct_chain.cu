@@ -180,12 +180,13 @@ __device__ void build_a_tile(const ChainParams& p, int M, int Fd, const int* fto
       }
     }
   }
-  for (int idx = t; idx < C_BM * per_row; idx += C_EPI * 32) {
-    const int a = idx / per_row, rem = idx - a * per_row;
-    if (a - (a / rpc) * rpc < M) continue;
-    const int kb = rem >> 3, c8 = rem & 7;
-    *reinterpret_cast<uint4*>(sA + kb * C_A_KB + a * 128 + ((c8 ^ (a & 7)) << 4)) =
-        make_uint4(0u, 0u, 0u, 0u);
+  {
+    // thread t clears row t of the tile when it lies past M in its copy
+    const int a = t;
+    if (a - (a / rpc) * rpc >= M)
+      for (int rem = 0; rem < per_row; ++rem)
+        *reinterpret_cast<uint4*>(sA + (rem >> 3) * C_A_KB + a * 128 + (((rem & 7) ^ (a & 7)) << 4)) =
+            make_uint4(0u, 0u, 0u, 0u);
   }
   {
     // one-hot row a (K-major, 32-byte swizzle: the two 16-byte halves of a row
@@ -673,6 +674,11 @@ __global__ void __launch_bounds__(C_THREADS, 1)
             const float z = ord2f((uint32_t)(top >> 32));
             const int tok = (int)(~(uint32_t)top);
             mkeys[rr * k + lane] = top != 0ull ? beam_key(fs[rr] + (z - lse), i, tok) : 0ull;
+            // every candidate may enter the beam: its E row heads to L2 now, so
+            // the next A tile's gather finds it there
+            if (top != 0ull && (unsigned)tok < (unsigned)p.V && d < p.D)
+              for (int j = 0; j < p.r; j += 64)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(p.E + (size_t)tok * p.r + j));
           }
         }
       }

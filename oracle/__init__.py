@@ -23,6 +23,10 @@ pages define, written step by step in their order and notation:
   longest matching root path, append the target's own token.
 * ``verify.tree_ancestor_mask`` -- the self-plus-ancestors mask used for tree
   attention in the verification forward.
+* ``costfit.cost_fit`` -- the non-negative least-squares fit of the
+  verification cost C_v(n; l) = a + b l + c n + e n^2 to latency samples
+  (CaDDTree summary, "Method": convex, non-decreasing cost profiled offline),
+  by exhaustive search over the 16 free sets.
 
 Parity status of each function (what pins it, other than itself, is in
 ``tests/test_oracle_*.py``):
@@ -38,6 +42,8 @@ Parity status of each function (what pins it, other than itself, is in
   closed form on uniform marginals, and by Monte Carlo acceptance.
 * ``tree_verify_accept``: pinned by the pages' worked round (4 accepted drafts
   plus 1 correction) and by planted paths.
+* ``cost_fit``: pinned by SciPy's NNLS on random problems, by the KKT
+  conditions and by exact recovery of noiseless convex costs.
 * ``tree_ancestor_mask``: pinned by an independent transitive closure of the
   parent relation.
 * ``accept_sim``: Monte Carlo walks of greedy verification on a tree (the
@@ -50,6 +56,7 @@ from .pctree import pct_tree_build, PCTreeResult, score_parents
 from .caddtree import cadd_tree_grow, CaddResult, cadd_cost
 from .verify import tree_verify_accept, tree_ancestor_mask, VerifyResult
 from .accept_sim import accept_sim, philox4x32_10, uniform24
+from .costfit import cost_fit
 
 __all__ = [
     "decode_bf16", "to_f64", "row_log_softmax",
@@ -57,4 +64,5 @@ __all__ = [
     "cadd_tree_grow", "CaddResult", "cadd_cost",
     "tree_verify_accept", "tree_ancestor_mask", "VerifyResult",
     "accept_sim", "philox4x32_10", "uniform24",
+    "cost_fit",
 ]

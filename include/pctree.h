@@ -258,6 +258,28 @@ int32_t tree_accept_sim(int32_t batch, int32_t n_stride, int32_t max_depth, cons
                         int64_t* hist, int32_t* dev_status, void* cuda_stream);
 
 /* ------------------------------------------------------------------------ *
+ * cadd_cost_fit -- the verification cost model from latency samples.
+ * "Cost-Aware Diffusion Draft Trees for Speculative Decoding" (gist.science
+ * summary), "Method: CaDDTree": C_v is profiled offline as a convex function
+ * of the tree size n that does not decrease as n grows, and grows with the
+ * context length l. With C_v(n; l) = a + b l + c n + e n^2 that is the
+ * non-negative least-squares fit
+ *   min || X beta - t ||^2, beta = (a, b, c, e) >= 0, X = [1, l, n, n^2].
+ * One launch on the stream, fp64 arithmetic: the normal equations over the
+ * samples, then the least squares of each of the 16 free sets on unit-norm
+ * columns (a free set whose columns are linearly dependent is skipped), the
+ * feasible one with the smallest residual kept.
+ *   n, ell, lat: device float32 [m], the samples (tree size, context length,
+ *                measured latency)
+ *   out:         device float64 [5], written: a, b, c, e and the root mean
+ *                square residual
+ *   dev_status:  device int32 [1], PCT_DEV_BAD_COST when a sample is not finite
+ * m in 1..2^31 - 1; PCT_EINVAL for a null pointer or m out of range.
+ * ------------------------------------------------------------------------ */
+int32_t cadd_cost_fit(int64_t m, const float* n, const float* ell, const float* lat,
+                      double* out, int32_t* dev_status, void* cuda_stream);
+
+/* ------------------------------------------------------------------------ *
  * Allocation-free variant of tree_verify_accept. The pages have no
  * counterpart to this call: it exists for users of the library whose code
  * cannot allocate device memory -- for example a component inside a serving

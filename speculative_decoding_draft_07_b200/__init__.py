@@ -18,6 +18,8 @@ missing:
 * ``tree_accept_sim``    -- Monte Carlo acceptance length (tau) of a batch of
   trees against a synthetic target given per node.
 * ``pct_score_parents``  -- one depth of PCTree's batched parent scoring.
+* ``cadd_cost_fit``      -- the non-negative fit of CaDDTree's verification cost
+  C_v(n; l) = a + b l + c n + e n^2 to latency samples, on the device.
 * ``budget.ddtree_grow`` -- the fixed-budget best-first tree (CaDDTree's growth
   with the stop disabled), a call of ``cadd_tree_grow``.
 
@@ -25,8 +27,8 @@ Host-side tools around the hot path (numpy on the host, not part of it and not
 marshalling): ``budget`` (Phi curves, the greedy size and the sweep of fixed
 budgets against the adaptive size, evaluated from the library's trees),
 ``tau`` (Monte Carlo acceptance length of a round's trees against a synthetic
-target) and ``costfit`` (non-negative fit of C_v(n; l) = a + b l + c n + e n^2
-to latency samples).
+target) and ``costfit`` (the same non-negative fit as ``cadd_cost_fit``, by
+the Lawson-Hanson method on the host).
 """
 from ._lib import (  # noqa: F401
     BuildDesc, CaddDesc, PctError, TreeOut, VerifyOut, LIB_PATH, EXPORTED,
@@ -35,7 +37,7 @@ from ._lib import (  # noqa: F401
     DEV_BAD_COST, DEV_TIMEOUT,
     lib, build_desc, cadd_desc, pct_tree_build_workspace, pct_tree_build, pct_score_parents,
     cadd_tree_grow, tree_ancestor_mask, tree_verify_accept, tree_verify_walk, tree_accept_sim,
-    trace_enable, trace_reset,
+    cadd_cost_fit, trace_enable, trace_reset,
     trace_read, version,
 )
 from . import budget  # noqa: F401,E402

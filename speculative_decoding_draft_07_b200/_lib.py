@@ -30,6 +30,7 @@ EXPORTED = [
     "tree_verify_accept_workspace", "tree_verify_accept", "pct_trace_enable", "pct_trace_reset",
     "pct_trace_read", "pct_version", "tree_verify_accept_noalloc", "tree_verify_walk",
     "tree_accept_sim",
+    "cadd_cost_fit",
 ]
 
 
@@ -87,6 +88,7 @@ def lib() -> ctypes.CDLL:
         "tree_verify_walk": (i32, [i32, i32, i32, i32, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]),
         "tree_accept_sim": (i32, [i32, i32, i32, vp, vp, vp, ctypes.c_int64, ctypes.c_uint64, vp,
                                   vp, vp]),
+        "cadd_cost_fit": (i32, [ctypes.c_int64, vp, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -346,6 +348,21 @@ def tree_accept_sim(parent: torch.Tensor, count: torch.Tensor, p_child: torch.Te
                                  _stream(stream))
     _raise(code, "tree_accept_sim")
     return hist, status
+
+
+def cadd_cost_fit(n: torch.Tensor, ell: torch.Tensor, lat: torch.Tensor, stream=None):
+    """Non-negative fit of C_v(n; l) = a + b l + c n + e n^2 to latency samples:
+    (out float64 [5] = a, b, c, e, rms; status [1])."""
+    dev = n.device
+    m = n.numel()
+    _check(n, "n", dev, (m,), torch.float32)
+    _check(ell, "ell", dev, (m,), torch.float32)
+    _check(lat, "lat", dev, (m,), torch.float32)
+    out = torch.empty(5, dtype=torch.float64, device=dev)
+    status = torch.empty(1, dtype=torch.int32, device=dev)
+    code = lib().cadd_cost_fit(m, _p(n), _p(ell), _p(lat), _p(out), _p(status), _stream(stream))
+    _raise(code, "cadd_cost_fit")
+    return out, status
 
 
 def trace_enable(on: bool = True) -> bool:

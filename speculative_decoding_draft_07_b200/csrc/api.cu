@@ -568,4 +568,15 @@ int32_t tree_accept_sim(int32_t batch, int32_t n_stride, int32_t max_depth, cons
   return PCT_OK;
 }
 
+int32_t cadd_cost_fit(int64_t m, const float* n, const float* ell, const float* lat,
+                      double* out, int32_t* dev_status, void* cuda_stream) {
+  if (m < 1 || m > 2147483647LL) return PCT_EINVAL;
+  if (!n || !ell || !lat || !out || !dev_status) return PCT_EINVAL;
+  if (!device_ok()) return PCT_EDEVICE;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  PCT_CU(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s));
+  PCT_CU(launch_cost_fit((long long)m, n, ell, lat, out, dev_status, s));
+  return PCT_OK;
+}
+
 }  // extern "C"

@@ -108,6 +108,11 @@ cudaError_t launch_gather_rows(int rows, const int32_t* toks, int V, int r, int 
                                int markov_dtype, const void* E, void* Eg, int32_t* status,
                                int status_div, const SeedArgs& seed, cudaStream_t s);
 
+// Non-negative least-squares fit of C_v(n; l) = a + b l + c n + e n^2 to m
+// samples: out = (a, b, c, e, rms), device float64 [5] (cost_fit.cu).
+cudaError_t launch_cost_fit(long long m, const float* n, const float* ell, const float* lat,
+                            double* out, int32_t* status, cudaStream_t s);
+
 // Seed data for every row of the logits [rows][V] (V % 8 == 0, bf16 W [r][V]):
 // the ks best columns (approximately), L at them, W's columns (bf16, zero
 // padded to r_pad) and their largest magnitude. scratch: drafter_topk_scratch

@@ -2,11 +2,14 @@
 
 One step is one round of the whole hot path over a batch of 64 requests
 (synthetic inputs resident in HBM when the timed region starts):
-  * PCTree build: V = 151936, B = 16 (D = 15), bf16 logits ~ N(0, 2) + peak
-    U[0, 6], bf16 Markov rank 256, k = 8, beam 32, N = 256;
-  * CaDDTree grow on the same drafter logits (as marginals) with C_d = 1,
+  * CaDDTree grow on the drafter logits (as marginals) with C_d = 1,
     C_v = 2 + 1e-4 l + 5e-3 n + 1e-5 n^2, n_max = 512, context lengths cycling
-    through 512 / 4096 / 32768 over the requests;
+    through 512 / 4096 / 32768 over the requests; its row pass also writes each
+    row's top 8 tokens (cadd_tree_grow_topk);
+  * PCTree build on the same logits: V = 151936, B = 16 (D = 15), bf16 logits
+    ~ N(0, 2) + peak U[0, 6], bf16 Markov rank 256, k = 8, beam 32, N = 256,
+    its top-k gates seeded with those tokens (pct_tree_build_seeded), so the
+    logits are streamed once for both trees;
   * ancestor mask of the PCTree trees (256 x 256 bits per request);
   * greedy verification against bf16 target logits [64][256][V] (4.98 GB), with
     an argmax planted along a random root path of each tree.
@@ -56,9 +59,10 @@ def set_requests(n):
 
 def workload_config():
     return {
-        "workload": "full_round: PCTree build (V=151936, B=16, r=256, k=8, beam=32, N=256) + "
-                    "CaDDTree grow (n_max=512, l in {512,4096,32768}) + ancestor mask + "
-                    "greedy verify of bf16 target logits [64][256][V]",
+        "workload": "full_round: CaDDTree grow (n_max=512, l in {512,4096,32768}; also each "
+                    "row's top 8) + PCTree build seeded with them (V=151936, B=16, r=256, k=8, "
+                    "beam=32, N=256) + ancestor mask + greedy verify of bf16 target logits "
+                    "[64][256][V]",
         "requests": W.batch, "vocab": W.vocab, "block": W.block, "rank": W.rank, "k": W.k,
         "beam": W.beam, "n_nodes": W.n_nodes, "cadd_n_max": C.n_max,
         "l2": "inputs larger than L2: 4.98 GB of target logits stream through L2 each step",
@@ -114,8 +118,12 @@ def algorithmic_work():
         "verify_argmax_walk": {"bound": "hbm", "bytes": float(W.batch * W.n_nodes * W.vocab * 2)},
         # every marginal row read once (bf16)
         "cadd_rowpass": {"bound": "hbm", "bytes": float(W.batch * W.depth * W.vocab * 2)},
-        # admission seeds: every drafter logit row read once (bf16)
+        # admission seeds found by a pass over the drafter logits (the unseeded build)
         "drafter_topk": {"bound": "hbm", "bytes": float(W.batch * W.depth * W.vocab * 2)},
+        # admission seeds from given columns: k rows of W's transpose (r bf16
+        # values each, contiguous) per logits row read and written
+        "seed_columns": {"bound": "latency",
+                         "bytes": float(W.batch * W.depth * W.k * W.rank * 2 * 2)},
         # per-depth beam merge: a few KB per request and depth, bound by latency
         "pct_merge_beam": {"bound": "latency", "bytes": merge_bytes_per_step()},
     }
@@ -128,7 +136,8 @@ def source_sha(fname):
 
 KERNEL_SOURCE = {"pct_score_pair": "pct_umma2.cu", "pct_score_umma": "pct_umma.cu",
                  "verify_argmax_walk": "verify.cu", "cadd_rowpass": "cadd.cu",
-                 "drafter_topk": "pct_seed.cu", "pct_merge_beam": "pct_merge.cu"}
+                 "drafter_topk": "pct_seed.cu", "pct_merge_beam": "pct_merge.cu",
+                 "seed_columns": "pct_seed.cu"}
 
 
 def ncu_traffic(kernel):
@@ -229,8 +238,14 @@ class Round(RoundInputs):
         import speculative_decoding_draft_07_b200 as pct
         super().__init__(dev, seed_offset)
         self.pct = pct
-        self.tree = pct.pct_tree_build(self.L, self.anchor, self.E, self.W, W.k, W.beam, W.n_nodes)
-        self.cadd = pct.cadd_tree_grow(self.L, self.anchor, self.ctx, C.n_max, **COST)
+        # each row's top k from the CaDDTree's row pass seeds the PCTree's gates
+        self.seeds = torch.empty((W.batch, W.depth, W.k), dtype=torch.int32, device=dev)
+        # W transposed once (a model constant): the seeds' W columns are contiguous there
+        self.Wt = pct.markov_transpose(self.W)
+        self.cadd = pct.cadd_tree_grow(self.L, self.anchor, self.ctx, C.n_max, **COST,
+                                       top_tok=self.seeds)
+        self.tree = pct.pct_tree_build(self.L, self.anchor, self.E, self.W, W.k, W.beam, W.n_nodes,
+                                       seeds=self.seeds, Wt=self.Wt)
         torch.cuda.synchronize(dev)
         # target logits planted along this batch's trees (drawn once, outside timing)
         self.T = workloads.target_logits(W.batch, W.n_nodes, W.vocab,
@@ -259,20 +274,20 @@ class Round(RoundInputs):
         """The same round with the lazy verification walk in place of the full
         argmax (identical acceptance; only the walked rows are read)."""
         pct = self.pct
-        pct.pct_tree_build(self.L, self.anchor, self.E, self.W, W.k, W.beam, W.n_nodes,
-                           out=self.tree, workspace=self.ws_tree)
         pct.cadd_tree_grow(self.L, self.anchor, self.ctx, C.n_max, **COST, out=self.cadd,
-                           workspace=self.ws_cadd)
+                           workspace=self.ws_cadd, top_tok=self.seeds)
+        pct.pct_tree_build(self.L, self.anchor, self.E, self.W, W.k, W.beam, W.n_nodes,
+                           out=self.tree, workspace=self.ws_tree, seeds=self.seeds, Wt=self.Wt)
         pct.tree_ancestor_mask(self.tree.parent, self.tree.count, mask=self.mask, status=self.mstat)
         pct.tree_verify_walk(self.tree.tok, self.tree.parent, self.tree.count, self.T,
                              max_depth=W.depth, out=self.walk)
 
     def step(self):
         pct = self.pct
-        pct.pct_tree_build(self.L, self.anchor, self.E, self.W, W.k, W.beam, W.n_nodes,
-                           out=self.tree, workspace=self.ws_tree)
         pct.cadd_tree_grow(self.L, self.anchor, self.ctx, C.n_max, **COST, out=self.cadd,
-                           workspace=self.ws_cadd)
+                           workspace=self.ws_cadd, top_tok=self.seeds)
+        pct.pct_tree_build(self.L, self.anchor, self.E, self.W, W.k, W.beam, W.n_nodes,
+                           out=self.tree, workspace=self.ws_tree, seeds=self.seeds, Wt=self.Wt)
         pct.tree_ancestor_mask(self.tree.parent, self.tree.count, mask=self.mask, status=self.mstat)
         pct.tree_verify_accept(self.tree.tok, self.tree.parent, self.tree.count, self.T,
                                max_depth=W.depth, out=self.ver, workspace=self.ws_ver)
@@ -692,11 +707,17 @@ def run_stage(args):
     import speculative_decoding_draft_07_b200 as pct
     dev = torch.device("cuda", 0)
     rnd = RoundInputs(dev)
+    # as in the round: the CaDDTree's row pass writes each row's top k, which
+    # seed the PCTree (W's transpose for their columns)
+    seeds = torch.empty((W.batch, W.depth, W.k), dtype=torch.int32, device=dev)
+    pct.cadd_tree_grow(rnd.L, rnd.anchor, rnd.ctx, C.n_max, **COST, top_tok=seeds)
+    Wt = pct.markov_transpose(rnd.W)
     for _ in range(args.warmup + args.steps):
         if args.profile_stage == "pctree":
-            out = pct.pct_tree_build(rnd.L, rnd.anchor, rnd.E, rnd.W, W.k, W.beam, W.n_nodes)
+            out = pct.pct_tree_build(rnd.L, rnd.anchor, rnd.E, rnd.W, W.k, W.beam, W.n_nodes,
+                                     seeds=seeds, Wt=Wt)
         else:
-            out = pct.cadd_tree_grow(rnd.L, rnd.anchor, rnd.ctx, C.n_max, **COST)
+            out = pct.cadd_tree_grow(rnd.L, rnd.anchor, rnd.ctx, C.n_max, **COST, top_tok=seeds)
     torch.cuda.synchronize(dev)
     print(f"{args.profile_stage}: {args.warmup + args.steps} runs, status "
           f"{int(out.status.abs().sum().item())}, nodes {int(out.count.sum().item())}")

@@ -3,7 +3,10 @@
  *
  * One round of tree-based speculative decoding on one GPU:
  *   pct_tree_build      parent-conditioned drafting tree (PCTree)
+ *   pct_tree_build_seeded   the same, with each row's gate seeded by given columns
+ *   pct_markov_transpose    W transposed once per model, for the seeded build
  *   cadd_tree_grow      cost-aware best-first tree (CaDDTree)
+ *   cadd_tree_grow_topk the same, plus each logits row's top-k tokens
  *   tree_ancestor_mask  self-plus-ancestor bitmask for tree attention
  *   tree_verify_accept  greedy verification: argmax, accept walk, correction
  *   pct_score_parents   one depth of PCTree's batched parent scoring
@@ -115,6 +118,37 @@ int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t*
                        int32_t* depth, float* score, int32_t* count, int32_t* dev_status,
                        void* workspace, size_t ws_bytes, void* cuda_stream);
 
+/* pct_tree_build with the columns that seed each row's top-k gate given by
+ * the caller instead of found by a pass over L (the tensor-core path keeps a
+ * parent's value at or above a gate taken from the exact values at k columns
+ * of the row; any columns give a valid gate, large L_d columns a tight one).
+ *   Wt       NULL, or [V][r_pad] bf16: W transposed by pct_markov_transpose;
+ *            with it each seed's W column is one contiguous read instead of r
+ *            scattered ones (markov_dtype PCT_BF16, 16-byte aligned)
+ *   seed_tok [batch][D][k] int32  columns for row d-1 of request b; entries
+ *            outside [0, V) and repeats within a row are ignored (-1 = none)
+ * The result is identical to pct_tree_build's whatever the seeds; only the
+ * speed depends on them. With markov_dtype PCT_F32 the seeds are unused.
+ * Same workspace as pct_tree_build. PCT_EINVAL when seed_tok is NULL. A use:
+ * the top-k tokens cadd_tree_grow_topk writes for the same L (one pass over L
+ * then serves both trees). */
+int32_t pct_tree_build_seeded(const pct_build_desc* desc, const void* L, const int32_t* anchor,
+                              const void* E, const void* W, const void* Wt,
+                              const int32_t* seed_tok, int32_t* tok, int32_t* parent,
+                              int32_t* depth, float* score, int32_t* count, int32_t* dev_status,
+                              void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* r_pad of a Markov rank: rank rounded up to a multiple of 64 (0 if rank is
+ * outside 1..256). */
+int32_t pct_markov_rank_pad(int32_t rank);
+
+/* Wt [vocab][r_pad] bf16 = W [rank][vocab] bf16 transposed, zero in columns
+ * rank..r_pad-1 (r_pad = pct_markov_rank_pad(rank)). W is a model constant,
+ * so this runs once per model, not per round; the caller owns Wt
+ * (vocab * r_pad * 2 bytes, 16-byte aligned). vocab % 8 == 0, <= 2^22. */
+int32_t pct_markov_transpose(int32_t vocab, int32_t rank, const void* W, void* Wt,
+                             void* cuda_stream);
+
 /* One depth of PCTree's batched parent scoring (the step inside
  * pct_tree_build before the beam): for request b and each of its n_par
  * parents p with token parent_tok[b][p],
@@ -172,6 +206,22 @@ int32_t cadd_tree_grow(const cadd_desc* desc, const void* L, const int32_t* anch
                        const int64_t* ctx_len, int32_t* tok, int32_t* parent, int32_t* depth,
                        float* score, int32_t* count, float* phi, int32_t* dev_status,
                        void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* cadd_tree_grow, and in the same pass over L each row's top_k tokens:
+ *   top_k    1..32
+ *   top_tok  [batch][D][top_k] int32  the top_k largest logits of row d-1 of
+ *            request b, value descending, ties to the lower token id; -1 past V.
+ * The row pass already keeps every value above the row's CaDDTree threshold,
+ * sorted, and writes the head of that list; only rows with fewer than top_k
+ * such values are read again, by one more kernel that selects their top_k
+ * exactly. Values order as IEEE floats except that -0.0 ranks below +0.0.
+ * Same workspace as cadd_tree_grow. PCT_EINVAL when top_k is outside 1..32 or
+ * top_tok is NULL. */
+int32_t cadd_tree_grow_topk(const cadd_desc* desc, const void* L, const int32_t* anchor,
+                            const int64_t* ctx_len, int32_t top_k, int32_t* tok, int32_t* parent,
+                            int32_t* depth, float* score, int32_t* count, float* phi,
+                            int32_t* top_tok, int32_t* dev_status, void* workspace,
+                            size_t ws_bytes, void* cuda_stream);
 
 /* ------------------------------------------------------------------------ *
  * Ancestor bitmask for tree attention: bit j of row i (word j / 32, bit

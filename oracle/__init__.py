@@ -46,6 +46,10 @@ Parity status of each function (what pins it, other than itself, is in
   conditions and by exact recovery of noiseless convex costs.
 * ``tree_ancestor_mask``: pinned by an independent transitive closure of the
   parent relation.
+* ``row_topk``: each row's k largest logits (value descending, ties to the
+  lower token id), the order best-first growth takes a position's tokens in;
+  pinned by a brute-force pairwise count of the tokens that precede each token
+  and by the children the best-first tree takes at depth 1.
 * ``accept_sim``: Monte Carlo walks of greedy verification on a tree (the
   acceptance length tau); pinned by the generator's published known answers,
   by walks worked out by hand, and by the identity E[accepted] = Phi(T) when the
@@ -53,7 +57,7 @@ Parity status of each function (what pins it, other than itself, is in
 """
 from .numerics import decode_bf16, to_f64, row_log_softmax
 from .pctree import pct_tree_build, PCTreeResult, score_parents
-from .caddtree import cadd_tree_grow, CaddResult, cadd_cost
+from .caddtree import cadd_tree_grow, CaddResult, cadd_cost, row_topk
 from .verify import tree_verify_accept, tree_ancestor_mask, VerifyResult
 from .accept_sim import accept_sim, philox4x32_10, uniform24
 from .costfit import cost_fit

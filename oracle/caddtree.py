@@ -177,3 +177,23 @@ def cadd_tree_grow(L, anchor, ctx_len, n_max: int, C_d: float, a: float, b: floa
         reasons.append(why)
         fv.append(f)
     return CaddResult(tok, par, dep, score, count, phi, excl, reasons, fv)
+
+
+def row_topk(L, k: int):
+    """The k largest logits of every row of L [..][V] as token ids, value
+    descending, equal values to the lower token id; -1 past V.
+
+    Best-first growth expands a position's tokens in this order (the children
+    of a node at depth d are taken by decreasing q_d, i.e. by decreasing
+    logit), so these are the first k children any node of depth d - 1 offers.
+    Plain definition: a stable sort of the row by decreasing value.
+    """
+    L = np.asarray(L, dtype=np.float64)
+    V = L.shape[-1]
+    flat = L.reshape(-1, V)
+    out = np.full((flat.shape[0], k), -1, np.int32)
+    for i, row in enumerate(flat):
+        order = np.argsort(-row, kind="stable")[:k]
+        out[i, :len(order)] = order
+    return out.reshape(L.shape[:-1] + (k,))
+

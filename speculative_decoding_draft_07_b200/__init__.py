@@ -7,9 +7,11 @@ missing:
 
 * ``pct_tree_build``     -- PCTree: parent-conditioned drafting tree (batched
   Markov scoring on tcgen05 tensor cores, log-softmax, local top-k, beam,
-  global top-N).
+  global top-N). With ``seeds=`` (and optionally ``Wt=markov_transpose(W)``)
+  the gates of its top-k start from given columns instead of a pass over L.
 * ``cadd_tree_grow``     -- CaDDTree: cost-aware best-first tree with a greedy
-  stop on (1 + Phi) / (C_d + C_v(n; l)).
+  stop on (1 + Phi) / (C_d + C_v(n; l)). With ``top_tok=`` its row pass also
+  writes each row's top-k tokens, which can seed the PCTree on the same L.
 * ``tree_ancestor_mask`` -- self-plus-ancestor bitmask for tree attention.
 * ``tree_verify_accept`` -- greedy verification: argmax per node, accept walk,
   correction token.
@@ -37,7 +39,7 @@ from ._lib import (  # noqa: F401
     DEV_BAD_COST, DEV_TIMEOUT,
     lib, build_desc, cadd_desc, pct_tree_build_workspace, pct_tree_build, pct_score_parents,
     cadd_tree_grow, tree_ancestor_mask, tree_verify_accept, tree_verify_walk, tree_accept_sim,
-    cadd_cost_fit, trace_enable, trace_reset,
+    cadd_cost_fit, markov_transpose, trace_enable, trace_reset,
     trace_read, version,
 )
 from . import budget  # noqa: F401,E402

@@ -30,7 +30,8 @@ EXPORTED = [
     "tree_verify_accept_workspace", "tree_verify_accept", "pct_trace_enable", "pct_trace_reset",
     "pct_trace_read", "pct_version", "tree_verify_accept_noalloc", "tree_verify_walk",
     "tree_accept_sim",
-    "cadd_cost_fit",
+    "cadd_cost_fit", "pct_tree_build_seeded", "cadd_tree_grow_topk", "pct_markov_rank_pad",
+    "pct_markov_transpose",
 ]
 
 
@@ -89,6 +90,12 @@ def lib() -> ctypes.CDLL:
         "tree_accept_sim": (i32, [i32, i32, i32, vp, vp, vp, ctypes.c_int64, ctypes.c_uint64, vp,
                                   vp, vp]),
         "cadd_cost_fit": (i32, [ctypes.c_int64, vp, vp, vp, vp, vp, vp]),
+        "pct_tree_build_seeded": (i32, [bd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                        sz, vp]),
+        "pct_markov_rank_pad": (i32, [i32]),
+        "pct_markov_transpose": (i32, [i32, i32, vp, vp, vp]),
+        "cadd_tree_grow_topk": (i32, [cd, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                      sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -163,9 +170,15 @@ def pct_tree_build_workspace(desc: BuildDesc) -> int:
 
 def pct_tree_build(L: torch.Tensor, anchor: torch.Tensor, E: torch.Tensor, W: torch.Tensor,
                    k: int, beam: int, n_nodes: int, out: Optional[TreeOut] = None,
-                   workspace: Optional[torch.Tensor] = None, stream=None) -> TreeOut:
+                   workspace: Optional[torch.Tensor] = None, stream=None,
+                   seeds: Optional[torch.Tensor] = None,
+                   Wt: Optional[torch.Tensor] = None) -> TreeOut:
     """PCTree for a batch of requests. L [batch][D][V], anchor [batch] int32,
-    E [V][r], W [r][V]; returns node tables [batch][N] in canonical BFS order."""
+    E [V][r], W [r][V]; returns node tables [batch][N] in canonical BFS order.
+    seeds [batch][D][k] int32 (optional): the columns that seed each row's top-k
+    gate (pct_tree_build_seeded), e.g. cadd_tree_grow's top_tok for the same L;
+    the result does not depend on them. Wt (optional, with seeds):
+    markov_transpose(W), read for the seeds' W columns."""
     dev = L.device
     batch, D, V = L.shape
     r = E.shape[1]
@@ -183,11 +196,34 @@ def pct_tree_build(L: torch.Tensor, anchor: torch.Tensor, E: torch.Tensor, W: to
     if nbytes == 0:
         _raise(PCT_EINVAL, "pct_tree_build_workspace")
     ws, wsb = _workspace(nbytes, dev, workspace)
+    if seeds is not None:
+        _check(seeds, "seeds", dev, (batch, D, k), torch.int32)
+        if Wt is not None:
+            _check(Wt, "Wt", dev, (V, int(lib().pct_markov_rank_pad(r))), torch.bfloat16)
+        code = lib().pct_tree_build_seeded(ctypes.byref(desc), _p(L), _p(anchor), _p(E), _p(W),
+                                           _p(Wt), _p(seeds), _p(out.tok), _p(out.parent),
+                                           _p(out.depth), _p(out.score), _p(out.count),
+                                           _p(out.status), _p(ws), wsb, _stream(stream))
+        _raise(code, "pct_tree_build_seeded")
+        return out
     code = lib().pct_tree_build(ctypes.byref(desc), _p(L), _p(anchor), _p(E), _p(W), _p(out.tok),
                                 _p(out.parent), _p(out.depth), _p(out.score), _p(out.count),
                                 _p(out.status), _p(ws), wsb, _stream(stream))
     _raise(code, "pct_tree_build")
     return out
+
+
+def markov_transpose(W: torch.Tensor, stream=None) -> torch.Tensor:
+    """Wt [V][r_pad] bf16: W [r][V] bf16 transposed, zero past r (once per model)."""
+    dev = W.device
+    r, V = W.shape
+    _check(W, "W", dev, dtype=torch.bfloat16)
+    r_pad = int(lib().pct_markov_rank_pad(r))
+    if r_pad == 0:
+        _raise(PCT_EINVAL, "pct_markov_rank_pad")
+    Wt = torch.empty((V, r_pad), dtype=torch.bfloat16, device=dev)
+    _raise(lib().pct_markov_transpose(V, r, _p(W), _p(Wt), _stream(stream)), "pct_markov_transpose")
+    return Wt
 
 
 def pct_score_parents(L_row: torch.Tensor, parent_tok: torch.Tensor, E: torch.Tensor,
@@ -225,9 +261,11 @@ def cadd_desc(batch, depth, vocab, n_max, logits_dtype, C_d, a, b, c, e) -> Cadd
 def cadd_tree_grow(L: torch.Tensor, anchor: torch.Tensor, ctx_len: torch.Tensor, n_max: int,
                    C_d: float, a: float, b: float, c: float, e: float,
                    out: Optional[TreeOut] = None, workspace: Optional[torch.Tensor] = None,
-                   stream=None) -> TreeOut:
+                   stream=None, top_tok: Optional[torch.Tensor] = None) -> TreeOut:
     """CaDDTree for a batch of requests. L [batch][D][V] marginal logits,
-    anchor [batch] int32, ctx_len [batch] int64; node tables [batch][n_max]."""
+    anchor [batch] int32, ctx_len [batch] int64; node tables [batch][n_max].
+    top_tok [batch][D][top_k] int32 (optional, top_k 1..32): also written with
+    each row's top_k tokens by logit (value desc, token asc), cadd_tree_grow_topk."""
     dev = L.device
     batch, D, V = L.shape
     _check(L, "L", dev)
@@ -244,6 +282,16 @@ def cadd_tree_grow(L: torch.Tensor, anchor: torch.Tensor, ctx_len: torch.Tensor,
     if nbytes == 0:
         _raise(PCT_EINVAL, "cadd_tree_grow_workspace")
     ws, wsb = _workspace(nbytes, dev, workspace)
+    if top_tok is not None:
+        if top_tok.dim() != 3:
+            raise ValueError("top_tok must be [batch][D][top_k]")
+        _check(top_tok, "top_tok", dev, (batch, D, top_tok.shape[2]), torch.int32)
+        code = lib().cadd_tree_grow_topk(ctypes.byref(desc), _p(L), _p(anchor), _p(ctx_len),
+                                         int(top_tok.shape[2]), _p(out.tok), _p(out.parent),
+                                         _p(out.depth), _p(out.score), _p(out.count), _p(out.phi),
+                                         _p(top_tok), _p(out.status), _p(ws), wsb, _stream(stream))
+        _raise(code, "cadd_tree_grow_topk")
+        return out
     code = lib().cadd_tree_grow(ctypes.byref(desc), _p(L), _p(anchor), _p(ctx_len), _p(out.tok),
                                 _p(out.parent), _p(out.depth), _p(out.score), _p(out.count),
                                 _p(out.phi), _p(out.status), _p(ws), wsb, _stream(stream))

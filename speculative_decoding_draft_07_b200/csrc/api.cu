@@ -193,7 +193,7 @@ int check_cadd(const cadd_desc* d) {
   return PCT_OK;
 }
 struct CaddPlan {
-  size_t o_lse, o_cnt, o_q, o_tok, o_seg, seg_bytes, total;
+  size_t o_lse, o_cnt, o_q, o_tok, o_seg, seg_bytes, o_topk, total;
 };
 void cadd_plan(const cadd_desc* d, CaddPlan* P) {
   const size_t rows = (size_t)d->batch * d->depth;
@@ -205,6 +205,7 @@ void cadd_plan(const cadd_desc* d, CaddPlan* P) {
   P->o_tok = o; o += align_up(rows * K1 * sizeof(int32_t));
   P->seg_bytes = cadd_seg_workspace(d->batch, d->depth, d->vocab, d->logits_dtype);
   P->o_seg = o; o += align_up(P->seg_bytes);
+  P->o_topk = o; o += align_up(cadd_topk_workspace(rows));   // cadd_tree_grow_topk only
   P->total = o;
 }
 
@@ -275,10 +276,14 @@ size_t pct_tree_build_workspace(const pct_build_desc* desc) {
   return P.total;
 }
 
-int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t* anchor,
-                       const void* E, const void* W, int32_t* tok, int32_t* parent,
-                       int32_t* depth, float* score, int32_t* count, int32_t* dev_status,
-                       void* workspace, size_t ws_bytes, void* cuda_stream) {
+// seed_tok: null, or [batch][depth][k] columns that seed each row's top-k gate
+// in place of the drafter top-k pass; Wt: null, or W transposed (their W columns).
+static int32_t pct_build_impl(const pct_build_desc* desc, const void* L, const int32_t* anchor,
+                              const void* E, const void* W, const void* Wt,
+                              const int32_t* seed_tok, int32_t* tok,
+                              int32_t* parent, int32_t* depth, float* score, int32_t* count,
+                              int32_t* dev_status, void* workspace, size_t ws_bytes,
+                              void* cuda_stream) {
   PctPlan P;
   const int st = make_plan(desc, &P);
   if (st != PCT_OK) return st;
@@ -306,8 +311,12 @@ int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t*
     int32_t* ccol = reinterpret_cast<int32_t*>(ws + P.o_scol);
     float* clval = reinterpret_cast<float*>(ws + P.o_slval);
     float* cwmax = reinterpret_cast<float*>(ws + P.o_swmax);
-    PCT_CU(launch_drafter_topk(P.batch * P.D, P.V, P.k, P.ldt, L, W, P.r, P.r_pad, ccol, clval,
-                               cwmax, ws + P.o_swcol, ws + P.o_sdk, s));
+    if (seed_tok)
+      PCT_CU(launch_seed_columns(P.batch * P.D, P.V, P.k, P.ldt, L, W, Wt, P.r, P.r_pad,
+                                 seed_tok, ccol, clval, cwmax, ws + P.o_swcol, s));
+    else
+      PCT_CU(launch_drafter_topk(P.batch * P.D, P.V, P.k, P.ldt, L, W, P.r, P.r_pad, ccol, clval,
+                                 cwmax, ws + P.o_swcol, ws + P.o_sdk, s));
     PCT_CU(launch_chain(chain_shape(P), L, anchor, E, W, ws + P.o_chain, ltok, lppos, ls, &cerr,
                         dev_status, ccol, clval, cwmax, ws + P.o_swcol, s));
     FinalArgs f;
@@ -342,7 +351,10 @@ int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t*
     sd.thr = row_thr;
     return sd;
   };
-  if (seeded)
+  if (seeded && seed_tok)
+    PCT_CU(launch_seed_columns(P.batch * P.D, P.V, P.k, P.ldt, L, W, Wt, P.r, P.r_pad, seed_tok,
+                               scol, slval, swmax, swcol, s));
+  else if (seeded)
     PCT_CU(launch_drafter_topk(P.batch * P.D, P.V, P.k, P.ldt, L, W, P.r, P.r_pad, scol, slval,
                                swmax, swcol, ws + P.o_sdk, s));
   PCT_CU(launch_gather_rows(P.batch, anchor, P.V, P.r, P.r_pad, P.mdt, E, Eg, dev_status, 1,
@@ -382,6 +394,40 @@ int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t*
   f.status = dev_status;
   f.err = err;
   PCT_CU(launch_final(f, s));
+  return PCT_OK;
+}
+
+int32_t pct_tree_build(const pct_build_desc* desc, const void* L, const int32_t* anchor,
+                       const void* E, const void* W, int32_t* tok, int32_t* parent,
+                       int32_t* depth, float* score, int32_t* count, int32_t* dev_status,
+                       void* workspace, size_t ws_bytes, void* cuda_stream) {
+  return pct_build_impl(desc, L, anchor, E, W, nullptr, nullptr, tok, parent, depth, score,
+                        count, dev_status, workspace, ws_bytes, cuda_stream);
+}
+
+int32_t pct_tree_build_seeded(const pct_build_desc* desc, const void* L, const int32_t* anchor,
+                              const void* E, const void* W, const void* Wt,
+                              const int32_t* seed_tok, int32_t* tok, int32_t* parent,
+                              int32_t* depth, float* score, int32_t* count, int32_t* dev_status,
+                              void* workspace, size_t ws_bytes, void* cuda_stream) {
+  if (!seed_tok) return PCT_EINVAL;
+  if (Wt && (!aligned(Wt, 16) || !desc || desc->markov_dtype != PCT_BF16)) return PCT_EINVAL;
+  return pct_build_impl(desc, L, anchor, E, W, Wt, seed_tok, tok, parent, depth, score, count,
+                        dev_status, workspace, ws_bytes, cuda_stream);
+}
+
+int32_t pct_markov_rank_pad(int32_t rank) {
+  return (rank < 1 || rank > 256) ? 0 : (rank + 63) / 64 * 64;
+}
+
+int32_t pct_markov_transpose(int32_t vocab, int32_t rank, const void* W, void* Wt,
+                             void* cuda_stream) {
+  const int r_pad = pct_markov_rank_pad(rank);
+  if (r_pad == 0 || vocab < 8 || vocab % 8 != 0 || vocab > (1 << 22) || !W || !Wt)
+    return PCT_EINVAL;
+  if (!aligned(W, 16) || !aligned(Wt, 16)) return PCT_EINVAL;
+  if (!device_ok()) return PCT_EDEVICE;
+  PCT_CU(launch_markov_transpose(vocab, rank, r_pad, W, Wt, static_cast<cudaStream_t>(cuda_stream)));
   return PCT_OK;
 }
 
@@ -466,14 +512,16 @@ size_t cadd_tree_grow_workspace(const cadd_desc* desc) {
   return P.total;
 }
 
-int32_t cadd_tree_grow(const cadd_desc* desc, const void* L, const int32_t* anchor,
-                       const int64_t* ctx_len, int32_t* tok, int32_t* parent, int32_t* depth,
-                       float* score, int32_t* count, float* phi, int32_t* dev_status,
-                       void* workspace, size_t ws_bytes, void* cuda_stream) {
+static int32_t cadd_grow_impl(const cadd_desc* desc, const void* L, const int32_t* anchor,
+                              const int64_t* ctx_len, int32_t top_k, int32_t* tok, int32_t* parent,
+                              int32_t* depth, float* score, int32_t* count, float* phi,
+                              int32_t* top_tok, int32_t* dev_status, void* workspace,
+                              size_t ws_bytes, void* cuda_stream) {
   const int st = check_cadd(desc);
   if (st != PCT_OK) return st;
   if (!L || !anchor || !ctx_len || !tok || !parent || !depth || !score || !count || !phi || !dev_status)
     return PCT_EINVAL;
+  if (top_k < 0 || top_k > 32 || (top_k > 0 && !top_tok)) return PCT_EINVAL;
   if (!device_ok()) return PCT_EDEVICE;
   CaddPlan P;
   cadd_plan(desc, &P);
@@ -483,12 +531,30 @@ int32_t cadd_tree_grow(const cadd_desc* desc, const void* L, const int32_t* anch
   char* ws = static_cast<char*>(workspace);
   PCT_CU(cudaMemsetAsync(dev_status, 0, sizeof(int32_t) * desc->batch, s));
   CaddParams p{desc->batch, desc->depth, desc->vocab, desc->n_max, desc->logits_dtype,
-               desc->C_d, desc->a, desc->b, desc->c, desc->e};
+               desc->C_d, desc->a, desc->b, desc->c, desc->e, top_k, top_tok};
   PCT_CU(launch_cadd(p, L, anchor, ctx_len, tok, parent, depth, score, count, phi, dev_status,
                      reinterpret_cast<float*>(ws + P.o_lse), reinterpret_cast<int32_t*>(ws + P.o_cnt),
                      reinterpret_cast<float*>(ws + P.o_q), reinterpret_cast<int32_t*>(ws + P.o_tok),
-                     P.seg_bytes ? ws + P.o_seg : nullptr, s));
+                     P.seg_bytes ? ws + P.o_seg : nullptr, ws + P.o_topk, s));
   return PCT_OK;
+}
+
+int32_t cadd_tree_grow(const cadd_desc* desc, const void* L, const int32_t* anchor,
+                       const int64_t* ctx_len, int32_t* tok, int32_t* parent, int32_t* depth,
+                       float* score, int32_t* count, float* phi, int32_t* dev_status,
+                       void* workspace, size_t ws_bytes, void* cuda_stream) {
+  return cadd_grow_impl(desc, L, anchor, ctx_len, 0, tok, parent, depth, score, count, phi,
+                        nullptr, dev_status, workspace, ws_bytes, cuda_stream);
+}
+
+int32_t cadd_tree_grow_topk(const cadd_desc* desc, const void* L, const int32_t* anchor,
+                            const int64_t* ctx_len, int32_t top_k, int32_t* tok, int32_t* parent,
+                            int32_t* depth, float* score, int32_t* count, float* phi,
+                            int32_t* top_tok, int32_t* dev_status, void* workspace,
+                            size_t ws_bytes, void* cuda_stream) {
+  if (top_k < 1) return PCT_EINVAL;
+  return cadd_grow_impl(desc, L, anchor, ctx_len, top_k, tok, parent, depth, score, count, phi,
+                        top_tok, dev_status, workspace, ws_bytes, cuda_stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -35,6 +35,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "select.cuh"
 
 namespace pct {
 namespace {
@@ -229,6 +230,22 @@ __device__ void select_topk_exact(const T* x, int V, bool vec, int K, unsigned l
   __syncthreads();
 }
 
+// Each row's top_k tokens (cadd_tree_grow_topk). The row pass holds, sorted,
+// every value of the row above the row's threshold (or the exact n best);
+// when there are at least top_k of them their head is the answer, written
+// here. Otherwise the row joins the list of rows cadd_topk_fill_kernel
+// selects exactly (in any order). Block-wide (every thread calls it, with the
+// same n).
+__device__ __forceinline__ void cadd_topk_head(const CaddParams& p, size_t row, int n,
+                                               const unsigned long long* keys) {
+  if (n >= p.top_k) {
+    for (int j = threadIdx.x; j < p.top_k; j += blockDim.x)
+      p.top_tok[row * p.top_k + j] = (int)(~(unsigned)(keys[j] & 0xffffffffu));
+  } else if (threadIdx.x == 0) {
+    p.top_list[atomicAdd(p.top_list_n, 1u)] = (int)row;
+  }
+}
+
 template <typename T>
 __global__ __launch_bounds__(kRowThreads, 3) void cadd_rowpass_kernel(
     CaddParams p, const T* __restrict__ L, const int64_t* __restrict__ ctx,
@@ -418,6 +435,7 @@ __global__ __launch_bounds__(kRowThreads, 3) void cadd_rowpass_kernel(
     cand_q[cbase + j] = z - lse;
     cand_tok[cbase + j] = (int)(~(unsigned)(kk & 0xffffffffu));
   }
+  if (p.top_k > 0) cadd_topk_head(p, row, n, keys);
   if (threadIdx.x == 0) {
     cand_cnt[row] = keep;
     row_lse[row] = lse;
@@ -846,10 +864,196 @@ __global__ __launch_bounds__(kFinThreads) void cadd_seg_finish_kernel(
     cand_q[cbase + j] = ord2f((unsigned)(kk >> 32)) - lse;
     cand_tok[cbase + j] = (int)(~(unsigned)(kk & 0xffffffffu));
   }
+  if (p.top_k > 0) cadd_topk_head(p, (size_t)row, n, keys);
   if (threadIdx.x == 0) {
     cand_cnt[row] = keep;
     row_lse[row] = lse;
   }
+}
+
+// ---------------------------------------------------------------------------
+// Exact top_k of the rows the row pass listed (fewer than top_k values above
+// their threshold), each row cut into parts; a block takes one part of a
+// listed row in two reads of it:
+//  1. every thread's best key (value desc, token asc: keys are distinct); the
+//     top_k-th best of the block's thread bests, g, is at most the part's
+//     top_k-th best key (top_k distinct keys of the part reach it);
+//  2. every key >= g into shared memory. Only the top_k threads whose best
+//     reaches g hold such keys, so there are few; they are sorted and the
+//     first top_k kept. Should more than kFillCap arrive (a part whose large
+//     values sit in a few threads' strides), every warp instead folds the part
+//     into a sorted 32-key list, exact at any size.
+// With more than one part the parts' lists are published and the row's last
+// block to arrive (a counter per row, cleared by the launcher, reset by that
+// block) merges them. Nothing waits on another block.
+constexpr int kFillThreads = 256;
+constexpr int kFillParts = 16;   // most parts of a row
+constexpr int kFillLoads = 8;    // 16-byte (or scalar) loads in flight per thread
+constexpr int kFillCap = 2048;   // keys collected in step 2
+
+// f(z, v) for the values of [v0, v1) (vector: 8-value groups [g0, g1)) that
+// this thread owns, kFillLoads loads in flight; the trip count is the same
+// for every thread of a warp.
+template <typename T, typename F>
+__device__ __forceinline__ void fill_visit(const T* x, bool vec, int lo, int hi, F&& f) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int step = kFillThreads * kFillLoads;
+  if (sizeof(T) == 2 && vec) {
+    const uint4* xg = reinterpret_cast<const uint4*>(x);
+    for (int base = lo + warp * 32 * kFillLoads; base < hi; base += step) {
+      uint4 q[kFillLoads];
+#pragma unroll
+      for (int u = 0; u < kFillLoads; ++u) {
+        const int g = base + 32 * u + lane;
+        q[u] = g < hi ? xg[g] : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kFillLoads; ++u) {
+        const int g = base + 32 * u + lane;
+        const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          f((e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]), 8 * g + e, g < hi);
+      }
+    }
+  } else {
+    for (int base = lo + warp * 32 * kFillLoads; base < hi; base += step) {
+      float z[kFillLoads];
+#pragma unroll
+      for (int u = 0; u < kFillLoads; ++u) {
+        const int v = base + 32 * u + lane;
+        z[u] = v < hi ? load_f(x + v) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kFillLoads; ++u) {
+        const int v = base + 32 * u + lane;
+        f(z[u], v, v < hi);
+      }
+    }
+  }
+}
+
+struct FillSmem {
+  unsigned long long keys[kFillCap];
+  unsigned long long g;
+  int n, last;
+};
+
+// One (row, part) item; every thread of the block calls it.
+template <typename T>
+__device__ void cadd_topk_fill_item(const CaddParams& p, const T* __restrict__ L, bool vec,
+                                    int row, int part, int parts, FillSmem& sm) {
+  const int V = p.V, top_k = p.top_k;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int nwarps = kFillThreads / 32;
+  unsigned long long* keys = sm.keys;
+  const T* x = L + (size_t)row * V;
+  const bool groups = sizeof(T) == 2 && vec;
+  const int n_units = groups ? V >> 3 : V;
+  const int lo = (int)((long long)n_units * part / parts);
+  const int hi = (int)((long long)n_units * (part + 1) / parts);
+
+  // 1. thread bests, then the top_k-th best of them
+  unsigned long long best = 0ull;
+  fill_visit(x, vec, lo, hi, [&](float z, int v, bool ok) {
+    const unsigned long long k = ok ? cand_key(z, v) : 0ull;
+    best = k > best ? k : best;
+  });
+  keys[threadIdx.x] = warp_sort_desc(best, lane);
+  if (threadIdx.x == 0) sm.n = 0;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned long long acc = keys[lane];
+#pragma unroll
+    for (int w = 1; w < nwarps; ++w) acc = warp_merge_top(acc, keys[32 * w + 31 - lane], lane);
+    if (lane == top_k - 1) sm.g = acc;
+  }
+  __syncthreads();
+  const unsigned long long g = sm.g;   // 0: fewer than top_k values, all of them qualify
+
+  // 2. every key >= g
+  fill_visit(x, vec, lo, hi, [&](float z, int v, bool ok) {
+    const unsigned long long k = ok ? cand_key(z, v) : 0ull;
+    if (k != 0ull && k >= g) {
+      const int at = atomicAdd(&sm.n, 1);
+      if (at < kFillCap) keys[at] = k;
+    }
+  });
+  __syncthreads();
+  const int n = sm.n;
+  unsigned long long acc = 0ull;
+  if (n <= 32) {
+    if (warp == 0) acc = warp_sort_desc(lane < n ? keys[lane] : 0ull, lane);
+  } else if (n <= kFillCap) {
+    int P = 1;
+    while (P < n) P <<= 1;
+    for (int j = n + threadIdx.x; j < P; j += kFillThreads) keys[j] = 0ull;
+    __syncthreads();
+    bitonic_desc(keys, P);
+    if (warp == 0) acc = keys[lane];
+  } else {
+    // exact at any size: each warp folds 32 keys at a time into its sorted list
+    unsigned long long list = 0ull, thr = 0ull;
+    fill_visit(x, vec, lo, hi, [&](float z, int v, bool ok) {
+      unsigned long long k = ok ? cand_key(z, v) : 0ull;
+      if (__any_sync(0xffffffffu, k > thr)) {
+        k = warp_sort_desc(k, lane);
+        list = warp_merge_top(list, __shfl_sync(0xffffffffu, k, 31 - lane), lane);
+        thr = __shfl_sync(0xffffffffu, list, top_k - 1);
+      }
+    });
+    __syncthreads();
+    keys[32 * warp + lane] = list;
+    __syncthreads();
+    if (warp == 0) {
+      acc = keys[lane];
+#pragma unroll
+      for (int w = 1; w < nwarps; ++w) acc = warp_merge_top(acc, keys[32 * w + 31 - lane], lane);
+    }
+  }
+  bool write = true;
+  if (parts > 1) {
+    unsigned long long* pk = p.top_keys + (size_t)row * kFillParts * 32;
+    if (warp == 0) pk[part * 32 + lane] = lane < top_k ? acc : 0ull;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) sm.last = atomicAdd(&p.top_cnt[row], 1u) == (unsigned)(parts - 1);
+    __syncthreads();
+    write = sm.last != 0;
+    if (write) {
+      __threadfence();
+      if (warp == 0) {
+        // every part's list in registers at once (the loads overlap), then merged
+        unsigned long long b[kFillParts];
+#pragma unroll
+        for (int q = 0; q < kFillParts; ++q)
+          b[q] = q < parts ? __ldcg(pk + q * 32 + (q == 0 ? lane : 31 - lane)) : 0ull;
+        acc = b[0];
+#pragma unroll
+        for (int q = 1; q < kFillParts; ++q)
+          if (q < parts) acc = warp_merge_top(acc, b[q], lane);
+        if (lane == 0) p.top_cnt[row] = 0u;   // ready for the next launch
+      }
+    }
+  }
+  if (write && warp == 0 && lane < top_k)
+    p.top_tok[(size_t)row * top_k + lane] = acc ? (int)(~(unsigned)(acc & 0xffffffffu)) : -1;
+  __syncthreads();   // the shared memory is free for the block's next item
+}
+
+// Items (listed row, part) are spread over a small grid: item i is part
+// i % parts of row top_list[i / parts]; blocks take items i = blockIdx.x,
+// blockIdx.x + gridDim.x, ...
+template <typename T>
+__global__ __launch_bounds__(kFillThreads) void cadd_topk_fill_kernel(CaddParams p,
+                                                                       const T* __restrict__ L,
+                                                                       bool vec, int parts) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ FillSmem sm;
+  const int items = (int)*p.top_list_n * parts;
+  for (int i = (int)blockIdx.x; i < items; i += (int)gridDim.x)
+    cadd_topk_fill_item(p, L, vec, p.top_list[i / parts], i % parts, parts, sm);
 }
 
 // ---------------------------------------------------------------------------
@@ -1040,11 +1244,29 @@ size_t cadd_seg_workspace(int batch, int D, int V, int dtype) {
          align256(slots * sizeof(float)) + 2 * rows * seg_words(V) * sizeof(uint32_t);
 }
 
-cudaError_t launch_cadd(const CaddParams& p, const void* L, const int32_t* anchor,
+size_t cadd_topk_workspace(size_t rows) {
+  return align256(rows * sizeof(int32_t)) + align256((rows + 1) * sizeof(unsigned)) +
+         rows * kFillParts * 32 * sizeof(unsigned long long);
+}
+
+cudaError_t launch_cadd(const CaddParams& p_in, const void* L, const int32_t* anchor,
                         const int64_t* ctx, int32_t* tok, int32_t* parent, int32_t* depth,
                         float* score, int32_t* count, float* phi, int32_t* status,
                         float* row_lse, int32_t* cand_cnt, float* cand_q, int32_t* cand_tok,
-                        void* seg_ws, cudaStream_t s) {
+                        void* seg_ws, void* topk_ws, cudaStream_t s) {
+  CaddParams p = p_in;
+  if (p.top_k > 0) {
+    const size_t rows = (size_t)p.batch * p.D;
+    char* c = static_cast<char*>(topk_ws);
+    if (!c || p.top_k > 32) return cudaErrorInvalidValue;
+    p.top_list = reinterpret_cast<int32_t*>(c);            c += align256(rows * sizeof(int32_t));
+    p.top_cnt = reinterpret_cast<unsigned*>(c);            // [rows] part counters, then the
+    p.top_list_n = p.top_cnt + rows;                       // list's length: cleared together
+    c += align256((rows + 1) * sizeof(unsigned));
+    p.top_keys = reinterpret_cast<unsigned long long*>(c);
+    cudaError_t e = cudaMemsetAsync(p.top_cnt, 0, (rows + 1) * sizeof(unsigned), s);
+    if (e != cudaSuccess) return e;
+  }
   const bool segmented = seg_ws != nullptr && p.dtype == PCT_BF16 && p.V % 8 == 0 &&
                          (reinterpret_cast<uintptr_t>(L) & 15u) == 0;
   if (segmented) {
@@ -1079,6 +1301,22 @@ cudaError_t launch_cadd(const CaddParams& p, const void* L, const int32_t* ancho
             : launch_pdl(cadd_rowpass_kernel<float>, grid, dim3(kRowThreads), 0, s, 1, p,
                          static_cast<const float*>(L), ctx, row_lse, cand_cnt, cand_q, cand_tok,
                          status);
+    if (e != cudaSuccess) return e;
+  }
+  if (p.top_k > 0) {
+    // exact top_k of the rows with fewer than top_k values above their threshold
+    // parts of about 8192 values (one or two loads per thread and read);
+    // the grid covers the SMs twice and loops over however many items there are
+    const int parts = std::max(1, std::min(kFillParts, (p.V + 8191) / 8192));
+    const bool vec = p.dtype == PCT_BF16 && p.V % 8 == 0 && (reinterpret_cast<uintptr_t>(L) & 15u) == 0;
+    const size_t items = (size_t)p.batch * p.D * parts;
+    const unsigned grid = (unsigned)std::min<size_t>(items, (size_t)2 * num_sms());
+    TraceScope t(s, "cadd_topk_fill");
+    cudaError_t e = p.dtype == PCT_BF16
+        ? launch_pdl(cadd_topk_fill_kernel<__nv_bfloat16>, dim3(grid), dim3(kFillThreads), 0, s, 1,
+                     p, static_cast<const __nv_bfloat16*>(L), vec, parts)
+        : launch_pdl(cadd_topk_fill_kernel<float>, dim3(grid), dim3(kFillThreads), 0, s, 1, p,
+                     static_cast<const float*>(L), vec, parts);
     if (e != cudaSuccess) return e;
   }
   const size_t base = (size_t)(p.n_max + 1) * 8 + (size_t)p.n_max * 4 * 6;

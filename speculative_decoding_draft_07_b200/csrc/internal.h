@@ -49,7 +49,16 @@ cudaError_t launch_accept_sim(int batch, int n_stride, int max_depth, const int3
 struct CaddParams {
   int batch, D, V, n_max, dtype;
   float C_d, a, b, c, e;
+  int top_k;                      // > 0: each row's top_k tokens into top_tok [rows][top_k]
+  int32_t* top_tok;
+  int32_t* top_list;              // [rows] rows the row pass left to the exact selection
+  unsigned* top_list_n;           // their number
+  unsigned* top_cnt;              // [rows] part counters of the exact selection
+  unsigned long long* top_keys;   // [rows][parts][32] the parts' lists
 };
+// Workspace of the top_k output (cadd_tree_grow_topk): top_list, top_cnt and
+// top_list_n, top_keys for `rows` rows, 256-byte aligned pieces.
+size_t cadd_topk_workspace(size_t rows);
 size_t cadd_rowpass_bytes_per_row(int n_max);
 // Workspace of the segmented row pass (bf16 rows with V % 8 == 0; else 0).
 size_t cadd_seg_workspace(int batch, int D, int V, int dtype);
@@ -57,7 +66,7 @@ cudaError_t launch_cadd(const CaddParams& p, const void* L, const int32_t* ancho
                         const int64_t* ctx, int32_t* tok, int32_t* parent, int32_t* depth,
                         float* score, int32_t* count, float* phi, int32_t* status,
                         float* row_lse, int32_t* cand_cnt, float* cand_q, int32_t* cand_tok,
-                        void* seg_ws, cudaStream_t s);
+                        void* seg_ws, void* topk_ws, cudaStream_t s);
 
 // ---- PCTree (pct_*.cu) ------------------------------------------------------
 // Partial results of one (row, V-slice): online log-sum-exp state and the
@@ -121,6 +130,18 @@ size_t drafter_topk_scratch(int rows);
 cudaError_t launch_drafter_topk(int rows, int V, int ks, int logits_dtype, const void* L,
                                 const void* W, int r, int r_pad, int32_t* cols, float* lval,
                                 float* wmax, void* wcol, void* scratch, cudaStream_t s);
+
+// Seed data for every row of the logits from caller-given columns in[rows][ks]
+// (dropped: entries outside [0, V) and repeats within a row); the same
+// outputs as launch_drafter_topk.
+// Wt: null, or W transposed [V][r_pad] (launch_markov_transpose), read instead of W.
+cudaError_t launch_seed_columns(int rows, int V, int ks, int logits_dtype, const void* L,
+                                const void* W, const void* Wt, int r, int r_pad,
+                                const int32_t* in, int32_t* cols, float* lval, float* wmax,
+                                void* wcol, cudaStream_t s);
+// Wt [V][r_pad] = W [r][V] transposed (bf16, zero past r; V % 8 == 0).
+cudaError_t launch_markov_transpose(int V, int r, int r_pad, const void* W, void* Wt,
+                                    cudaStream_t s);
 
 struct MergeArgs {
   int batch, F_prev, F_new, k, beam, S, V, r, r_pad, markov_dtype, depth;

@@ -200,7 +200,151 @@ __global__ void __launch_bounds__(kSeedThreads) drafter_topk_kernel(
   }
 }
 
+// Seed data from given columns, one block per row of L: in[row][ks] are the
+// caller's columns; entries outside [0, V) and repeats of an earlier entry of
+// the row are dropped (-1), so the kept columns are distinct. W's columns are
+// gathered kColLoads strided loads per thread at a time (one 2-byte value of
+// each of r rows of W per column); their largest magnitude is a warp max (a
+// warp's 32 consecutive entries lie in one column, r_pad being a multiple of
+// 32) and one shared-memory max per warp.
+constexpr int kColThreads = 128;
+constexpr int kColLoads = 16;
+
+// With Wt (W transposed, [V][r_pad], zero past r) a column is one contiguous
+// run of r_pad values instead: 16-byte loads, r_pad / 8 per column.
+template <typename TL>
+__global__ void __launch_bounds__(kColThreads) seed_columns_kernel(
+    int V, int ks, const TL* __restrict__ L, const __nv_bfloat16* __restrict__ W,
+    const __nv_bfloat16* __restrict__ Wt, int r, int r_pad, const int32_t* __restrict__ in,
+    int32_t* __restrict__ cols, float* __restrict__ lval, float* __restrict__ wmax,
+    __nv_bfloat16* __restrict__ wcol) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int sc[kSeedMaxK];
+  __shared__ unsigned smax[kSeedMaxK];
+  const int rowi = (int)blockIdx.x;
+  const size_t e0 = (size_t)rowi * ks;
+  if (threadIdx.x < ks) {
+    int c = in[e0 + threadIdx.x];
+    if (c < 0 || c >= V) c = -1;
+    for (int j = 0; j < (int)threadIdx.x; ++j)
+      if (c >= 0 && in[e0 + j] == c) c = -1;   // the first occurrence stays
+    sc[threadIdx.x] = c;
+    smax[threadIdx.x] = 0u;
+  }
+  __syncthreads();
+  const int n = ks * r_pad;   // a multiple of 32: the loop below is warp-uniform
+  __nv_bfloat16* dst = wcol + e0 * r_pad;
+  if (Wt) {
+    const int cpc = r_pad / 8;   // 16-byte chunks per column
+    for (int e = threadIdx.x; e < ks * cpc; e += kColThreads) {
+      const int c = e / cpc, j = e - c * cpc;
+      const int col = sc[c];
+      uint4 q = make_uint4(0u, 0u, 0u, 0u);
+      if (col >= 0) q = *reinterpret_cast<const uint4*>(Wt + (size_t)col * r_pad + 8 * j);
+      *reinterpret_cast<uint4*>(dst + (size_t)c * r_pad + 8 * j) = q;
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+      float m = 0.f;
+#pragma unroll
+      for (int h = 0; h < 4; ++h) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[h])), fabsf(bf16_hi(w[h]))));
+      atomicMax(&smax[c], __float_as_uint(m));
+    }
+  } else
+  for (int e = threadIdx.x; e < n; e += kColLoads * kColThreads) {
+    __nv_bfloat16 w[kColLoads];
+#pragma unroll
+    for (int u = 0; u < kColLoads; ++u) {
+      const int f = e + u * kColThreads;
+      w[u] = __float2bfloat16(0.f);
+      if (f < n) {
+        const int c = f / r_pad, j = f - c * r_pad;
+        const int col = sc[c];
+        if (col >= 0 && j < r) w[u] = W[(size_t)j * V + col];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kColLoads; ++u) {
+      const int f = e + u * kColThreads;
+      if (f < n) {
+        dst[f] = w[u];
+        const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(__bfloat162float(w[u]))));
+        if ((threadIdx.x & 31) == 0) atomicMax(&smax[f / r_pad], m);
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < ks) {
+    const int c = sc[threadIdx.x];
+    cols[e0 + threadIdx.x] = c;
+    lval[e0 + threadIdx.x] = c >= 0 ? load_f(L + (size_t)rowi * V + c) : neg_inf();
+    wmax[e0 + threadIdx.x] = __uint_as_float(smax[threadIdx.x]);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_seed_columns(int rows, int V, int ks, int logits_dtype, const void* L,
+                                const void* W, const void* Wt, int r, int r_pad,
+                                const int32_t* in, int32_t* cols, float* lval, float* wmax,
+                                void* wcol, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  if (ks < 1 || ks > kSeedMaxK || r > kSeedMaxR || r_pad > kSeedMaxR || r_pad % 32 != 0)
+    return cudaErrorInvalidValue;
+  const __nv_bfloat16* Wb = static_cast<const __nv_bfloat16*>(W);
+  const __nv_bfloat16* Wtb = static_cast<const __nv_bfloat16*>(Wt);
+  __nv_bfloat16* wc = static_cast<__nv_bfloat16*>(wcol);
+  TraceScope t(s, "seed_columns");
+  if (logits_dtype == PCT_BF16)
+    return launch_pdl(seed_columns_kernel<__nv_bfloat16>, dim3((unsigned)rows), dim3(kColThreads),
+                      0, s, 1, V, ks, static_cast<const __nv_bfloat16*>(L), Wb, Wtb, r, r_pad, in,
+                      cols, lval, wmax, wc);
+  return launch_pdl(seed_columns_kernel<float>, dim3((unsigned)rows), dim3(kColThreads), 0, s, 1,
+                    V, ks, static_cast<const float*>(L), Wb, Wtb, r, r_pad, in, cols, lval, wmax,
+                    wc);
+}
+
+// W [r][V] -> Wt [V][r_pad] (bf16, zero past r): a block per 64 columns of W,
+// staged through shared memory so that both sides move in 16-byte pieces.
+constexpr int kTrCols = 64;
+__global__ void __launch_bounds__(256) markov_transpose_kernel(int V, int r, int r_pad,
+                                                              const __nv_bfloat16* __restrict__ W,
+                                                              __nv_bfloat16* __restrict__ Wt) {
+  __shared__ __align__(16) __nv_bfloat16 tile[kSeedMaxR][kTrCols + 8];   // rows of 144 bytes
+  const int v0 = (int)blockIdx.x * kTrCols;
+  const int nv = min(kTrCols, V - v0);   // a multiple of 8 (V % 8 == 0)
+  for (int i = threadIdx.x; i < r * (kTrCols / 8); i += blockDim.x) {
+    const int j = i / (kTrCols / 8), c = i - j * (kTrCols / 8);
+    if (8 * c < nv)
+      *reinterpret_cast<uint4*>(&tile[j][8 * c]) =
+          *reinterpret_cast<const uint4*>(W + (size_t)j * V + v0 + 8 * c);
+  }
+  __syncthreads();
+  const int cpc = r_pad / 8;
+  for (int i = threadIdx.x; i < nv * cpc; i += blockDim.x) {
+    const int cc = i / cpc, jc = i - cc * cpc;
+    uint32_t w[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const int j = 8 * jc + 2 * h;
+      const uint32_t lo = j < r ? __bfloat16_as_ushort(tile[j][cc]) : 0u;
+      const uint32_t hi = j + 1 < r ? __bfloat16_as_ushort(tile[j + 1][cc]) : 0u;
+      w[h] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4*>(Wt + (size_t)(v0 + cc) * r_pad + 8 * jc) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+cudaError_t launch_markov_transpose(int V, int r, int r_pad, const void* W, void* Wt,
+                                    cudaStream_t s) {
+  if (V <= 0 || V % 8 != 0 || r < 1 || r > kSeedMaxR || r_pad < r || r_pad > kSeedMaxR ||
+      r_pad % 8 != 0)
+    return cudaErrorInvalidValue;
+  TraceScope t(s, "markov_transpose");
+  markov_transpose_kernel<<<(V + kTrCols - 1) / kTrCols, 256, 0, s>>>(
+      V, r, r_pad, static_cast<const __nv_bfloat16*>(W), static_cast<__nv_bfloat16*>(Wt));
+  return cudaGetLastError();
+}
 
 size_t drafter_topk_scratch(int rows) {
   return ((size_t)rows * sizeof(unsigned) + 255) / 256 * 256 +

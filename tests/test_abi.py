@@ -111,6 +111,33 @@ def test_cadd_rejects_bad_descriptors(bad):
     assert rc == pct.PCT_EINVAL
 
 
+def test_one_pass_entry_points_reject_bad_arguments():
+    """pct_tree_build_seeded without seeds or with a misaligned Wt, pct_markov_transpose
+    with a bad shape, cadd_tree_grow_topk with top_k outside 1..32 or no output:
+    PCT_EINVAL on the host, before the device is looked at."""
+    L = pct.lib()
+    dummy = ctypes.c_void_p(256)
+    d = _desc()
+    rc = L.pct_tree_build_seeded(ctypes.byref(d), dummy, dummy, dummy, dummy, None, None,
+                                 *([dummy] * 6), dummy, 1 << 30, None)
+    assert rc == pct.PCT_EINVAL
+    # Wt needs bf16 Markov parameters and 16-byte alignment
+    rc = L.pct_tree_build_seeded(ctypes.byref(d), dummy, dummy, dummy, dummy,
+                                 ctypes.c_void_p(264), dummy, *([dummy] * 6), dummy, 1 << 30, None)
+    assert rc == pct.PCT_EINVAL
+    assert L.pct_markov_rank_pad(1) == 64 and L.pct_markov_rank_pad(256) == 256
+    assert L.pct_markov_rank_pad(0) == 0 and L.pct_markov_rank_pad(257) == 0
+    assert L.pct_markov_transpose(1004, 64, dummy, dummy, None) == pct.PCT_EINVAL   # V % 8
+    assert L.pct_markov_transpose(1024, 0, dummy, dummy, None) == pct.PCT_EINVAL
+    assert L.pct_markov_transpose(1024, 64, None, dummy, None) == pct.PCT_EINVAL
+    c = pct.cadd_desc(batch=4, depth=15, vocab=1000, n_max=64, logits_dtype=pct.PCT_BF16,
+                      C_d=1.0, a=2.0, b=1e-4, c=5e-3, e=1e-5)
+    for k, out in ((0, dummy), (33, dummy), (-1, dummy), (8, None)):
+        rc = L.cadd_tree_grow_topk(ctypes.byref(c), dummy, dummy, dummy, k, *([dummy] * 6), out,
+                                   dummy, dummy, 1 << 30, None)
+        assert rc == pct.PCT_EINVAL, k
+
+
 def test_verify_and_mask_reject_bad_shapes():
     L = pct.lib()
     dummy = ctypes.c_void_p(256)

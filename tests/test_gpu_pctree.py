@@ -109,11 +109,12 @@ def test_score_parents_fp32_logits_bf16_markov(batch, n_par):
     _score_parents_case("bf16", 2000, 64, 8, batch, n_par, logits_dtype=torch.float32)
 
 
-def _build_and_compare(L, anchor, E, W, k, beam, N, label="", max_unresolved=0):
+def _build_and_compare(L, anchor, E, W, k, beam, N, label="", max_unresolved=0, seeds=None):
     """GPU build of every request, each compared with the oracle (near ties
     resolved toward the GPU's nodes; at most ``max_unresolved`` requests may
-    stay unmatched)."""
-    out = pct.pct_tree_build(L.to(DEV), anchor.to(DEV), E.to(DEV), W.to(DEV), k, beam, N)
+    stay unmatched). seeds: the gate columns of pct_tree_build_seeded."""
+    out = pct.pct_tree_build(L.to(DEV), anchor.to(DEV), E.to(DEV), W.to(DEV), k, beam, N,
+                             seeds=None if seeds is None else seeds.to(DEV))
     torch.cuda.synchronize()
     check_tree_invariants(out, anchor.numpy(), N, label)
     Ef, Wf, an = f64(E), f64(W), anchor.numpy()

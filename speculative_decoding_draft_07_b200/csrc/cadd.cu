@@ -1135,9 +1135,16 @@ __global__ __launch_bounds__(32) void cadd_bestfirst_kernel(
   auto q_at = [&](int depth, int rank) {
     return STAGED ? sq[(depth - 1) * K1 + rank] : cand_q[(row0 + depth - 1) * K1 + rank];
   };
+  // The pool is unsorted; slot j belongs to lane j % 32, which keeps the best
+  // key of its slots (lbest at lslot) in registers. A pop is the warp's
+  // largest lbest (keys are distinct), found by two 32-bit warp maxima; then
+  // only the owner of the popped slot and the owner of a new slot update.
   int pool_n = 0;
+  unsigned long long lbest = 0ull;
+  int lslot = -1;
   if (D >= 1 && nmax > 1 && cnt_at(1) > 0) {
-    if (lane == 0) pool[0] = pool_key(q_at(1, 0), 1, 0, 0);
+    const unsigned long long k0 = pool_key(q_at(1, 0), 1, 0, 0);
+    if (lane == 0) { pool[0] = k0; lbest = k0; lslot = 0; }
     pool_n = 1;
   }
   __syncwarp();
@@ -1147,16 +1154,14 @@ __global__ __launch_bounds__(32) void cadd_bestfirst_kernel(
   int n = 1;
   float phi = 0.f;
   while (n < nmax) {
-    unsigned long long best = 0ull;
-    int bslot = -1;
-    for (int j = lane; j < pool_n; j += 32) {
-      const unsigned long long k = pool[j];
-      if (k > best) { best = k; bslot = j; }
-    }
-    const unsigned long long wbest = warp_max_u64(best);
-    if (wbest == 0ull) break;                                     // no candidate left
-    const unsigned own = __ballot_sync(0xffffffffu, best == wbest);
-    bslot = __shfl_sync(0xffffffffu, bslot, __ffs(own) - 1);
+    const unsigned hi = __reduce_max_sync(0xffffffffu, (unsigned)(lbest >> 32));
+    const bool top_hi = lbest != 0ull && (unsigned)(lbest >> 32) == hi;
+    const unsigned lo = __reduce_max_sync(0xffffffffu, top_hi ? (unsigned)lbest : 0u);
+    const unsigned long long wbest = ((unsigned long long)hi << 32) | lo;
+    const unsigned own = __ballot_sync(0xffffffffu, top_hi && (unsigned)lbest == lo);
+    if (own == 0u) break;                                         // no candidate left
+    const int owner = __ffs(own) - 1;
+    const int bslot = __shfl_sync(0xffffffffu, lslot, owner);
     const float s = ord2f((unsigned)(wbest >> 32));
     const int depth = 63 - (int)((wbest >> 20) & 63);
     const int pidx = 1023 - (int)((wbest >> 10) & 1023);
@@ -1173,12 +1178,24 @@ __global__ __launch_bounds__(32) void cadd_bestfirst_kernel(
     if (rank + 1 < cnt_at(depth)) sib = pool_key(ns[np] + q_at(depth, rank + 1), depth, np, rank + 1);
     if (depth < D && cnt_at(depth + 1) > 0) child = pool_key(s + q_at(depth + 1, 0), depth + 1, n, 0);
     __syncwarp();
-    if (lane == 0) {
-      ntok[n] = tk; npar[n] = np; ndep[n] = depth; ns[n] = s;
+    if (lane == 0) { ntok[n] = tk; npar[n] = np; ndep[n] = depth; ns[n] = s; }
+    if (lane == owner) {
+      // the popped slot takes the sibling; the owner's best is found again
       pool[bslot] = sib;
-      if (child) pool[pool_n] = child;
+      lbest = 0ull;
+      lslot = -1;
+      for (int j = lane; j < pool_n; j += 32) {
+        const unsigned long long k = j == bslot ? sib : pool[j];
+        if (k > lbest) { lbest = k; lslot = j; }
+      }
     }
-    if (child) ++pool_n;
+    if (child) {
+      if (lane == (pool_n & 31)) {
+        pool[pool_n] = child;
+        if (child > lbest) { lbest = child; lslot = pool_n; }
+      }
+      ++pool_n;
+    }
     phi += expf(s);
     ++n;
     __syncwarp();

@@ -216,3 +216,52 @@ def test_full_round_one_pass_serves_both_trees():
     rng = np.random.default_rng(7)
     for b, dd in zip(rng.integers(0, batch, 24), rng.integers(0, D, 24)):
         np.testing.assert_array_equal(topn[b, dd], oracle.row_topk(f64(L[b, dd].cpu()), w.k))
+
+
+@pytest.mark.parametrize("V,top_k", [(20488, 1), (10240, 32), (10248, 16), (183520, 8)])
+def test_grow_topk_segment_edges(V, top_k):
+    """Segment boundaries (a last segment of one 16-byte group, exactly one full
+    segment, eighteen segments) and the extreme top_k; every row of a flat batch
+    (sigma 0.05, stop disabled) is left to the exact selection, in 16 parts at the
+    largest V."""
+    L = _sharp_logits(2, 3, V, seed=V % 89 + top_k, sigma=2.0, peak=(0.0, 6.0))
+    _check_topk(L, np.arange(2), np.array([4096, 32768]), 64, COST, top_k)
+    flat = _sharp_logits(2, 3, V, seed=V % 83, sigma=0.05, peak=(0.0, 0.1))
+    _check_topk(flat, np.arange(2), np.zeros(2), 1, dict(C_d=1.0, a=1.0, b=0.0, c=0.0, e=0.0),
+                top_k)
+
+
+def test_grow_topk_repeated_calls_reuse_the_workspace():
+    """The exact selection's counters and row list are reset by every call: ten
+    calls on one workspace, alternating flat rows (every row left to the exact
+    selection) and wide rows (none left)."""
+    batch, D, V = 4, 5, 30000
+    La = _sharp_logits(batch, D, V, seed=51, sigma=0.05, peak=(0.0, 0.5))
+    Lb = _sharp_logits(batch, D, V, seed=52, sigma=2.0, peak=(0.0, 6.0))   # hundreds above θ
+    a = torch.arange(batch, dtype=torch.int32, device=DEV)
+    c = torch.full((batch,), 4096, dtype=torch.int64, device=DEV)
+    cost = dict(C_d=1.0, a=1.0, b=0.0, c=1e-3, e=0.0)
+    cdesc = pct.cadd_desc(batch, D, V, 32, pct.PCT_BF16, *cost.values())
+    import ctypes
+    ws = torch.empty(int(pct.lib().cadd_tree_grow_workspace(ctypes.byref(cdesc))), dtype=torch.uint8,
+                     device=DEV)
+    refs = {id(La): oracle.row_topk(f64(La), 8), id(Lb): oracle.row_topk(f64(Lb), 8)}
+    Ld = {id(La): La.to(DEV), id(Lb): Lb.to(DEV)}
+    for i in range(10):
+        L = La if i % 2 == 0 else Lb
+        top = torch.full((batch, D, 8), -7, dtype=torch.int32, device=DEV)
+        pct.cadd_tree_grow(Ld[id(L)], a, c, 32, **cost, workspace=ws, top_tok=top)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(host(top), refs[id(L)], err_msg=f"call {i}")
+
+
+@pytest.mark.parametrize("k,beam,N", [(16, 32, 200), (1, 4, 7)])
+def test_seeded_build_extreme_k(k, beam, N):
+    """k = 16 (the largest: sixteen seed columns per row) and k = 1 (chains)."""
+    L, anchor, E, W = _problem(17, 5, 4096, 64, seed=60 + k)
+    seeds = _cadd_seeds(L, k)
+    plain, seeded, names = _unseeded_and_seeded(L, anchor, E, W, k, beam, N, seeds,
+                                                transposed=True)
+    torch.cuda.synchronize()
+    _same_tree(plain, seeded)
+    _build_and_compare(L, anchor, E, W, k, beam, N, label=f"seeded k={k}", seeds=seeds)

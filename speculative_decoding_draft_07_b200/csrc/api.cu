@@ -365,7 +365,7 @@ static int32_t pct_build_impl(const pct_build_desc* desc, const void* L, const i
     a.logits_dtype = P.ldt; a.markov_dtype = P.mdt;
     a.L = static_cast<const char*>(L) + (size_t)(d - 1) * P.V * esize(P.ldt);
     a.L_req_stride = (long long)P.D * P.V;
-    a.Eg = Eg; a.M_pad = P.M_pad; a.W = W; a.part = part; a.S = P.S[d]; a.err = err;
+    a.Eg = Eg; a.M_pad = P.M_pad; a.W = W; a.Wt = Wt; a.part = part; a.S = P.S[d]; a.err = err;
     a.row_thr = row_thr;
     a.thr_seeded = seeded;
     PCT_CU(launch_score(a, s));
@@ -496,7 +496,7 @@ int32_t pct_score_parents(const pct_build_desc* desc, int32_t n_par, const void*
   ScoreArgs a;
   a.n_req = P.batch; a.n_par = n_par; a.V = P.V; a.r = P.r; a.r_pad = P.r_pad; a.k = P.k;
   a.logits_dtype = P.ldt; a.markov_dtype = P.mdt; a.L = L_row; a.L_req_stride = P.V;
-  a.Eg = ws + o_eg; a.M_pad = P.M_pad; a.W = W; a.part = part; a.S = S; a.err = err;
+  a.Eg = ws + o_eg; a.M_pad = P.M_pad; a.W = W; a.Wt = nullptr; a.part = part; a.S = S; a.err = err;
   a.row_thr = reinterpret_cast<uint32_t*>(ws + o_thr);
   a.thr_seeded = false;
   PCT_CU(launch_score(a, s));

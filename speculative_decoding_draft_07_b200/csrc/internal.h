@@ -87,6 +87,7 @@ struct ScoreArgs {
   const void* Eg;         // [M_pad][r_pad] (bf16) or [M_pad][r] (f32)
   int M_pad;
   const void* W;          // [r][V]
+  const void* Wt;         // null, or W transposed [V][r_pad] (bf16): read instead of W
   Partials part;
   int S;                  // V-slices (partials per row)
   int32_t* err;           // device word, set on a timed-out wait

@@ -50,7 +50,8 @@ namespace {
 constexpr int BM = 128;                  // UMMA M (rows per tile)
 constexpr int BN = 128;                  // UMMA N (vocabulary columns per tile)
 constexpr int BK = 64;                   // K per ring slot: one 128-byte swizzle row of bf16
-constexpr int STAGES = 4;
+constexpr int STAGES = 4;                // ring slots after the A tiles
+constexpr int STAGES_MAX = 8;            // with one row tile, the second tile's space holds 4 more
 constexpr int KBMAX = 4;                 // r_pad <= 256
 constexpr int NSUBMAX = 2;               // row tiles per CTA
 constexpr int A_TILE_BYTES = BM * BK * 2;        // 16 KB
@@ -90,6 +91,7 @@ struct UmmaParams {
   int32_t* pidx;
   int32_t* err;
   uint32_t* row_thr;   // [M] best published k-th value per row (ordered key, 0 = none)
+  int b_kmajor;        // 1: W's tiles come from its transpose [V][r_pad] (K-major)
 };
 
 // LMODE (L_GLOBAL / L_STAGE / L_FOLD) says how the drafter logits L_d join
@@ -112,8 +114,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   constexpr bool STAGE = LMODE == L_STAGE;
   constexpr bool FOLD = LMODE == L_FOLD;
   uint64_t* full = reinterpret_cast<uint64_t*>(sL + 2 * L_SLOT_BYTES);
-  uint64_t* empty = full + STAGES;
-  uint64_t* afull = empty + STAGES;
+  uint64_t* empty = full + STAGES_MAX;
+  uint64_t* afull = empty + STAGES_MAX;
   uint64_t* tfull = afull + 1;      // [2]
   uint64_t* tempty = tfull + 2;     // [2]
   uint64_t* lfull = tempty + 2;     // [2]
@@ -128,9 +130,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int t_end = (int)((long long)(sl + 1) * p.tiles_total / p.S);
   const int ntiles = t_end - t_begin;
   const int row0 = mt * p.rows_per_cta;
+  // W ring: slots 0..3 after the A tiles; with a single row tile (and L_d not
+  // folded, whose per-slot parts have room for four) slots 4..7 in the unused
+  // second A tile, so that two N-tiles of W are in flight instead of one
+  const int nst = (!FOLD && p.nsub == 1) ? STAGES_MAX : STAGES;
+  uint8_t* const sB2 = sA + KBMAX * A_TILE_BYTES;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < STAGES_MAX; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     mbar_init(afull, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
@@ -192,22 +199,22 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t larmed = 0;
       for (int it = 0; it < ntiles && ok; ++it) {
         const int n0 = (t_begin + it) * BN;
-        if (STAGE) {
-          const int slot = it & 1;
-          if (!wait_bar(&lempty[slot], (((uint32_t)it >> 1) & 1u) ^ 1u, abort_flag, p.err)) { ok = false; break; }
-          mbar_expect_tx(&lfull[slot], (uint32_t)(2 * 64 * p.LB * 2));
-          uint8_t* dst = sL + slot * L_SLOT_BYTES;
-          tma_load_2d(dst, &tmL, n0, req0, &lfull[slot]);
-          tma_load_2d(dst + 64 * p.LB * 2, &tmL, n0 + 64, req0, &lfull[slot]);
-          larmed = (uint32_t)it + 1;
-        }
+        // W first: its slots free as the MMAs finish, the staged L_d slots only
+        // as the epilogue does, so waiting for an L_d slot before a tile's W
+        // would hold W back by a tile
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!wait_bar(&empty[stage], phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
           const bool lpart = FOLD && kb == 0;
           mbar_expect_tx(&full[stage], B_STAGE_BYTES + (lpart ? LF_PART_BYTES : 0));
-          uint8_t* dst = sB + stage * B_STAGE_BYTES;
-          tma_load_2d(dst, &tmB, n0, kb * BK, &full[stage]);
-          tma_load_2d(dst + B_STAGE_BYTES / 2, &tmB, n0 + 64, kb * BK, &full[stage]);
+          uint8_t* dst = stage < STAGES ? sB + stage * B_STAGE_BYTES
+                                        : sB2 + (stage - STAGES) * B_STAGE_BYTES;
+          if (p.b_kmajor) {
+            // [128 N rows][64 K] of W's transpose: one contiguous 16 KB piece
+            tma_load_2d(dst, &tmB, kb * BK, n0, &full[stage]);
+          } else {
+            tma_load_2d(dst, &tmB, n0, kb * BK, &full[stage]);
+            tma_load_2d(dst + B_STAGE_BYTES / 2, &tmB, n0 + 64, kb * BK, &full[stage]);
+          }
           if (lpart) {
             // the CTA's requests' L_d rows as the extra K block: [16 K][2 x 64 N]
             uint8_t* ldst = sL + stage * LF_PART_BYTES;
@@ -216,13 +223,22 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == nst) { stage = 0; phase ^= 1u; }
+        }
+        if (STAGE && ok) {
+          const int slot = it & 1;
+          if (!wait_bar(&lempty[slot], (((uint32_t)it >> 1) & 1u) ^ 1u, abort_flag, p.err)) { ok = false; break; }
+          mbar_expect_tx(&lfull[slot], (uint32_t)(2 * 64 * p.LB * 2));
+          uint8_t* dst = sL + slot * L_SLOT_BYTES;
+          tma_load_2d(dst, &tmL, n0, req0, &lfull[slot]);
+          tma_load_2d(dst + 64 * p.LB * 2, &tmL, n0 + 64, req0, &lfull[slot]);
+          larmed = (uint32_t)it + 1;
         }
       }
       // every load this thread issued has landed before the CTA may exit
       drain_wait(afull, 0);
 #pragma unroll
-      for (int i = 0; i < STAGES; ++i)
+      for (int i = 0; i < STAGES_MAX; ++i)
         if (armed & (1u << i)) drain_wait(&full[i], (armed_par >> i) & 1u);
       // the last one or two L_d slots armed (tiles larmed-1 and larmed-2)
       for (int t = (int)larmed - 2; t < (int)larmed; ++t)
@@ -242,7 +258,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       const uint64_t a_desc0 = make_desc(smem_u32(sA), 16, 1024);      // row tile 0, K block 0
-      const uint64_t b_desc0 = make_desc(smem_u32(sB), 8192, 1024);    // ring slot 0
+      // B: [64 K][2 x 64 V] V-major (W), +2048 bytes per 16 K rows; or, from
+      // W's transpose, [128 V][64 K] K-major like A, +32 bytes per 16 K
+      const uint32_t b_lbo = p.b_kmajor ? 16u : 8192u;
+      const uint64_t b_desc0 = make_desc(smem_u32(sB), b_lbo, 1024);    // ring slot 0
+      const uint64_t b_desc4 = make_desc(smem_u32(sB2), b_lbo, 1024);   // ring slot 4 (one row tile)
+      const uint64_t b_k16 = p.b_kmajor ? 2u : 128u;
+      const uint32_t idesc_w = p.b_kmajor ? (IDESC & ~(1u << 16)) : IDESC;
       // folded L_d: one-hot rows (K-major, 32-byte swizzle, 8-row groups 256
       // bytes apart) times the L_d part of ring slot `stage` (V-major,
       // 128-byte swizzle, the two 64-column halves 2048 bytes apart)
@@ -258,19 +280,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t d1 = d0 + BN;
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!wait_bar(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
-          const uint64_t bd = b_desc0 + (uint64_t)((stage * B_STAGE_BYTES) >> 4);
+          const uint64_t bd = stage < STAGES ? b_desc0 + (uint64_t)((stage * B_STAGE_BYTES) >> 4)
+                                             : b_desc4 + (uint64_t)(((stage - STAGES) * B_STAGE_BYTES) >> 4);
           const uint64_t ad = a_desc0 + (uint64_t)((kb * A_TILE_BYTES) >> 4);
           const uint32_t acc0 = kb != 0;
-          // B: [64 K][2 x 64 V] V-major, +2048 bytes per 16 K rows;
           // A: [128 rows][64 K] K-major, +32 bytes per 16 K columns
-          umma_f16(d0, ad, bd, IDESC, acc0);
-          if (two) umma_f16(d1, ad + (KBMAX * A_TILE_BYTES >> 4), bd, IDESC, acc0);
+          umma_f16(d0, ad, bd, idesc_w, acc0);
+          if (two) umma_f16(d1, ad + (KBMAX * A_TILE_BYTES >> 4), bd, idesc_w, acc0);
 #pragma unroll
           for (int k4 = 1; k4 < BK / 16; ++k4) {
-            umma_f16(d0, ad + (uint64_t)(k4 * 2), bd + (uint64_t)(k4 * 128), IDESC, 1u);
+            umma_f16(d0, ad + (uint64_t)(k4 * 2), bd + k4 * b_k16, idesc_w, 1u);
             if (two)
               umma_f16(d1, ad + (uint64_t)((KBMAX * A_TILE_BYTES >> 4) + k4 * 2),
-                       bd + (uint64_t)(k4 * 128), IDESC, 1u);
+                       bd + k4 * b_k16, idesc_w, 1u);
           }
           if (FOLD && kb == 0) {
             const uint64_t ld = l_desc0 + (uint64_t)((stage * LF_PART_BYTES) >> 4);
@@ -278,7 +300,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (two) umma_f16(d1, x_desc0 + (uint64_t)(LF_ONEHOT_BYTES >> 4), ld, IDESC, 1u);
           }
           umma_commit(&empty[stage]);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == nst) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         umma_commit(&tfull[buf]);
@@ -499,8 +521,17 @@ cudaError_t launch_score(const ScoreArgs& a, cudaStream_t s) {
   if (rows >= pair_rows_min()) return launch_score_pair(a, s);
   CUtensorMap tmA, tmB;
   if (!encode_2d_bf16(&tmA, a.Eg, (uint64_t)a.r_pad, (uint64_t)a.M_pad, BK, BM)) return cudaErrorInvalidValue;
-  if (!encode_2d_bf16(&tmB, a.W, (uint64_t)a.V, (uint64_t)a.r, 64, BK)) return cudaErrorInvalidValue;
+  // W's transpose, when the caller has it, is read as K-major tiles: an N-tile
+  // is then one contiguous run of 128 rows instead of r strided pieces
+  const bool kmaj = a.Wt != nullptr && a.r_pad % BK == 0;
+  if (kmaj) {
+    if (!encode_2d_bf16(&tmB, a.Wt, (uint64_t)a.r_pad, (uint64_t)a.V, BK, BN))
+      return cudaErrorInvalidValue;
+  } else if (!encode_2d_bf16(&tmB, a.W, (uint64_t)a.V, (uint64_t)a.r, 64, BK)) {
+    return cudaErrorInvalidValue;
+  }
   UmmaParams p;
+  p.b_kmajor = kmaj ? 1 : 0;
   p.M = rows;
   p.nsub = umma_nsub(rows);
   p.rows_per_cta = BM * p.nsub;

@@ -214,7 +214,11 @@ int32_t cadd_tree_grow(const cadd_desc* desc, const void* L, const int32_t* anch
  * The row pass already keeps every value above the row's CaDDTree threshold,
  * sorted, and writes the head of that list; only rows with fewer than top_k
  * such values are read again, by one more kernel that selects their top_k
- * exactly. Values order as IEEE floats except that -0.0 ranks below +0.0.
+ * exactly. That kernel runs beside the best-first growth on a second stream
+ * the library keeps per device (forked from and joined back into cuda_stream
+ * with events inside the call, so the call stays ordered on cuda_stream and
+ * can be captured in a graph; the stream is created by the first call in a
+ * context, which should come before any capture). Values order as IEEE floats except that -0.0 ranks below +0.0.
  * Same workspace as cadd_tree_grow. PCT_EINVAL when top_k is outside 1..32 or
  * top_tok is NULL. */
 int32_t cadd_tree_grow_topk(const cadd_desc* desc, const void* L, const int32_t* anchor,

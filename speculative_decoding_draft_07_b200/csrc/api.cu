@@ -1,6 +1,7 @@
 // C ABI of libpctree: argument checks, workspace planning and the launch
 // sequence of each call. Everything here runs on the host and only enqueues
 // work on the caller's stream; no call synchronises or allocates device memory.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -36,6 +37,62 @@ bool device_ok() {
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
   return major == 10;
 }
+
+// ---------------------------------------------------------------------------
+// auxiliary stream, per device and context
+namespace {
+typedef CUresult (*CurCtxFn)(CUcontext*);
+CurCtxFn cur_ctx_fn() {
+  static CurCtxFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CurCtxFn>(p);
+  }
+  return fn;
+}
+struct AuxSlot {
+  CUcontext ctx;   // the context the handles belong to
+  cudaStream_t s;
+  cudaEvent_t fork, join;
+};
+std::mutex g_aux_mu;          // the slots
+AuxSlot g_aux[64] = {};
+std::mutex g_aux_use[64];     // one call's fork ... join on a device
+}  // namespace
+
+int aux_stream(AuxStream* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PCT_ECUDA;
+  if (dev < 0 || dev >= 64) return PCT_EUNSUPPORTED;
+  CurCtxFn cur = cur_ctx_fn();
+  if (!cur) return PCT_ECUDA;
+  std::lock_guard<std::mutex> lk(g_aux_mu);
+  CUcontext ctx = nullptr;
+  if (cur(&ctx) != CUDA_SUCCESS) return PCT_ECUDA;
+  AuxSlot& a = g_aux[dev];
+  if (ctx == nullptr || a.s == nullptr || a.ctx != ctx) {
+    // a new context (first use, or the old one was reset): new handles; the
+    // old ones went with their context
+    AuxSlot n{};
+    if (cudaStreamCreateWithFlags(&n.s, cudaStreamNonBlocking) != cudaSuccess) return PCT_ECUDA;
+    if (cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming) != cudaSuccess)
+      return PCT_ECUDA;
+    if (cur(&ctx) != CUDA_SUCCESS || ctx == nullptr) return PCT_ECUDA;
+    n.ctx = ctx;
+    a = n;
+  }
+  out->s = a.s;
+  out->fork = a.fork;
+  out->join = a.join;
+  out->mu = &g_aux_use[dev];
+  return PCT_OK;
+}
+void aux_lock(const AuxStream& a) { static_cast<std::mutex*>(a.mu)->lock(); }
+void aux_unlock(const AuxStream& a) { static_cast<std::mutex*>(a.mu)->unlock(); }
 
 // ---------------------------------------------------------------------------
 // kernel trace

@@ -1320,22 +1320,23 @@ cudaError_t launch_cadd(const CaddParams& p_in, const void* L, const int32_t* an
                          status);
     if (e != cudaSuccess) return e;
   }
-  if (p.top_k > 0) {
-    // exact top_k of the rows with fewer than top_k values above their threshold
+  // exact top_k of the rows with fewer than top_k values above their threshold:
+  // it needs only the finishing kernel, like the best-first growth below, so it
+  // runs beside the growth on the library's second stream when there is one
+  auto launch_fill = [&](cudaStream_t fs) -> cudaError_t {
     // parts of about 8192 values (one or two loads per thread and read);
     // the grid covers the SMs twice and loops over however many items there are
     const int parts = std::max(1, std::min(kFillParts, (p.V + 8191) / 8192));
     const bool vec = p.dtype == PCT_BF16 && p.V % 8 == 0 && (reinterpret_cast<uintptr_t>(L) & 15u) == 0;
     const size_t items = (size_t)p.batch * p.D * parts;
     const unsigned grid = (unsigned)std::min<size_t>(items, (size_t)2 * num_sms());
-    TraceScope t(s, "cadd_topk_fill");
-    cudaError_t e = p.dtype == PCT_BF16
-        ? launch_pdl(cadd_topk_fill_kernel<__nv_bfloat16>, dim3(grid), dim3(kFillThreads), 0, s, 1,
+    TraceScope t(fs, "cadd_topk_fill");
+    return p.dtype == PCT_BF16
+        ? launch_pdl(cadd_topk_fill_kernel<__nv_bfloat16>, dim3(grid), dim3(kFillThreads), 0, fs, 1,
                      p, static_cast<const __nv_bfloat16*>(L), vec, parts)
-        : launch_pdl(cadd_topk_fill_kernel<float>, dim3(grid), dim3(kFillThreads), 0, s, 1, p,
+        : launch_pdl(cadd_topk_fill_kernel<float>, dim3(grid), dim3(kFillThreads), 0, fs, 1, p,
                      static_cast<const float*>(L), vec, parts);
-    if (e != cudaSuccess) return e;
-  }
+  };
   const size_t base = (size_t)(p.n_max + 1) * 8 + (size_t)p.n_max * 4 * 6;
   const size_t staged = base + (size_t)p.D * std::max(p.n_max - 1, 1) * 8;
   const bool stage = staged <= 160 * 1024;
@@ -1345,9 +1346,37 @@ cudaError_t launch_cadd(const CaddParams& p_in, const void* L, const int32_t* an
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  TraceScope t(s, "cadd_bestfirst");
-  return launch_pdl(kern, dim3(p.batch), dim3(32), smem, s, 1, p, anchor, ctx, cand_cnt, cand_q,
-                    cand_tok, tok, parent, depth, score, count, phi, status);
+  AuxStream ax{};
+  const bool fork = p.top_k > 0 && aux_stream(&ax) == PCT_OK;
+  if (p.top_k > 0 && !fork) {
+    cudaError_t e = launch_fill(s);
+    if (e != cudaSuccess) return e;
+  }
+  if (fork) aux_lock(ax);
+  cudaError_t fe = cudaSuccess;
+  if (fork) {
+    fe = cudaEventRecord(ax.fork, s);
+    if (fe == cudaSuccess) fe = cudaStreamWaitEvent(ax.s, ax.fork, 0);
+    if (fe == cudaSuccess) fe = launch_fill(ax.s);
+    if (fe == cudaSuccess) fe = cudaEventRecord(ax.join, ax.s);
+    if (fe != cudaSuccess) {
+      aux_unlock(ax);
+      return fe;
+    }
+  }
+  cudaError_t e;
+  {
+    TraceScope t(s, "cadd_bestfirst");
+    e = launch_pdl(kern, dim3(p.batch), dim3(32), smem, s, 1, p, anchor, ctx, cand_cnt, cand_q,
+                   cand_tok, tok, parent, depth, score, count, phi, status);
+  }
+  if (fork) {
+    // the caller's stream goes on only after the selection too
+    const cudaError_t je = cudaStreamWaitEvent(s, ax.join, 0);
+    aux_unlock(ax);
+    if (e == cudaSuccess) e = je;
+  }
+  return e;
 }
 
 }  // namespace pct

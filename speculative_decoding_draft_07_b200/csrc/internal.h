@@ -23,6 +23,23 @@ struct TraceScope {
 int num_sms();          // SMs of the current device (cached per device)
 bool device_ok();       // compute capability 10.x
 
+// ---- auxiliary stream (api.cu) -----------------------------------------------
+// A second stream of the current device and context (created on first use,
+// kept for the process) with two events, for work inside one call that does
+// not depend on the caller's stream's next kernel: record `fork` on the
+// caller's stream, make `s` wait for it, launch there, record `join` on `s`,
+// make the caller's stream wait for it, all under `mu` (calls from several
+// host threads share the stream and events). A graph capture of the caller's
+// stream takes the forked work in as a branch.
+struct AuxStream {
+  cudaStream_t s;
+  cudaEvent_t fork, join;
+  void* mu;   // std::mutex*
+};
+int aux_stream(AuxStream* out);   // PCT_OK or an error code
+void aux_lock(const AuxStream& a);
+void aux_unlock(const AuxStream& a);
+
 // ---- verify.cu --------------------------------------------------------------
 cudaError_t launch_ancestor_mask(int batch, int n_stride, const int32_t* parent,
                                  const int32_t* count, uint32_t* mask, int32_t* status,

@@ -265,3 +265,84 @@ def test_seeded_build_extreme_k(k, beam, N):
     torch.cuda.synchronize()
     _same_tree(plain, seeded)
     _build_and_compare(L, anchor, E, W, k, beam, N, label=f"seeded k={k}", seeds=seeds)
+
+
+def test_one_pass_round_in_a_cuda_graph():
+    """cadd_tree_grow_topk forks its exact selection to the library's second
+    stream and joins it back: captured in a graph with the seeded build, the
+    replay gives the eager results bit for bit (new inputs copied in between)."""
+    import ctypes
+    batch, D, V, r, k = 17, 5, 4096, 64, 8
+    L, anchor, E, W = _problem(batch, D, V, r, seed=71)
+    L2, _, _, _ = _problem(batch, D, V, r, seed=72)
+    Ld, ad, Ed, Wd = L.to(DEV), anchor.to(DEV), E.to(DEV), W.to(DEV)
+    ctx = torch.full((batch,), 4096, dtype=torch.int64, device=DEV)
+    Wt = pct.markov_transpose(Wd)
+    top = torch.empty((batch, D, k), dtype=torch.int32, device=DEV)
+    cdesc = pct.cadd_desc(batch, D, V, 64, pct.PCT_BF16, *COST.values())
+    ws_c = torch.empty(int(pct.lib().cadd_tree_grow_workspace(ctypes.byref(cdesc))), dtype=torch.uint8,
+                       device=DEV)
+    bdesc = pct.build_desc(batch, D, V, r, k, 16, 64, pct.PCT_BF16, pct.PCT_BF16)
+    ws_t = torch.empty(pct.pct_tree_build_workspace(bdesc), dtype=torch.uint8, device=DEV)
+    cad = pct.cadd_tree_grow(Ld, ad, ctx, 64, **COST, workspace=ws_c, top_tok=top)
+    tree = pct.pct_tree_build(Ld, ad, Ed, Wd, k, 16, 64, workspace=ws_t, seeds=top, Wt=Wt)
+    torch.cuda.synchronize()
+
+    def eager(Lx):
+        t2 = torch.empty_like(top)
+        c = pct.cadd_tree_grow(Lx.to(DEV), ad, ctx, 64, **COST, top_tok=t2)
+        b = pct.pct_tree_build(Lx.to(DEV), ad, Ed, Wd, k, 16, 64, seeds=t2, Wt=Wt)
+        torch.cuda.synchronize()
+        return c, b, host(t2)
+
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            pct.cadd_tree_grow(Ld, ad, ctx, 64, **COST, out=cad, workspace=ws_c, top_tok=top,
+                               stream=s)
+            pct.pct_tree_build(Ld, ad, Ed, Wd, k, 16, 64, out=tree, workspace=ws_t, seeds=top,
+                               Wt=Wt, stream=s)
+    for Lx in (L2, L):
+        Ld.copy_(Lx.to(DEV))
+        g.replay()
+        torch.cuda.synchronize()
+        c, b, t2 = eager(Lx)
+        _same_tree(c, cad, phi=True)
+        _same_tree(b, tree)
+        np.testing.assert_array_equal(host(top), t2)
+
+
+def test_grow_topk_from_two_host_threads():
+    """Two host threads, each on its own stream and workspace, call
+    cadd_tree_grow_topk at the same time (the second stream and its events are
+    shared under a lock): every result equals the single-threaded one."""
+    import threading
+    batch, D, V = 6, 4, 20000
+    Ls = [_sharp_logits(batch, D, V, seed=80 + i, sigma=0.05 if i % 2 else 2.0,
+                        peak=(0.0, 0.5 if i % 2 else 6.0)) for i in range(2)]
+    refs = [oracle.row_topk(f64(x), 8) for x in Ls]
+    a = torch.arange(batch, dtype=torch.int32, device=DEV)
+    c = torch.full((batch,), 4096, dtype=torch.int64, device=DEV)
+    errors = []
+    torch.cuda.synchronize()
+
+    def work(i):
+        try:
+            st = torch.cuda.Stream()
+            with torch.cuda.stream(st):
+                Ld = Ls[i].to(DEV)
+                for _ in range(20):
+                    top = torch.full((batch, D, 8), -7, dtype=torch.int32, device=DEV)
+                    pct.cadd_tree_grow(Ld, a, c, 32, **COST, top_tok=top, stream=st)
+                    st.synchronize()
+                    np.testing.assert_array_equal(host(top), refs[i])
+        except Exception as e:  # noqa: BLE001 - reported below
+            errors.append(e)
+
+    th = [threading.Thread(target=work, args=(i,)) for i in range(2)]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join()
+    assert not errors, errors

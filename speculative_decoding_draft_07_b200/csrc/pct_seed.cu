@@ -1,15 +1,22 @@
 // Seed columns for the PCTree scoring gate: for every (request, depth) row of
-// the drafter logits L_d, a handful of columns with large L_d.
+// the drafter logits L_d, a handful of columns with large L_d, with L_d and the
+// W column at each.
 //
 // PCTree article (qiita), section on the tree that replaces the chain draft:
 // z_d(p) = L_d + Markov(p) for every parent of a depth, so the columns where
 // L_d is largest are the natural place to look for each parent's top-k. The
-// columns found here only seed a lower bound (the bound is exact whatever
-// columns are chosen), so the search need not be exact either: each thread
-// keeps the best 8-column group of its strided share of a slice of the row,
-// the column of that group's maximum is recovered with one reload, each block
-// keeps the ks best of its 256 thread winners and the row's last block merges
-// the slices' picks. One streaming pass over L (HBM bound).
+// columns only seed a lower bound (the bound is exact whatever columns are
+// chosen), so the search need not be exact either. Three kernels:
+//  * drafter_topk_kernel (pct_tree_build): one streaming pass over L (HBM
+//    bound); each thread keeps the best 8-column group of its strided share of
+//    a slice of the row, the column of that group's maximum is recovered with
+//    one reload, each block keeps the ks best of its 256 thread winners and the
+//    row's last block merges the slices' picks and gathers their W columns;
+//  * seed_columns_kernel (pct_tree_build_seeded): the columns are given (for
+//    example the CaDDTree row pass's top-k of the same L); it drops invalid and
+//    repeated entries and gathers L and the W columns, from W's transpose when
+//    the caller has it (one contiguous row per column);
+//  * markov_transpose_kernel: that transpose, once per model.
 #include <algorithm>
 #include <climits>
 

@@ -35,6 +35,9 @@ def test_algorithmic_work_matches_closed_forms():
     assert abs(w["verify_argmax_walk"]["bytes"] / 1e9 - 4.979) < 1e-3
     assert w["cadd_rowpass"]["bytes"] == 64 * 15 * V * 2         # 291.7 MB
     assert abs(w["cadd_rowpass"]["bytes"] / 1e6 - 291.7) < 0.05
+    # seeds from given columns: k rows of W's transpose (r bf16 values) read
+    # and copied per logits row
+    assert w["seed_columns"]["bytes"] == 64 * 15 * 8 * r * 2 * 2   # 7.9 MB
 
 
 def test_pair_kernel_row_split():

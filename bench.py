@@ -606,6 +606,20 @@ def warm_cold_ms(fn, dev, warm_runs, cold_runs, flush):
     return warm, tot / cold_runs
 
 
+def traced_kernels_us(fn, runs, dev):
+    """Per-kernel device time of fn with L2 warm: two events around every launch
+    on its stream (the library's trace), microseconds and launches per run."""
+    import speculative_decoding_draft_07_b200 as pct
+    pct.trace_enable(True)
+    pct.trace_reset()
+    for _ in range(runs):
+        fn()
+    torch.cuda.synchronize(dev)
+    t = pct.trace_read()
+    pct.trace_enable(False)
+    return {n: {"launches": c / runs, "us": round(ms * 1e3 / runs, 2)} for n, (c, ms) in t.items()}
+
+
 def oracle_legs(fn, batch):
     """The oracle on one request on one thread, and on min(batch, cores) requests
     one per thread on all host cores; rates scaled to the configuration's batch."""
@@ -661,7 +675,8 @@ def config_results(dev, pk, quick=False):
              "tflops_cold": flop / cold / 1e9, "frac_bf16_burst_cold": flop / cold / 1e9 / tc,
              "stream_gbs_cold": wbytes / cold / 1e6, "frac_hbm_cold": wbytes / cold / 1e6 / hbm,
              "stream_gbs_warm": wbytes / warm / 1e6,
-             "bound": "tensor" if name == "long_block" else ("hbm" if name != "tiny" else "launch")}
+             "bound": "tensor" if name == "long_block" else ("hbm" if name != "tiny" else "launch"),
+             "kernels_warm": traced_kernels_us(fn, 10, dev)}
         if not quick:
             Lh, Eh, Wh, ah = L.cpu(), f64(E), f64(Wm), a.cpu().numpy()
             e["oracle"] = oracle_legs(lambda b: oracle.pct_tree_build(
@@ -678,7 +693,8 @@ def config_results(dev, pk, quick=False):
         e = {"workload": f"caddtree_l{ell}", "requests": C.batch, "rounds_per_s_warm": 1e3 / warm,
              "rounds_per_s_cold": 1e3 / cold, "ms_per_round_cold": cold,
              "gbs_cold": nbytes / cold / 1e6, "frac_hbm_cold": nbytes / cold / 1e6 / hbm,
-             "mean_nodes": float(out.count.float().mean()), "bound": "hbm"}
+             "mean_nodes": float(out.count.float().mean()), "bound": "hbm",
+             "kernels_warm": traced_kernels_us(fn, 10, dev)}
         if not quick:
             Lh, ah, ch = L.cpu(), a.cpu().numpy(), ctx.cpu().numpy()
             e["oracle"] = oracle_legs(lambda b: oracle.cadd_tree_grow(
